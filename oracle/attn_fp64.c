@@ -1,0 +1,155 @@
+/*
+ * Oracle for exact attention, plain fp64 on the CPU.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline leg of bench.py may load this library.  It shares no code,
+ * header, table or helper with the CUDA path.
+ *
+ * What it computes is the plain definition of attention,
+ *     out_i = softmax(scale * q_i . K^T) V ,
+ * from "Lesson 8: Context Parallelism", section 1 (the attention formula
+ * that every query must see every key).  Blockwise ring attention with the
+ * online-softmax merge reaches exactly this value (same lesson, section 3,
+ * and "Sequence parallelism and ring attention", FAQ on online softmax), so
+ * the oracle is that definition written out, with no blocking, no online
+ * rescaling and no chunk order:
+ *
+ *   for each requested query row (b, h, i):
+ *     J    = allowed keys: j < kv_len[b] (when lengths are given) and, when
+ *            causal, kpos[j] <= qpos[i] ("Lesson 8", section 4: query i sees
+ *            keys j <= i)
+ *     s_j  = scale * sum_d q[b,i,h,d] * k[b,j,g,d]      with g = h / (Hq/Hkv)
+ *     m    = max_j s_j ,  Z = sum_j exp(s_j - m)
+ *     out  = sum_j exp(s_j - m) v[b,j,g,:] / Z ,   lse = m + ln Z
+ *
+ * The whole score row is materialised before it is normalised.  Inputs are
+ * float32 arrays holding the exact values of the device inputs (bf16 values
+ * are exact in float32); every operation is done in double.
+ *
+ * Layouts (row-major, last index fastest):
+ *   q   [B, Sq , Hq , D]      k, v [B, Skv, Hkv, D]
+ *   qpos[Sq]  (global position of each query row; NULL means the row index)
+ *   kpos[Skv] (global position of each key row;   NULL means the row index)
+ *   kv_len[B] (keys j >= kv_len[b] are not allowed; NULL means all Skv)
+ *   rows [nrows][3] = (b, h, i)
+ *   out  [nrows][D]  lse [nrows]
+ * A row with no allowed key gets out = 0 and lse = -inf.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <sched.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <unistd.h>
+
+typedef struct {
+  const float *q, *k, *v;
+  int B, Sq, Skv, Hq, Hkv, D;
+  const int64_t *qpos, *kpos;
+  int causal;
+  const int64_t *kv_len;
+  double scale;
+  const int32_t *rows;
+  int64_t r0, r1;
+  double *out, *lse;
+  int err;
+} job_t;
+
+static void one_row(const job_t *J, int64_t r, double *s /* [Skv] */) {
+  const int b = J->rows[3 * r + 0], h = J->rows[3 * r + 1], i = J->rows[3 * r + 2];
+  const int G = J->Hq / J->Hkv;
+  const int g = h / G;
+  const int D = J->D;
+  const float *qi = J->q + (((int64_t)b * J->Sq + i) * J->Hq + h) * D;
+  const int64_t qp = J->qpos ? J->qpos[i] : i;
+  const int64_t nkeys = J->kv_len ? J->kv_len[b] : J->Skv;
+  double *o = J->out + r * D;
+  for (int d = 0; d < D; ++d) o[d] = 0.0;
+
+  /* 1. materialise the score row over the allowed keys */
+  double m = -INFINITY;
+  int any = 0;
+  for (int64_t j = 0; j < J->Skv; ++j) {
+    const int64_t kp = J->kpos ? J->kpos[j] : j;
+    const int allowed = (j < nkeys) && (!J->causal || kp <= qp);
+    if (!allowed) { s[j] = -INFINITY; continue; }
+    const float *kj = J->k + (((int64_t)b * J->Skv + j) * J->Hkv + g) * D;
+    double acc = 0.0;
+    for (int d = 0; d < D; ++d) acc += (double)qi[d] * (double)kj[d];
+    s[j] = J->scale * acc;
+    if (s[j] > m) m = s[j];
+    any = 1;
+  }
+  if (!any) { J->lse[r] = -INFINITY; return; }
+
+  /* 2. exponentiate against the row max and sum */
+  double Z = 0.0;
+  for (int64_t j = 0; j < J->Skv; ++j) {
+    if (s[j] == -INFINITY) { s[j] = 0.0; continue; }
+    s[j] = exp(s[j] - m);
+    Z += s[j];
+  }
+  /* 3. weighted sum of the value rows, then normalise */
+  for (int64_t j = 0; j < J->Skv; ++j) {
+    if (s[j] == 0.0) continue;
+    const float *vj = J->v + (((int64_t)b * J->Skv + j) * J->Hkv + g) * D;
+    const double w = s[j];
+    for (int d = 0; d < D; ++d) o[d] += w * (double)vj[d];
+  }
+  for (int d = 0; d < D; ++d) o[d] /= Z;
+  J->lse[r] = m + log(Z);
+}
+
+static void *worker(void *arg) {
+  job_t *J = (job_t *)arg;
+  double *s = (double *)malloc(sizeof(double) * (size_t)(J->Skv > 0 ? J->Skv : 1));
+  if (!s) { J->err = 1; return NULL; }
+  for (int64_t r = J->r0; r < J->r1; ++r) one_row(J, r, s);
+  free(s);
+  return NULL;
+}
+
+/* Number of host cores this process may run on. */
+int oracle_cores(void) {
+  cpu_set_t set;
+  if (sched_getaffinity(0, sizeof(set), &set) == 0) return CPU_COUNT(&set);
+  long n = sysconf(_SC_NPROCESSORS_ONLN);
+  return n > 0 ? (int)n : 1;
+}
+
+/* Returns 0 on success, nonzero on a bad argument or an allocation failure. */
+int oracle_attn_rows(const float *q, const float *k, const float *v,
+                     int B, int Sq, int Skv, int Hq, int Hkv, int D,
+                     const int64_t *qpos, const int64_t *kpos, int causal,
+                     const int64_t *kv_len, double scale,
+                     const int32_t *rows, int64_t nrows,
+                     double *out, double *lse, int nthreads) {
+  if (B <= 0 || Sq <= 0 || Skv < 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return 1;
+  if (Hq % Hkv != 0) return 1;
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0 || i >= Sq) return 1;
+  }
+  if (nthreads <= 0) nthreads = oracle_cores();
+  if (nthreads > nrows) nthreads = nrows > 0 ? (int)nrows : 1;
+  job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
+  pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+  if (!jobs || !th) { free(jobs); free(th); return 2; }
+  int err = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    job_t *J = &jobs[t];
+    J->q = q; J->k = k; J->v = v;
+    J->B = B; J->Sq = Sq; J->Skv = Skv; J->Hq = Hq; J->Hkv = Hkv; J->D = D;
+    J->qpos = qpos; J->kpos = kpos; J->causal = causal; J->kv_len = kv_len;
+    J->scale = scale; J->rows = rows;
+    J->r0 = nrows * t / nthreads; J->r1 = nrows * (t + 1) / nthreads;
+    J->out = out; J->lse = lse;
+    if (pthread_create(&th[t], NULL, worker, J) != 0) { J->r1 = J->r0; err = 3; th[t] = 0; }
+  }
+  for (int t = 0; t < nthreads; ++t) {
+    if (th[t]) pthread_join(th[t], NULL);
+    if (jobs[t].err) err = 2;
+  }
+  free(jobs); free(th);
+  return err;
+}
