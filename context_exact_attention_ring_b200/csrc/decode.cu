@@ -1,0 +1,402 @@
+// Split-KV single-token decode ("NVIDIA unveils Helix Parallelism", Phase 1:
+// the KV cache sharded along the sequence; each shard yields a partial result
+// that is merged afterwards).
+//
+// Work unit = (chunk p, batch b, kv head g, sub-split s): RPS consecutive rows
+// of one chunk.  A persistent grid (one CTA per SM) walks the units in chunk
+// order, so the always-full early chunks come first and the ragged tails of
+// the sequences last.  Per CTA:
+//   warp 0      TMA producer: 64-row K and V boxes into a 5-stage ring of
+//               shared memory (bounded waits on the stage barriers);
+//   warps 1..8  consumers: 32 groups of 8 lanes, each group owns two rows of a
+//               stage; a lane holds 16 of the 128 dims of the G query heads of
+//               the kv head (scaled by scale*log2 e), computes partial dot
+//               products, reduces them inside its group with shuffles, and
+//               folds the rows into a running (m, l, O) -- the online-softmax
+//               update of "Lesson 8: Context Parallelism", section 3 -- keeping
+//               a stale max until a score exceeds it by 2^8 (exact: the same
+//               base scales l and O).
+// At the end of a unit the 32 group states are folded (shuffles, then shared
+// memory).  A chunk covered by one sub-split writes its partial directly;
+// otherwise every sub-split writes to the workspace and the last CTA to
+// arrive (atomic counter, reset by that CTA) folds them into the chunk's
+// partial.  The kernel is HBM-bound: each valid K/V byte is read once.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace ra {
+
+namespace dec {
+constexpr int D = 128;
+constexpr int ROWS = 64;                    // rows per stage
+constexpr int NST = 5;                      // stages
+constexpr int RPS = 4096;                   // rows per sub-split
+constexpr int STAGE_BYTES = 2 * ROWS * D * 2;
+constexpr int NCW = 8;                      // consumer warps
+constexpr int THREADS = 32 * (1 + NCW);
+constexpr float LAZY = 8.f;                 // log2 of the largest tolerated growth before rescaling
+}  // namespace dec
+
+struct DecGeom {
+  int Cd;      // rows per chunk
+  int nsub;    // sub-splits per chunk
+  int units;
+};
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float* f) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(u[i] << 16);
+    f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+  }
+}
+
+template <int G>
+struct DecSmem {
+  alignas(1024) uint8_t stage[dec::NST][dec::STAGE_BYTES];
+  float wpart[dec::NCW][G][dec::D];
+  float wm[dec::NCW][G];
+  float wl[dec::NCW][G];
+  alignas(8) uint64_t full[dec::NST];
+  alignas(8) uint64_t empty[dec::NST];
+  int is_last;
+  int abort_flag;
+};
+
+template <int G>
+__global__ void __launch_bounds__(dec::THREADS, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DecodeArgs a,
+                  DecGeom geo) {
+  using namespace dec;
+  extern __shared__ uint8_t smem_raw[];
+  DecSmem<G>& sm = *reinterpret_cast<DecSmem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(smem_u32(&sm.full[s]), 1);
+      mbar_init(smem_u32(&sm.empty[s]), NCW);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint64_t pol = l2_policy_evict_first();
+      uint32_t cnt = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < geo.units && ok; u += gridDim.x) {
+        int t = u;
+        const int sub = t % geo.nsub; t /= geo.nsub;
+        const int g = t % a.Hkv; t /= a.Hkv;
+        const int b = t % a.B;
+        const int p = t / a.B;
+        const int len = min(max(a.seqlens[b], 0), a.Smax);
+        const int r0 = p * geo.Cd + sub * RPS;
+        const int r1 = min(r0 + RPS, min(len, (p + 1) * geo.Cd));
+        for (int row = r0; row < r1; row += ROWS) {
+          const int s = cnt % NST;
+          const uint32_t ph = (cnt / NST) & 1u;
+          if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag, kWaitDecodeEmpty, a.err)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&sm.full[s]);
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t dst = smem_u32(sm.stage[s]);
+          tma_load_4d(dst, &tmK, fb, 0, g, row, b, pol);
+          tma_load_4d(dst + ROWS * D * 2, &tmV, fb, 0, g, row, b, pol);
+          ++cnt;
+        }
+      }
+      // do not leave while copies are still landing in shared memory
+      for (uint32_t c = (cnt > (uint32_t)NST ? cnt - NST : 0); c < cnt; ++c) {
+        const int s = c % NST;
+        mbar_wait(smem_u32(&sm.full[s]), (c / NST) & 1u, nullptr, kWaitTeardown, a.err);
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int cw = warp - 1;                 // consumer warp 0..7
+  const int ctid = threadIdx.x - 32;       // 0..255
+  const int grp = lane >> 3, j = lane & 7;
+  const int gidx = cw * 4 + grp;           // row group 0..31 -> rows gidx, gidx + 32 of a stage
+  const float qscale = a.scale * 1.4426950408889634f;
+  uint32_t cnt = 0;
+  const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(a.q);
+
+  for (int u = blockIdx.x; u < geo.units; u += gridDim.x) {
+    int t = u;
+    const int sub = t % geo.nsub; t /= geo.nsub;
+    const int g = t % a.Hkv; t /= a.Hkv;
+    const int b = t % a.B;
+    const int p = t / a.B;
+    const int len = min(max(a.seqlens[b], 0), a.Smax);
+    const int c0 = p * geo.Cd;
+    const int nvalid_chunk = max(0, min(len - c0, geo.Cd));
+    const int n_live = (nvalid_chunk + RPS - 1) / RPS;
+    const int r0 = c0 + sub * RPS;
+    const int r1 = min(r0 + RPS, c0 + nvalid_chunk);
+
+    if (nvalid_chunk == 0) {
+      if (sub == 0) {
+        for (int e = ctid; e < G * D; e += 256) {
+          const int h = e / D, d = e - h * D;
+          a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = 0.f;
+        }
+        if (ctid < G) a.part_lse[(size_t)(b * a.Hq + g * G + ctid) * a.P + p] = -CUDART_INF_F;
+      }
+      continue;
+    }
+    if (r0 >= r1) continue;
+
+    // this lane's slice of the G query heads: dims [8j, 8j+8) and [64+8j, 64+8j+8)
+    float qf[G][16];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const __nv_bfloat16* qh = qb + ((size_t)b * a.Hq + g * G + h) * D;
+      const uint4 w0 = *reinterpret_cast<const uint4*>(qh + 8 * j);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(qh + 64 + 8 * j);
+      bf16x8_to_f32(w0, qf[h]);
+      bf16x8_to_f32(w1, qf[h] + 8);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) qf[h][i] *= qscale;
+    }
+    float m[G], l[G], o[G][16];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      m[h] = -CUDART_INF_F;
+      l[h] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) o[h][i] = 0.f;
+    }
+
+    bool ok = true;
+    for (int row = r0; row < r1 && ok; row += ROWS) {
+      const int s = cnt % NST;
+      const uint32_t ph = (cnt / NST) & 1u;
+      if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, kWaitDecodeFull, a.err)) { ok = false; break; }
+      const uint8_t* Ks = sm.stage[s];
+      const uint8_t* Vs = Ks + ROWS * D * 2;
+      const bool vA = row + gidx < r1, vB = row + gidx + 32 < r1;
+      float kA[16], kB[16];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + gidx * 256 + 16 * j), kA);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + gidx * 256 + 128 + 16 * j), kA + 8);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + (gidx + 32) * 256 + 16 * j), kB);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + (gidx + 32) * 256 + 128 + 16 * j), kB + 8);
+      float sA[G], sB[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float x = 0.f, y = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          x = fmaf(qf[h][i], kA[i], x);
+          y = fmaf(qf[h][i], kB[i], y);
+        }
+        sA[h] = x;
+        sB[h] = y;
+      }
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          sA[h] += __shfl_xor_sync(0xffffffffu, sA[h], off);
+          sB[h] += __shfl_xor_sync(0xffffffffu, sB[h], off);
+        }
+      }
+      float vAf[16], vBf[16];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + gidx * 256 + 16 * j), vAf);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + gidx * 256 + 128 + 16 * j), vAf + 8);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + (gidx + 32) * 256 + 16 * j), vBf);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + (gidx + 32) * 256 + 128 + 16 * j), vBf + 8);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));   // this warp is done with the stage
+      ++cnt;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (!vA) sA[h] = -CUDART_INF_F;
+        if (!vB) sB[h] = -CUDART_INF_F;
+        const float smax = fmaxf(sA[h], sB[h]);
+        if (smax > m[h] + LAZY) {
+          const float f = (m[h] == -CUDART_INF_F) ? 0.f : ex2(m[h] - smax);
+          l[h] *= f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[h][i] *= f;
+          m[h] = smax;
+        }
+        const bool live = m[h] != -CUDART_INF_F;
+        const float pA = (live && vA) ? ex2(sA[h] - m[h]) : 0.f;
+        const float pB = (live && vB) ? ex2(sB[h] - m[h]) : 0.f;
+        l[h] += pA + pB;
+        if (vA) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[h][i] = fmaf(pA, vAf[i], o[h][i]);
+        }
+        if (vB) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[h][i] = fmaf(pB, vBf[i], o[h][i]);
+        }
+      }
+    }
+    // (after an expired wait the unit still runs through every named barrier
+    // below, so that all consumer warps leave the loop together)
+
+    // fold the 4 groups of this warp (lanes with equal j hold the same dims)
+#pragma unroll
+    for (int off = 8; off < 32; off <<= 1) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
+        const float mc = fmaxf(m[h], mo);
+        const float f = (m[h] == -CUDART_INF_F) ? 0.f : ex2(m[h] - mc);
+        l[h] *= f;
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          o[h][i] *= f;
+          o[h][i] += __shfl_xor_sync(0xffffffffu, o[h][i], off);
+        }
+        m[h] = mc;
+      }
+    }
+    if (grp == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          sm.wpart[cw][h][8 * j + i] = o[h][i];
+          sm.wpart[cw][h][64 + 8 * j + i] = o[h][8 + i];
+        }
+        if (j == 0) {
+          sm.wm[cw][h] = m[h];
+          sm.wl[cw][h] = l[h];
+        }
+      }
+    }
+    named_bar_sync(1, 256);
+
+    // fold the 8 warps: thread -> (head, dim) pairs; natural-log lse at the end
+    float* ws_unit = a.ws_part + ((((size_t)(b * a.Hkv + g) * a.P + p) * geo.nsub + sub) * G) * (D + 1);
+    for (int e = ctid; e < G * D; e += 256) {
+      const int h = e / D, d = e - h * D;
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, sm.wm[w][h]);
+      float L = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const float f = (sm.wm[w][h] == -CUDART_INF_F) ? 0.f : ex2(sm.wm[w][h] - mx);
+        L = fmaf(sm.wl[w][h], f, L);
+        acc = fmaf(sm.wpart[w][h][d], f, acc);
+      }
+      const float od = acc / L;
+      const float lse = (mx + log2f(L)) * 0.6931471805599453f;
+      if (n_live == 1) {
+        a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = od;
+        if (d == 0) a.part_lse[(size_t)(b * a.Hq + g * G + h) * a.P + p] = lse;
+      } else {
+        ws_unit[h * (D + 1) + d] = od;
+        if (d == 0) ws_unit[h * (D + 1) + D] = lse;
+      }
+    }
+    if (n_live > 1) {
+      __threadfence();
+      named_bar_sync(1, 256);
+      if (ctid == 0) {
+        unsigned int* ctr = a.ws_count + (size_t)(b * a.Hkv + g) * a.P + p;
+        const unsigned int old = atomicAdd(ctr, 1u);
+        const int last = (old == (unsigned int)(n_live - 1));
+        if (last) atomicExch(ctr, 0u);       // leave the counter at zero for the next call
+        sm.is_last = last;
+      }
+      named_bar_sync(1, 256);
+      if (sm.is_last) {
+        __threadfence();
+        const float* ws_chunk = a.ws_part + (((size_t)(b * a.Hkv + g) * a.P + p) * geo.nsub) * G * (D + 1);
+        for (int e = ctid; e < G * D; e += 256) {
+          const int h = e / D, d = e - h * D;
+          float mx = -CUDART_INF_F;
+          for (int s2 = 0; s2 < n_live; ++s2) mx = fmaxf(mx, __ldcg(ws_chunk + (s2 * G + h) * (D + 1) + D));
+          float L = 0.f, acc = 0.f;
+          for (int s2 = 0; s2 < n_live; ++s2) {
+            const float* r = ws_chunk + (s2 * G + h) * (D + 1);
+            const float w = expf(__ldcg(r + D) - mx);
+            L += w;
+            acc = fmaf(w, __ldcg(r + d), acc);
+          }
+          a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = acc / L;
+          if (d == 0) a.part_lse[(size_t)(b * a.Hq + g * G + h) * a.P + p] = mx + logf(L);
+        }
+      }
+    }
+    // shared fold buffers are free again; leave together if any wait expired
+    if (named_bar_any(1, 256, !ok || *abort_flag)) break;
+  }
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || P < 1 || Smax < P || D < 1 || Hq % Hkv) return 0;
+  const int G = Hq / Hkv;
+  const int Cd = Smax / P;
+  const int nsub = (Cd + dec::RPS - 1) / dec::RPS;
+  const size_t chunks = (size_t)B * Hkv * P;
+  size_t part = chunks * nsub * G * (D + 1) * sizeof(float);
+  part = (part + 255) & ~size_t(255);
+  return part + ((chunks * sizeof(unsigned int) + 255) & ~size_t(255));
+}
+
+void decode_workspace_split(void* ws, int B, int Hq, int Hkv, int Smax, int D, int P, float** part,
+                            unsigned int** count) {
+  const int G = Hq / Hkv;
+  const int Cd = Smax / P;
+  const int nsub = (Cd + dec::RPS - 1) / dec::RPS;
+  const size_t chunks = (size_t)B * Hkv * P;
+  size_t bytes = chunks * nsub * G * (D + 1) * sizeof(float);
+  bytes = (bytes + 255) & ~size_t(255);
+  *part = reinterpret_cast<float*>(ws);
+  *count = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) + bytes);
+}
+
+template <int G>
+static cudaError_t launch_decode_g(const DecodeArgs& a, cudaStream_t st) {
+  CUtensorMap tk, tv;
+  if (!make_tmap_bhsd(&tk, a.k, a.B, a.Smax, a.Hkv, a.D, dec::D, dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_bhsd(&tv, a.v, a.B, a.Smax, a.Hkv, a.D, dec::D, dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  DecGeom geo;
+  geo.Cd = a.Smax / a.P;
+  geo.nsub = (geo.Cd + dec::RPS - 1) / dec::RPS;
+  const long long units = (long long)a.P * a.B * a.Hkv * geo.nsub;
+  if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+  geo.units = (int)units;
+  const size_t smem = sizeof(DecSmem<G>) + 1024;
+  auto kern = decode_kernel<G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = num_sms();
+  kern<<<grid, dec::THREADS, smem, st>>>(tk, tv, a, geo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_partial(const DecodeArgs& a, cudaStream_t st) {
+  const int G = a.Hq / a.Hkv;
+  switch (G) {
+    case 1: return launch_decode_g<1>(a, st);
+    case 2: return launch_decode_g<2>(a, st);
+    case 4: return launch_decode_g<4>(a, st);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace ra

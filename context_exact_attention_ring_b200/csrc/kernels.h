@@ -1,0 +1,76 @@
+// Host-side launchers of the library's kernels (internal; the public ABI is
+// include/ring_attn.h).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "ring_sched.h"
+
+namespace ra {
+
+// CUDA-core ring attention (ring or step mode, fp32 or bf16 inputs).
+cudaError_t launch_attn_simt(const Plan& p, bool bf16, const void* q, const void* k, const void* v, void* out,
+                             float* lse, float* m, float* l, float* O, float scale, cudaStream_t st);
+
+// Tensor-core (tcgen05) ring attention, bf16 in / fp32 accumulate.
+struct TcArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;            // ring mode: [B,Sq,Hq,D] bf16
+  float* lse;           // ring mode: [B,Hq,Sq]
+  float* m;             // step mode state
+  float* l;
+  float* O;
+  unsigned long long* counters;  // optional [2 + P]
+  float scale;
+  unsigned int* err;             // device error word
+};
+cudaError_t launch_attn_tc(const Plan& p, const TcArgs& a, cudaStream_t st);
+
+cudaError_t launch_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D, cudaStream_t st);
+cudaError_t launch_state_finalize(const float* m, const float* l, const float* O, void* out, float* lse, int B,
+                                  int Hq, int S, int D, bool bf16, cudaStream_t st);
+cudaError_t launch_merge(const float* part, const float* plse, void* out, float* out_lse, int B, int Hq, int P,
+                         int D, bool bf16, cudaStream_t st);
+
+// Split-KV decode.
+struct DecodeArgs {
+  const void* q;        // [B,Hq,D] bf16
+  const void* k;        // [B,Smax,Hkv,D] bf16
+  const void* v;
+  const int32_t* seqlens;
+  float* partials;      // [B,Hq,P,D]
+  float* part_lse;      // [B,Hq,P]
+  float* ws_part;       // sub-split results
+  unsigned int* ws_count;  // per-chunk arrival counters (zero between calls)
+  int B, Hq, Hkv, Smax, D, P;
+  float scale;
+  unsigned int* err;    // device error word
+};
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P);
+void decode_workspace_split(void* ws, int B, int Hq, int Hkv, int Smax, int D, int P, float** part,
+                            unsigned int** count);
+cudaError_t launch_decode_partial(const DecodeArgs& a, cudaStream_t st);
+
+// Driver entry point for building TMA descriptors (resolved at run time, so
+// the library does not link libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+// 4-D bf16 tensor map over a [B, rows, heads, D] tensor with box
+// {box_d, 1, box_rows, 1}.
+bool make_tmap_bhsd(CUtensorMap* m, const void* base, int B, int rows, int heads, int D, int box_d, int box_rows,
+                    CUtensorMapSwizzle swz);
+
+int num_sms();
+
+// Device address of the library's error word on the current device.
+unsigned int* error_word();
+
+}  // namespace ra

@@ -1,0 +1,208 @@
+// Ring scheduler shared by every prefill kernel and by the host statistics.
+//
+// Ownership of chunks, the ring visiting order and the causal tile filter of
+// "Lesson 8: Context Parallelism":
+//   * section 4A -- contiguous split: P chunks, rank r owns chunk r;
+//   * section 4B -- zig-zag split: 2P chunks, rank r owns chunks r, 2P-1-r;
+//   * section 2  -- at ring step t rank r holds the K/V block that started on
+//                   rank (r - t) mod P;
+//   * section 4  -- causal rule: query position i sees key position j <= i,
+//                   so K/V tiles that start after the last query of a tile
+//                   are never issued, and only tiles straddling the diagonal
+//                   (or a ragged chunk end) need the element mask.
+// Everything is index arithmetic: no work list is stored, so the library
+// needs no memory of its own.  Work items are handed out longest-first
+// (queries at later positions meet more keys), which balances the
+// persistent CTAs.
+#pragma once
+#include <cstdint>
+
+#if defined(__CUDACC__)
+#define RA_HD __host__ __device__ __forceinline__
+#else
+#define RA_HD inline
+#endif
+
+namespace ra {
+
+enum { kLayoutContiguous = 0, kLayoutZigzag = 1 };
+enum { kModeRing = 0, kModeStep = 1 };
+
+struct Plan {
+  int B, Hq, Hkv, D;
+  int causal;
+  int mode;      // kModeRing: buffers hold the whole sequence; kModeStep: one hop
+  int layout;    // ring mode: split of the sequence
+  int P;         // ring mode: virtual ranks
+  int C;         // tokens per chunk
+  int nqc, nkc;  // chunks held in the Q buffer and in the K/V buffer
+  int qid[2];    // step mode: global chunk index of each Q-buffer chunk
+  int kid[2];    // step mode: global chunk index of each K/V-buffer chunk
+  int Sq, Skv;   // rows of the Q buffer / K/V buffer (nqc*C, nkc*C)
+};
+
+RA_HD int imin(int a, int b) { return a < b ? a : b; }
+RA_HD int imax(int a, int b) { return a > b ? a : b; }
+RA_HD int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+RA_HD int chunks_per_rank(const Plan& p) { return p.layout == kLayoutZigzag ? 2 : 1; }
+
+// Owner rank of global chunk c (ring mode).
+RA_HD int chunk_owner(const Plan& p, int c) {
+  if (p.layout == kLayoutZigzag) return c < p.P ? c : 2 * p.P - 1 - c;
+  return c;
+}
+
+// j-th chunk (j < chunks_per_rank) owned by rank r.
+RA_HD int rank_chunk(const Plan& p, int r, int j) {
+  if (p.layout == kLayoutZigzag) return j == 0 ? r : 2 * p.P - 1 - r;
+  return r;
+}
+
+RA_HD int q_gid(const Plan& p, int slot) { return p.mode == kModeRing ? slot : p.qid[slot]; }
+RA_HD int kv_gid(const Plan& p, int slot) { return p.mode == kModeRing ? slot : p.kid[slot]; }
+
+// idx-th K/V slot visited by queries of Q slot `qslot`: ring order of the
+// owning rank in ring mode, buffer order in step mode.
+RA_HD int kv_slot(const Plan& p, int qslot, int idx) {
+  if (p.mode == kModeStep) return idx;
+  const int r = chunk_owner(p, qslot);
+  const int cpr = chunks_per_rank(p);
+  const int t = idx / cpr, j = idx - t * cpr;
+  int src = (r - t) % p.P;
+  if (src < 0) src += p.P;
+  return rank_chunk(p, src, j);
+}
+
+// One K/V tile: rows [row0, row0 + nvalid) of the K/V buffer, global
+// positions [pos0, pos0 + nvalid), chunk slot and global chunk id.
+struct KvTile {
+  int row0, pos0, nvalid, slot, gid, first_in_chunk;
+};
+
+struct KvIter {
+  int idx, kt;
+};
+
+// Next K/V tile (of BN keys) for queries whose last valid global position is
+// qhi.  Tiles entirely after qhi are skipped when causal.
+RA_HD bool kv_next(const Plan& p, int qslot, int qhi, int BN, KvIter& it, KvTile& t) {
+  const int tiles = cdiv(p.C, BN);
+  while (it.idx < p.nkc) {
+    const int slot = kv_slot(p, qslot, it.idx);
+    const int gid = kv_gid(p, slot);
+    const int k0 = it.kt * BN;
+    const int pos0 = gid * p.C + k0;
+    if (it.kt >= tiles || (p.causal && pos0 > qhi)) {
+      it.idx++;
+      it.kt = 0;
+      continue;
+    }
+    t.row0 = slot * p.C + k0;
+    t.pos0 = pos0;
+    t.nvalid = imin(BN, p.C - k0);
+    t.slot = slot;
+    t.gid = gid;
+    t.first_in_chunk = (it.kt == 0);
+    it.kt++;
+    return true;
+  }
+  return false;
+}
+
+// Q slots ordered by decreasing global chunk id (longest work first).
+RA_HD int q_slot_by_rank(const Plan& p, int k) {
+  if (p.mode == kModeRing) return p.nqc - 1 - k;
+  if (p.nqc == 1) return 0;
+  const bool first_later = p.qid[0] > p.qid[1];
+  return (k == 0) == first_later ? 0 : 1;
+}
+
+// ---------------------------------------------------------------------------
+// Work items of the tensor-core kernel: two 128-row query tiles that share
+// every K/V tile.  When the GQA group G = Hq/Hkv is even the two tiles are two
+// query heads of one K/V head at the same rows (identical masks); otherwise
+// they are two consecutive row tiles of one head inside one chunk.
+// ---------------------------------------------------------------------------
+struct Item {
+  int b, hkv, h[2];
+  int qslot;
+  int qrow0[2];  // first row of tile i in the Q buffer
+  int qpos0[2];  // global position of that row
+  int nrows[2];  // valid rows of tile i (0..BM)
+  int qlo, qhi;  // first / last valid global position over both tiles
+  int tile_in_chunk[2];
+};
+
+struct ItemSpace {
+  int head_pairs;  // 1: two heads per item; 0: two row tiles per item
+  int tq;          // BM-row tiles per Q chunk
+  int per_chunk;   // items per Q chunk and head group
+  int nbh;         // head groups x batch
+  int count;       // total items
+};
+
+RA_HD ItemSpace item_space(const Plan& p, int BM) {
+  ItemSpace s;
+  const int G = p.Hq / p.Hkv;
+  s.head_pairs = (G % 2 == 0) ? 1 : 0;
+  s.tq = cdiv(p.C, BM);
+  s.per_chunk = s.head_pairs ? s.tq : cdiv(s.tq, 2);
+  s.nbh = s.head_pairs ? p.B * p.Hkv * (G / 2) : p.B * p.Hq;
+  s.count = s.nbh * p.nqc * s.per_chunk;
+  return s;
+}
+
+RA_HD Item item_at(const Plan& p, const ItemSpace& s, int BM, int L) {
+  Item it;
+  const int pos_index = L / s.nbh;
+  const int bh = L - pos_index * s.nbh;
+  const int slot_rank = pos_index / s.per_chunk;
+  const int within = s.per_chunk - 1 - (pos_index - slot_rank * s.per_chunk);
+  it.qslot = q_slot_by_rank(p, slot_rank);
+  const int G = p.Hq / p.Hkv;
+  int t0, t1;
+  if (s.head_pairs) {
+    const int hp_per_b = p.Hkv * (G / 2);
+    it.b = bh / hp_per_b;
+    const int r = bh - it.b * hp_per_b;
+    it.hkv = r / (G / 2);
+    const int pair = r - it.hkv * (G / 2);
+    it.h[0] = it.hkv * G + 2 * pair;
+    it.h[1] = it.h[0] + 1;
+    t0 = t1 = within;
+  } else {
+    it.b = bh / p.Hq;
+    it.h[0] = it.h[1] = bh - it.b * p.Hq;
+    it.hkv = it.h[0] / G;
+    t0 = 2 * within;
+    t1 = 2 * within + 1;
+  }
+  const int cbase_row = it.qslot * p.C;
+  const int cbase_pos = q_gid(p, it.qslot) * p.C;
+  const int ts[2] = {t0, t1};
+  it.qlo = 0x7fffffff;
+  it.qhi = -1;
+  for (int i = 0; i < 2; ++i) {
+    const int off = ts[i] * BM;
+    it.tile_in_chunk[i] = ts[i];
+    it.qrow0[i] = cbase_row + off;
+    it.qpos0[i] = cbase_pos + off;
+    it.nrows[i] = ts[i] < s.tq ? imin(BM, p.C - off) : 0;
+    if (it.nrows[i] > 0) {
+      it.qlo = imin(it.qlo, it.qpos0[i]);
+      it.qhi = imax(it.qhi, it.qpos0[i] + it.nrows[i] - 1);
+    }
+  }
+  return it;
+}
+
+// Causal class of a tile with valid query positions [q0,q1] and key positions
+// [k0,k1]: 0 full (no mask), 1 partial (mask), 2 skipped.
+RA_HD int tile_class(int causal, int q0, int q1, int k0, int k1) {
+  if (!causal || k1 <= q0) return 0;
+  if (k0 > q1) return 2;
+  return 1;
+}
+
+}  // namespace ra

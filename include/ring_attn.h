@@ -1,0 +1,251 @@
+/*
+ * ring_attn.h -- C ABI of a B200 (sm_100a) library for exact ring attention
+ * emulated on one GPU.
+ *
+ * What is computed.  A sequence of S tokens is cut into chunks and dealt to P
+ * virtual ranks ("Lesson 8: Context Parallelism", section 1 and Fig. 8-2).
+ * Each rank keeps its query shard fixed and meets the K/V blocks of every
+ * rank in ring order -- at step t the block that started on rank (r-t) mod P
+ * (section 2, Fig. 8-3) -- folding each block into a running state (m, l, O)
+ * with the online-softmax update of section 3.  After the full loop each
+ * query has seen every allowed key, so the result is exact attention
+ * softmax(scale * Q K^T) V (section 1; "Sequence parallelism and ring
+ * attention", FAQ).  Causal masking follows section 4 (query i sees keys
+ * j <= i, global positions); the contiguous split is section 4A, the zig-zag
+ * split (2P chunks, rank r owns chunks r and 2P-1-r) section 4B.  The decode
+ * entry points shard the KV cache of one-token queries along the sequence
+ * ("NVIDIA unveils Helix Parallelism", Phase 1, KV parallelism) and merge the
+ * per-shard partial results.
+ *
+ * Conventions shared by every entry point.
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no memory and keeps no state except one device error word.
+ *   - Row-major layouts, last index contiguous:
+ *       q, out        [B, S, Hq, D]        k, v  [B, S, Hkv, D]
+ *       lse           [B, Hq, S]  float, natural log: lse = m + ln l
+ *     Query head h reads K/V head h / (Hq / Hkv) (grouped-query attention).
+ *   - dtype RING_BF16: q, k, v, out are bfloat16, accumulation is float32 on
+ *     the tensor cores (tcgen05, accumulators in tensor memory).
+ *     dtype RING_FP32: q, k, v, out are float32, float32 FMA on CUDA cores.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream) and does not synchronise the host.
+ *   - Pointers must be 16-byte aligned.  Errors are returned, never printed;
+ *     nothing aborts.
+ *   - RING_ETIMEOUT is reported by ring_attn_device_error(): every wait inside
+ *     a kernel is bounded; a wait that expires sets the device error word and
+ *     the kernel returns early (its outputs are then undefined).
+ */
+#ifndef RING_ATTN_H_
+#define RING_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RING_OK = 0,
+  RING_EINVAL = -1,        /* bad argument: null/misaligned pointer, shape not divisible, ... */
+  RING_EUNSUPPORTED = -2,  /* valid but not built: head dim, dtype combination */
+  RING_ECUDA = -3,         /* a CUDA runtime / driver call or a launch failed */
+  RING_ETIMEOUT = -4       /* a bounded wait inside a kernel expired */
+} ring_status;
+
+typedef enum { RING_CONTIGUOUS = 0, RING_ZIGZAG = 1 } ring_layout; /* how the sequence is split */
+typedef enum { RING_BF16 = 0, RING_FP32 = 1 } ring_dtype;
+
+/* Global chunk indices carried by one ring step (see ring_attn_step). */
+typedef struct {
+  int32_t n_q;        /* query chunks in the shard: 1 (contiguous) or 2 (zig-zag) */
+  int32_t q[2];       /* their global chunk indices, in shard order            */
+  int32_t n_kv;       /* K/V chunks in the block: 1 or 2                        */
+  int32_t kv[2];      /* their global chunk indices, in buffer order            */
+  int32_t chunk_len;  /* tokens per chunk (all chunks have this length)        */
+  int32_t causal;     /* 1: key at global position j is allowed for query i iff j <= i */
+} ring_chunk_ids;
+
+/*
+ * ring_attn_fwd -- the whole ring loop of every virtual rank, fused in one
+ * persistent launch ("Lesson 8", sections 2-4).
+ *
+ * q [B,S,Hq,D], k/v [B,S,Hkv,D] in natural token order; out [B,S,Hq,D] (same
+ * dtype as q), lse [B,Hq,S] float.  The sequence is split into P chunks
+ * (layout RING_CONTIGUOUS, chunk length S/P) or 2P chunks (RING_ZIGZAG,
+ * chunk length S/(2P)).  For every rank and every query tile the kernel folds
+ * K/V tiles into the on-chip (m, l, O) state in the rank's ring order,
+ * skipping tiles that the causal mask removes entirely; the state never
+ * leaves the chip between ring steps.
+ *
+ * Returns RING_EINVAL for a null or misaligned pointer, B/Hq/Hkv/S/P < 1,
+ * Hq % Hkv != 0, S not divisible by the number of chunks, layout or dtype out
+ * of range, or a non-finite / non-positive scale; RING_EUNSUPPORTED for
+ * D not in {64, 128}; RING_ECUDA if a launch fails.
+ */
+ring_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                          int B, int Hq, int Hkv, int S, int D, int P, int causal, int layout,
+                          float scale, int dtype, void* stream);
+
+/*
+ * ring_attn_fwd_counted -- ring_attn_fwd that also counts, on the device, the
+ * work the scheduler actually issued.  `counters` is a device array of
+ * (2 + P) uint64 that the call ADDS to (zero it first):
+ *   counters[0]      128x128 tiles computed without a mask, summed over (b, hq)
+ *   counters[1]      128x128 tiles computed with the causal / ragged mask
+ *   counters[2 + r]  causal chunk pairs (query chunk, K/V chunk) with at least
+ *                    one allowed key met by virtual rank r, summed over (b, hq)
+ * Tiles are 128 query rows x 128 keys cut inside each chunk pair (the last
+ * tile of a chunk may be shorter).  Only dtype RING_BF16 counts; other
+ * arguments and errors as ring_attn_fwd.
+ */
+ring_status ring_attn_fwd_counted(const void* q, const void* k, const void* v, void* out, float* lse,
+                                  int B, int Hq, int Hkv, int S, int D, int P, int causal, int layout,
+                                  float scale, int dtype, unsigned long long* counters, void* stream);
+
+/*
+ * ring_attn_fwd_simt -- the same computation as ring_attn_fwd on CUDA cores
+ * with float32 FMA for both dtypes (bf16 inputs are widened exactly).  Slow;
+ * it exists to cross-check the tensor-core path on the GPU.
+ */
+ring_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse,
+                               int B, int Hq, int Hkv, int S, int D, int P, int causal, int layout,
+                               float scale, int dtype, void* stream);
+
+/*
+ * ring_attn_state_init -- set a ring state to its starting value
+ * m = -inf, l = 0, O = 0 ("Lesson 8", section 3, before the first block).
+ * m, l [B,Hq,S_loc] float; O [B,S_loc,Hq,D] float.
+ */
+ring_status ring_attn_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D,
+                                 void* stream);
+
+/*
+ * ring_attn_step -- one hop of the ring for one rank ("Lesson 8", section 2:
+ * local attention of the fixed Q_r against the K/V block currently held,
+ * merged into O_r with the section-3 update).
+ *
+ * q_shard [B, n_q*C, Hq, D]: the rank's query chunks ids->q[0..n_q) stacked in
+ * that order (C = ids->chunk_len); kchunk, vchunk [B, n_kv*C, Hkv, D]: the
+ * held K/V chunks ids->kv[0..n_kv) stacked in that order.  State, read and
+ * written in place:  m, l [B, Hq, n_q*C] float (m is the running max of the
+ * scaled scores, natural units; l = sum exp(s - m)) and O [B, n_q*C, Hq, D]
+ * float, normalised (O = sum exp(s - m) v / l), as in section 3.  Rows whose
+ * block has no allowed key keep their state.  Fully masked tiles are skipped.
+ *
+ * Returns RING_EINVAL for null/misaligned pointers, ids == NULL, n_q or n_kv
+ * outside {1,2}, chunk_len < 1, negative chunk ids, Hq % Hkv != 0, bad dtype
+ * or scale; RING_EUNSUPPORTED for D not in {64,128}; RING_ECUDA on launch
+ * failure.
+ */
+ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* vchunk,
+                           float* m, float* l, float* O, const ring_chunk_ids* ids,
+                           int B, int Hq, int Hkv, int D, float scale, int dtype, void* stream);
+
+/*
+ * ring_attn_state_finalize -- out = O (cast to dtype), lse = m + ln l, for a
+ * state produced by ring_attn_step.  out [B,S_loc,Hq,D]; lse [B,Hq,S_loc].
+ * A row with l == 0 gets out = 0 and lse = -inf.
+ */
+ring_status ring_attn_state_finalize(const float* m, const float* l, const float* O, void* out,
+                                     float* lse, int B, int Hq, int S_loc, int D, int dtype,
+                                     void* stream);
+
+/*
+ * ring_attn_decode_partial -- split-KV single-token decode, the KV cache
+ * sharded along the sequence into P chunks ("Helix Parallelism", Phase 1).
+ *
+ * q [B,Hq,D] bf16 (one query token per sequence); k, v [B,Smax,Hkv,D] bf16;
+ * seqlens [B] int32 on the device (keys j < seqlens[b] are valid; 0 <= seqlens
+ * <= Smax, checked by the kernel: out-of-range entries are clamped and raise
+ * no fault).  Chunk p covers rows [p*Smax/P, (p+1)*Smax/P).  Writes, per
+ * (b, hq, p), the normalised partial output partials[B,Hq,P,D] float and
+ * part_lse[B,Hq,P] float; a chunk with no valid key gives O = 0 and
+ * lse = -inf.  Inside a chunk the rows are further split across CTAs and
+ * recombined with the same update; `workspace` (device, at least
+ * ring_attn_decode_workspace_bytes(...) bytes, 256-byte aligned) holds those
+ * sub-results and per-chunk arrival counters.  The counters must be zero
+ * before the first call on a workspace; every call leaves them zero again.
+ * Calls that share a workspace must not overlap on the GPU.
+ *
+ * Returns RING_EINVAL for null/misaligned pointers, Smax % P != 0, shapes < 1,
+ * Hq % Hkv != 0, workspace too small; RING_EUNSUPPORTED unless dtype ==
+ * RING_BF16 and D == 128; RING_ECUDA on launch failure.
+ */
+ring_status ring_attn_decode_partial(const void* q, const void* k, const void* v,
+                                     const int32_t* seqlens, float* partials, float* part_lse,
+                                     int B, int Hq, int Hkv, int Smax, int D, int P, float scale,
+                                     int dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/* Bytes of workspace ring_attn_decode_partial needs for these sizes (0 on bad sizes). */
+size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P);
+
+/*
+ * ring_attn_merge -- combine P normalised partial results per (b, hq):
+ *   lse = m* + ln sum_p exp(lse_p - m*),  m* = max_p lse_p
+ *   out = sum_p exp(lse_p - lse) O_p
+ * (the section-3 update of "Lesson 8" applied to whole partial states).
+ * partials [B,Hq,P,D] float, part_lse [B,Hq,P] float; out [B,Hq,D] of
+ * out_dtype (RING_BF16 or RING_FP32), out_lse [B,Hq] float (may be NULL).
+ * If every part is empty: out = 0, lse = -inf.
+ * Returns RING_EINVAL / RING_EUNSUPPORTED (D not a multiple of 4 or > 1024) /
+ * RING_ECUDA.
+ */
+ring_status ring_attn_merge(const float* partials, const float* part_lse, void* out, float* out_lse,
+                            int B, int Hq, int P, int D, int out_dtype, void* stream);
+
+/*
+ * ring_attn_decode -- the whole split-KV decode: ring_attn_decode_partial
+ * followed by ring_attn_merge on the same stream.  partials / part_lse are
+ * the caller's buffers for the per-chunk results (as above); out [B,Hq,D]
+ * bf16 and out_lse [B,Hq] float (may be NULL) receive attention over all
+ * seqlens[b] keys.  Errors as the two calls.
+ */
+ring_status ring_attn_decode(const void* q, const void* k, const void* v, const int32_t* seqlens, float* partials,
+                             float* part_lse, void* out, float* out_lse, int B, int Hq, int Hkv, int Smax, int D,
+                             int P, float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ring_attn_sched_stats -- the scheduler's host-side view of one (batch, head)
+ * of a causal or full ring, without running anything: per-rank unmasked
+ * chunk pairs (a diagonal pair counts once; "Lesson 8", section 4B: 2P+1 per
+ * zig-zag rank, section 4A: r+1 per contiguous rank) and tile classes for
+ * tile_q x tile_k tiles cut inside each chunk pair (full: no mask needed;
+ * partial: masked; skipped: fully masked, never issued).
+ * per_rank_pairs has room for P values.  Any output pointer may be NULL.
+ */
+ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile_q, int tile_k,
+                                  int64_t* per_rank_pairs, int64_t* full, int64_t* partial,
+                                  int64_t* skipped);
+
+/*
+ * ring_attn_device_error -- synchronise the current device and read-and-clear
+ * the library's device error word.  Returns RING_ETIMEOUT if a bounded wait
+ * in any kernel expired since the last call, RING_ECUDA if the device
+ * reports an error, else RING_OK.  `where` (may be NULL) receives a code of
+ * the wait that expired (0 if none).
+ */
+ring_status ring_attn_device_error(int* where);
+
+/*
+ * ring_attn_selftest_wait -- launch one thread that waits on an mbarrier no
+ * one completes, giving up after limit_us microseconds (1..1e6) exactly as
+ * every wait inside the library's kernels gives up after its own limit.  The
+ * next ring_attn_device_error() then reports RING_ETIMEOUT.  No fault, trap
+ * or hang is involved; it exists to test the error path.
+ */
+ring_status ring_attn_selftest_wait(int limit_us, void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* ring_attn_strerror(ring_status status);
+
+/* Library version and the SM architecture it was compiled for (e.g. 100). */
+int ring_attn_version(void);
+int ring_attn_built_arch(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RING_ATTN_H_ */

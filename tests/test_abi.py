@@ -1,0 +1,137 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads and exports
+every function include/ring_attn.h declares, argument checks return their
+documented codes without touching a device, and the scheduler's host view
+(ring_attn_sched_stats) equals the oracle's enumeration exactly."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import context_exact_attention_ring_b200 as ra
+from oracle import schedule as sch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ring_attn.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from context_exact_attention_ring_b200 import build
+    build.build()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(ring_attn_[a-z0-9_]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_header_declares_the_three_core_calls():
+    names = declared_functions()
+    for n in ("ring_attn_fwd", "ring_attn_step", "ring_attn_merge"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported():
+    L = ra.lib()
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(ra.EXPORTED) <= set(names)
+
+
+def test_version_and_arch():
+    assert ra.lib().ring_attn_version() >= 1
+    assert ra.lib().ring_attn_built_arch() == 100
+
+
+def test_strerror():
+    for s in (0, -1, -2, -3, -4):
+        assert ra.strerror(s)
+    assert ra.strerror(-4) != ra.strerror(-1)
+
+
+FAKE = 0x10000  # aligned, non-null; never dereferenced: every case below fails before any launch
+
+
+def fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, S=256, D=64, P=4, causal=1, layout=0,
+             scale=0.125, dtype=1)
+    a.update(kw)
+    return ra.lib().ring_attn_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["S"],
+                                  a["D"], a["P"], a["causal"], a["layout"], a["scale"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), ra.RING_EINVAL), (dict(lse=None), ra.RING_EINVAL), (dict(k=FAKE + 4), ra.RING_EINVAL),
+    (dict(B=0), ra.RING_EINVAL), (dict(Hq=3), ra.RING_EINVAL), (dict(S=250), ra.RING_EINVAL),
+    (dict(layout=1, S=260), ra.RING_EINVAL), (dict(layout=7), ra.RING_EINVAL), (dict(dtype=5), ra.RING_EINVAL),
+    (dict(scale=0.0), ra.RING_EINVAL), (dict(scale=float("nan")), ra.RING_EINVAL), (dict(P=0), ra.RING_EINVAL),
+    (dict(D=96), ra.RING_EUNSUPPORTED), (dict(D=256), ra.RING_EUNSUPPORTED),
+])
+def test_fwd_argument_checks(kw, code):
+    assert fwd(**kw) == code
+
+
+def test_step_argument_checks():
+    L = ra.lib()
+    ids = ra.ChunkIds()
+    ids.n_q, ids.n_kv, ids.chunk_len, ids.causal = 1, 1, 64, 1
+    ids.q[0], ids.kv[0] = 0, 0
+    args = lambda i, D=64: (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(i), 1, 2, 2, D, 0.125, 1, None)
+    assert L.ring_attn_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 64, 0.125, 1, None) == ra.RING_EINVAL
+    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.n_q = 3
+    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
+    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.kv[0] = -1
+    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
+    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.chunk_len = 0
+    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
+    assert L.ring_attn_step(*args(ids, D=80)) == ra.RING_EUNSUPPORTED
+
+
+def test_decode_and_merge_argument_checks():
+    L = ra.lib()
+    ws = ra.ring_attn_decode_workspace_bytes(8, 32, 8, 1 << 20, 128, 32)
+    assert ws > 0
+    assert ra.ring_attn_decode_workspace_bytes(8, 32, 8, 1000, 128, 32) == 0      # Smax % P
+    base = dict(q=FAKE, k=FAKE, v=FAKE, sl=FAKE, part=FAKE, plse=FAKE, B=8, Hq=32, Hkv=8, Smax=1 << 20, D=128, P=32,
+                scale=0.088, dtype=0, ws=FAKE * 16, wsb=ws)
+
+    def dec(**kw):
+        a = dict(base); a.update(kw)
+        return L.ring_attn_decode_partial(a["q"], a["k"], a["v"], a["sl"], a["part"], a["plse"], a["B"], a["Hq"],
+                                          a["Hkv"], a["Smax"], a["D"], a["P"], a["scale"], a["dtype"], a["ws"],
+                                          a["wsb"], None)
+    assert dec(sl=None) == ra.RING_EINVAL
+    assert dec(Smax=1000) == ra.RING_EINVAL
+    assert dec(wsb=ws - 1) == ra.RING_EINVAL
+    assert dec(ws=FAKE + 16) == ra.RING_EINVAL          # workspace must be 256-byte aligned
+    assert dec(D=64) == ra.RING_EUNSUPPORTED
+    assert dec(dtype=1) == ra.RING_EUNSUPPORTED
+    assert dec(Hq=64) == ra.RING_EUNSUPPORTED            # GQA group of 8 is not built
+    assert L.ring_attn_merge(FAKE, FAKE, None, None, 1, 1, 1, 128, 0, None) == ra.RING_EINVAL
+    assert L.ring_attn_merge(FAKE, FAKE, FAKE, None, 1, 1, 1, 130, 0, None) == ra.RING_EUNSUPPORTED
+    assert L.ring_attn_merge(FAKE, FAKE, FAKE, None, 1, 1, 0, 128, 0, None) == ra.RING_EINVAL
+
+
+@pytest.mark.parametrize("S,P,layout,causal,tq,tk", [
+    (256, 4, "contiguous", False, 64, 64), (8192, 8, "contiguous", True, 128, 128),
+    (32768, 8, "zigzag", True, 128, 128), (131072, 16, "zigzag", True, 128, 128),
+    (1536, 3, "zigzag", True, 128, 128), (1000, 4, "zigzag", True, 128, 128), (960, 5, "contiguous", True, 64, 128),
+])
+def test_sched_stats_equals_oracle_enumeration(S, P, layout, causal, tq, tk):
+    per, full, partial, skipped = ra.ring_attn_sched_stats(S, P, causal, layout, tq, tk)
+    o_full, o_partial, o_skipped, _ = sch.tile_classes(S, P, layout, causal, tq, tk)
+    assert (full, partial, skipped) == (o_full, o_partial, o_skipped)
+    assert per == sch.per_rank_pairs(P, layout, causal)
+
+
+def test_sched_stats_zigzag_closed_form():
+    for P in (2, 8, 16):
+        per, *_ = ra.ring_attn_sched_stats(64 * 2 * P, P, True, "zigzag")
+        assert per == [2 * P + 1] * P
+        per, *_ = ra.ring_attn_sched_stats(64 * P, P, True, "contiguous")
+        assert per == [r + 1 for r in range(P)]

@@ -1,0 +1,119 @@
+"""GPU parity of the split-KV decode (per-chunk partials, intra-chunk
+sub-split combine, the (O, lse) merge) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import context_exact_attention_ring_b200 as ra
+import oracle
+import workloads as W
+from oracle import merge as omerge
+from tests.helpers import TOL_BF16_LSE, TOL_BF16_OUT, host, need_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_decode(q, k, v, lens, scale, heads=None, chunk=None):
+    """Per (b, hq): attention of the single query over keys j < lens[b]
+    (restricted to [p*chunk, (p+1)*chunk) when chunk=(p, C))."""
+    qh, B = host(q), q.shape[0]
+    Hq, Hkv = q.shape[1], k.shape[2]
+    G = Hq // Hkv
+    outs, lses = {}, {}
+    for b in range(B):
+        for g in range(Hkv):
+            hs = [h for h in range(g * G, (g + 1) * G) if heads is None or (b, h) in heads]
+            if not hs:
+                continue
+            L = int(lens[b])
+            lo, hi = (0, k.shape[1]) if chunk is None else (chunk[0] * chunk[1], (chunk[0] + 1) * chunk[1])
+            ks = host(k[b:b + 1, lo:hi, g:g + 1])
+            vs = host(v[b:b + 1, lo:hi, g:g + 1])
+            kl = np.array([max(0, min(L - lo, hi - lo))])
+            qq = qh[b:b + 1, None, g * G:(g + 1) * G, :]
+            rows = [(0, h - g * G, 0) for h in hs]
+            o, l = oracle.attention_rows(qq, ks, vs, rows, scale=scale, causal=False, kv_len=kl)
+            for n, h in enumerate(hs):
+                outs[(b, h)] = o[n]
+                lses[(b, h)] = l[n]
+    return outs, lses
+
+
+def make(B, Hq, Hkv, cap, lens, seed):
+    cfg = W.Decode("t", B, Hq, Hkv, 128, cap, 1, seed, fixed_lens=tuple(lens))
+    q, k, v, sl = W.decode_inputs(cfg, "cuda")
+    return cfg, q, k, v, sl
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 2), (3, 3)])
+def test_decode_small(Hq, Hkv):
+    need_cuda()
+    lens = [0, 1, 5000, 8192, 8193, 32768, 12345, 20000]
+    cfg, q, k, v, sl = make(len(lens), Hq, Hkv, 32768, lens, 61)
+    P = 4
+    ws = ra.decode_workspace(cfg.B, Hq, Hkv, cfg.capacity, 128, P)
+    part, plse = ra.ring_attn_decode_partial(q, k, v, sl, P, cfg.scale, workspace=ws)
+    out, out_lse = ra.ring_attn_merge(part, plse)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    C = cfg.capacity // P
+    # per-chunk partials: the oracle over each chunk's valid keys
+    for p in range(P):
+        ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale, chunk=(p, C))
+        for (b, h), ro in ref_o.items():
+            rl = ref_l[(b, h)]
+            gl = float(host(plse)[b, h, p])
+            if np.isneginf(rl):
+                assert np.isneginf(gl) and np.all(host(part)[b, h, p] == 0)
+            else:
+                assert abs(gl - rl) <= TOL_BF16_LSE
+                assert np.max(np.abs(host(part)[b, h, p] - ro)) <= TOL_BF16_OUT
+    # merged result: attention over all valid keys
+    ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale)
+    for (b, h), ro in ref_o.items():
+        if lens[b] == 0:
+            assert np.isneginf(host(out_lse)[b, h]) and np.all(host(out)[b, h] == 0)
+            continue
+        assert abs(host(out_lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
+        assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+    # the arrival counters are back at zero: a second call on the same workspace agrees
+    out2, lse2 = ra.ring_attn_decode(q, k, v, sl, P, cfg.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out) and torch.equal(lse2, out_lse)
+
+
+def test_merge_kernel_against_oracle_formula():
+    need_cuda()
+    g = torch.Generator(device="cuda").manual_seed(71)
+    B, Hq, P, D = 3, 5, 37, 128
+    part = torch.randn((B, Hq, P, D), generator=g, device="cuda")
+    plse = torch.randn((B, Hq, P), generator=g, device="cuda") * 4
+    plse[0, 1, ::3] = float("-inf")
+    plse[2, 4, :] = float("-inf")           # every part empty
+    for dt in (torch.float32, torch.bfloat16):
+        out, lse = ra.ring_attn_merge(part, plse, dtype=dt)
+        ro, rl = omerge.merge(host(part), host(plse))
+        tol = 1e-5 if dt == torch.float32 else TOL_BF16_OUT
+        assert np.max(np.abs(host(out) - ro)) <= tol
+        fin = np.isfinite(rl)
+        assert np.max(np.abs(host(lse)[fin] - rl[fin])) <= 1e-5
+        assert np.all(np.isneginf(host(lse)[~fin]))
+
+
+def test_cfg5_full_size_sampled():
+    # KV-sharded decode at full size: B8, Hq32, Hkv8, D128, 2^20 context, P=32, lengths U[0.5M, 1M]
+    need_cuda()
+    cfg = W.CFG5
+    q, k, v, sl = W.decode_inputs(cfg, "cuda")
+    out, out_lse = ra.ring_attn_decode(q, k, v, sl, cfg.P, cfg.scale)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    lens = host(sl).astype(np.int64)
+    rng = np.random.default_rng(cfg.seed + 1000)
+    G = cfg.Hq // cfg.Hkv
+    groups = {b: int(rng.integers(cfg.Hkv)) for b in range(cfg.B)}   # one kv head per sequence, all its q heads
+    heads = {(b, g * G + i) for b, g in groups.items() for i in range(G)}
+    ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale, heads=heads)
+    err_o = max(np.max(np.abs(host(out)[b, h] - ro)) for (b, h), ro in ref_o.items())
+    err_l = max(abs(host(out_lse)[b, h] - ref_l[(b, h)]) for (b, h) in ref_o)
+    assert err_o <= TOL_BF16_OUT and err_l <= TOL_BF16_LSE, (err_o, err_l)
