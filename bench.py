@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the ring-attention hot path on B200.
+
+One "step" is one pass of the whole hot path on one batch of synthetic input:
+  * prefill: the fused ring (all P virtual ranks) of the causal zig-zag GQA
+    workload B1 Hq32 Hkv8 S131072 D128 P16 -- the headline metric,
+    causal-adjusted TFLOP/s (4*B*Hq*S^2*D/2 per step);
+  * decode: the split-KV single-token decode B8 Hq32 Hkv8 D128, 2^20-token
+    capacity in 32 chunks, valid lengths U[0.5M, 1M] (partials + merge),
+    reported in the same line as GB/s of algorithmic bytes.
+Inputs are resident in HBM before the timed region (both workloads' inputs
+exceed the 126 MB L2).  Times are CUDA events on the launching stream;
+multi-GPU runs are independent replicas (no collective on the data path),
+timed as the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (the reference arm of this build).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        return dist, int(os.environ["RANK"]), world
+    return None, 0, 1
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- the hot path
+def decode_bytes(cfg, lens: np.ndarray) -> float:
+    """Algorithmic bytes of one split-KV decode: every valid K and V row once,
+    q, the partial results written and read back, the output and lse."""
+    kv = float(lens.sum()) * cfg.Hkv * cfg.D * 2 * 2
+    q = cfg.B * cfg.Hq * cfg.D * 2
+    parts = cfg.B * cfg.Hq * cfg.P * (cfg.D + 1) * 4 * 2
+    out = cfg.B * cfg.Hq * (cfg.D * 2 + 4)
+    return kv + q + parts + out
+
+
+def run_ours(args):
+    import context_exact_attention_ring_b200 as ra
+
+    dist, rank, world = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    st = torch.cuda.current_stream()
+    pk, pk_kind = peaks()
+    cfg, dcfg = W.CFG4, W.CFG5
+
+    q, k, v = W.prefill_inputs(cfg, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.S), device=dev, dtype=torch.float32)
+    dq, dk, dv, dl = W.decode_inputs(dcfg, dev)
+    lens = dl.cpu().numpy().astype(np.int64)
+    part = torch.empty((dcfg.B, dcfg.Hq, dcfg.P, dcfg.D), device=dev, dtype=torch.float32)
+    plse = torch.empty((dcfg.B, dcfg.Hq, dcfg.P), device=dev, dtype=torch.float32)
+    dout = torch.empty((dcfg.B, dcfg.Hq, dcfg.D), device=dev, dtype=torch.bfloat16)
+    dlse = torch.empty((dcfg.B, dcfg.Hq), device=dev, dtype=torch.float32)
+    ws = ra.decode_workspace(dcfg.B, dcfg.Hq, dcfg.Hkv, dcfg.capacity, dcfg.D, dcfg.P, dev)
+    torch.cuda.synchronize()
+
+    def prefill():
+        ra.ring_attn_fwd(q, k, v, cfg.P, causal=True, layout=cfg.layout, scale=cfg.scale, out=out, lse=lse)
+
+    def decode():
+        ra.ring_attn_decode(dq, dk, dv, dl, dcfg.P, dcfg.scale, partials=part, part_lse=plse, out=dout,
+                            out_lse=dlse, workspace=ws)
+
+    for _ in range(args.warmup):
+        prefill()
+        decode()
+    torch.cuda.synchronize()
+    st_err = ra.ring_attn_device_error()[0]
+    if st_err != ra.RING_OK:
+        raise RuntimeError(f"device error during warm-up: {st_err}")
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(dist)
+    torch.cuda.synchronize()
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(st)
+    for e0, e1, e2 in ev:
+        e0.record(st)
+        prefill()
+        e1.record(st)
+        decode()
+        e2.record(st)
+    t_all1.record(st)
+    torch.cuda.synchronize()
+    barrier(dist)
+    clk = clocks.stop()
+    if ra.ring_attn_device_error()[0] != ra.RING_OK:
+        raise RuntimeError("device error during the timed region")
+
+    pre_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    dec_ms = [b.elapsed_time(c) for _, b, c in ev]
+    total_ms = t_all0.elapsed_time(t_all1)
+    total_ms = max_over_ranks(dist, total_ms)
+    pre_sum = max_over_ranks(dist, sum(pre_ms))
+    dec_sum = max_over_ranks(dist, sum(dec_ms))
+
+    flops = cfg.flops()
+    value = flops * args.steps * world / (pre_sum / 1e3) / 1e12          # causal-adjusted TFLOP/s, all ranks
+    dbytes = decode_bytes(dcfg, lens)
+    dvalue = dbytes * args.steps * world / (dec_sum / 1e3) / 1e9         # GB/s, all ranks
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        e2e_steps = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            q2 = hq.to(dev, non_blocking=True)
+            k2 = hk.to(dev, non_blocking=True)
+            v2 = hv.to(dev, non_blocking=True)
+            o2, l2 = ra.ring_attn_fwd(q2, k2, v2, cfg.P, causal=True, layout=cfg.layout, scale=cfg.scale)
+            hout.copy_(o2, non_blocking=True)
+            hlse.copy_(l2, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(dist)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(st)
+        for _ in range(e2e_steps):
+            e2e_step()
+        a1.record(st)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(dist, a0.elapsed_time(a1))
+        h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+        d2h = hout.numel() * 2 + hlse.numel() * 4
+        e2e = {"value": round(flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e2e_ms / e2e_steps, 3), "path": "pinned host -> ring_attn_fwd -> pinned host"}
+
+    # ---------------------------------------------------------------- roofline of the dominant kernel
+    pre_avg = statistics.mean(pre_ms)
+    achieved_tf = flops / (pre_avg / 1e3) / 1e12
+    peak_tf = pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]
+    dec_avg = statistics.mean(dec_ms)
+    achieved_gb = dbytes / (dec_avg / 1e3) / 1e9
+    traffic = load_traffic()
+
+    line = {
+        "metric": "causal-adjusted attention TFLOP/s at S=128k (1 GPU); split-KV decode GB/s",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), bf16; no dataset)",
+        "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "S": cfg.S, "D": cfg.D,
+                   "P": cfg.P, "layout": cfg.layout, "causal": True,
+                   "flops_per_step": flops, "l2": "inputs larger than L2 (q 1.07 GB, k+v 0.54 GB)",
+                   "decode_workload": dcfg.name, "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(achieved_tf / peak_tf, 4), "traffic": traffic.get("attn_tc"),
+                     "kernel": "attn_tc_kernel<128>", "peak_kind": f"{pk_kind} bf16 dense, sustained"},
+        "decode": {"metric": "split-KV decode GB/s", "value": round(dvalue, 1), "unit": "GB/s",
+                   "ms_per_step": round(dec_avg, 3), "bytes_per_step": dbytes,
+                   "roofline": {"bound": "hbm", "achieved": round(achieved_gb, 1), "peak": pk["hbm_gbs"],
+                                "unit": "GB/s", "frac": round(achieved_gb / pk["hbm_gbs"], 4),
+                                "traffic": traffic.get("decode"), "kernel": "decode_kernel<4> + merge_kernel",
+                                "peak_kind": f"{pk_kind} HBM copy"}},
+        "prefill_ms_per_step": round(pre_avg, 3),
+        "e2e": e2e,
+        "gpu_launches": args.steps * 3,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(cfg, q, k, v, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summary (None if absent)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f)
+    return {}
+
+
+# --------------------------------------------------------------------------- oracle on the host cores
+def cpu_baseline(cfg, q=None, k=None, v=None, seconds=15.0):
+    """fp64 oracle on a bounded sample of the workload's query rows, on every
+    host core; value in causal-adjusted TFLOP/s of the rows processed."""
+    import oracle
+    if q is None:
+        q, k, v = W.prefill_inputs(cfg, "cpu")
+    hq = q.float().cpu().numpy()
+    hk = k.float().cpu().numpy()
+    hv = v.float().cpu().numpy()
+    rng = np.random.default_rng(cfg.seed + 7)
+    cores = oracle.cores()
+    # calibrate on a small batch, then size the sample to about `seconds`
+    def rows_of(n):
+        b = rng.integers(0, cfg.B, n)
+        h = rng.integers(0, cfg.Hq, n)
+        i = rng.integers(0, cfg.S, n)
+        return np.stack([b, h, i], 1).astype(np.int32)
+    def flops_of(rows):
+        return float(np.sum(4.0 * cfg.D * (rows[:, 2].astype(np.float64) + 1)))
+    cal = rows_of(4 * cores)
+    t0 = time.perf_counter()
+    oracle.attention_rows(hq, hk, hv, cal, scale=cfg.scale, causal=True)
+    dt = time.perf_counter() - t0
+    rate = flops_of(cal) / max(dt, 1e-6)
+    n = int(max(4 * cores, min(200000, seconds * rate / (4.0 * cfg.D * cfg.S / 2))))
+    rows = rows_of(n)
+    t0 = time.perf_counter()
+    oracle.attention_rows(hq, hk, hv, rows, scale=cfg.scale, causal=True)
+    dt = time.perf_counter() - t0
+    return {"value": round(flops_of(rows) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} uniformly drawn query rows of {cfg.name} (causal fp64 rows, all allowed keys), "
+                      f"{dt:.1f} s", "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    """The reference arm: the oracle as it stands, timed on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = W.CFG4
+    q, k, v = W.prefill_inputs(cfg, "cpu")
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, q, k, v, seconds=1.0)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(cfg, q, k, v, seconds=args.cpu_seconds / max(1, args.steps)))
+    wall = time.perf_counter() - t0
+    value = statistics.mean(v_["value"] for v_ in vals)
+    line = {"impl": "reference", "metric": "causal-adjusted attention TFLOP/s at S=128k (1 GPU); split-KV decode GB/s",
+            "value": value, "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall * 1e3 / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1), bf16 values read exactly)",
+            "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "S": cfg.S, "D": cfg.D,
+                       "P": cfg.P, "layout": cfg.layout, "causal": True},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": vals[0]["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("note: warm-up raised to 3 steps", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

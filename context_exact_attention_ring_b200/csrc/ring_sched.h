@@ -153,10 +153,16 @@ RA_HD ItemSpace item_space(const Plan& p, int BM) {
   return s;
 }
 
+// Items are ordered head group by head group, and inside one head group by
+// decreasing query position.  A wave of concurrently running CTAs therefore
+// streams the K/V of a single kv head (which stays resident in L2), and the
+// persistent CTAs, which take items with a stride of the grid size, each get
+// an even spread of long and short items; the shortest come last.
 RA_HD Item item_at(const Plan& p, const ItemSpace& s, int BM, int L) {
   Item it;
-  const int pos_index = L / s.nbh;
-  const int bh = L - pos_index * s.nbh;
+  const int per_bh = p.nqc * s.per_chunk;
+  const int bh = L / per_bh;
+  const int pos_index = L - bh * per_bh;
   const int slot_rank = pos_index / s.per_chunk;
   const int within = s.per_chunk - 1 - (pos_index - slot_rank * s.per_chunk);
   it.qslot = q_slot_by_rank(p, slot_rank);
