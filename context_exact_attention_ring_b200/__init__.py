@@ -34,7 +34,7 @@ EXPORTED = (
     "ring_attn_fwd", "ring_attn_fwd_counted", "ring_attn_fwd_simt", "ring_attn_state_init", "ring_attn_step",
     "ring_attn_state_finalize", "ring_attn_decode_partial", "ring_attn_decode_workspace_bytes", "ring_attn_decode",
     "ring_attn_merge", "ring_attn_sched_stats", "ring_attn_device_error", "ring_attn_strerror",
-    "ring_attn_version", "ring_attn_built_arch", "ring_attn_selftest_wait",
+    "ring_attn_version", "ring_attn_built_arch", "ring_attn_selftest_wait", "ring_attn_decode_partial_noalloc",
 )
 
 
@@ -71,6 +71,7 @@ def lib():
         "ring_attn_state_finalize": [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp],
         "ring_attn_decode_partial": [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz, vp],
         "ring_attn_decode": [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz, vp],
+        "ring_attn_decode_partial_noalloc": [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp],
         "ring_attn_merge": [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp],
         "ring_attn_sched_stats": [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp],
         "ring_attn_device_error": [ctypes.POINTER(ctypes.c_int)],
@@ -254,6 +255,24 @@ def ring_attn_decode_partial(q, k, v, seqlens, P, scale=None, partials=None, par
                                         B, Hq, Hkv, Smax, D, int(P), scale, _dtype_code(q), _ptr(workspace),
                                         workspace.numel(), _stream())
     _check(st, "ring_attn_decode_partial")
+    return partials, part_lse
+
+
+def ring_attn_decode_partial_noalloc(q, k, v, seqlens, P, scale=None, partials=None, part_lse=None):
+    """ring_attn_decode_partial using the library's fixed scratch array (no
+    workspace, no allocation inside the call; see include/ring_attn.h).
+    Pass preallocated `partials` and `part_lse` to avoid torch allocations."""
+    _cuda(q, k, v, seqlens, partials, part_lse)
+    B, Hq, Hkv, Smax, D = _decode_shapes(q, k, seqlens, P)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if partials is None:
+        partials = torch.empty((B, Hq, P, D), device=q.device, dtype=torch.float32)
+    if part_lse is None:
+        part_lse = torch.empty((B, Hq, P), device=q.device, dtype=torch.float32)
+    st = lib().ring_attn_decode_partial_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), _ptr(partials),
+                                                _ptr(part_lse), B, Hq, Hkv, Smax, D, int(P), scale, _dtype_code(q),
+                                                _stream())
+    _check(st, "ring_attn_decode_partial_noalloc")
     return partials, part_lse
 
 

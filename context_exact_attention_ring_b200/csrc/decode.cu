@@ -400,3 +400,80 @@ cudaError_t launch_decode_partial(const DecodeArgs& a, cudaStream_t st) {
 }
 
 }  // namespace ra
+
+// ---------------------------------------------------------------------------
+// ring_attn_decode_partial_noalloc: the same decode, with its scratch (the
+// sub-split results and the per-chunk arrival counters) in a fixed array of
+// this library instead of a caller-provided workspace.
+//
+// It is for callers that cannot call cudaMalloc or hand this call a
+// workspace: host programs whose own allocator owns all device memory (a
+// fixed budget or a caching pool that must not be bypassed), and code on a
+// latency-critical path where an allocation, which may synchronise the
+// device, is not acceptable.  The array below is reserved on every GPU that
+// loads this library and held until the process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+#include "../../include/ring_attn.h"
+
+namespace ra {
+
+static __device__ __align__(256) unsigned char g_decode_scratch[RING_DECODE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_decode_scratch on the current device.  Host code must
+// not pass the symbol itself to a kernel: on the host it only names a
+// stand-in.  Looked up once per device (with that device current) on the
+// first call made on it.
+static cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  static void* cache[64] = {nullptr};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    cache[dev] = p;
+  }
+  *out = cache[dev];
+  return cudaSuccess;
+}
+
+}  // namespace ra
+
+extern "C" ring_status ring_attn_decode_partial_noalloc(const void* q, const void* k, const void* v,
+                                                        const int32_t* seqlens, float* partials, float* part_lse,
+                                                        int B, int Hq, int Hkv, int Smax, int D, int P, float scale,
+                                                        int dtype, void* stream) {
+  using namespace ra;
+  auto a16 = [](const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(q) || !a16(k) || !a16(v) || !seqlens || !a16(partials) || !a16(part_lse)) return RING_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Smax < 1 || P < 1 || D < 1 || Hq % Hkv || Smax % P) return RING_EINVAL;
+  if (!(scale > 0.f) || scale != scale || scale == __builtin_huge_valf()) return RING_EINVAL;
+  if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
+  if ((long long)B * Smax * Hkv * D >= (1LL << 42)) return RING_EINVAL;
+  if (dtype != RING_BF16 || D != 128) return RING_EUNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4) return RING_EUNSUPPORTED;
+  const size_t need = decode_workspace_bytes(B, Hq, Hkv, Smax, D, P);
+  if (need == 0 || need > (size_t)RING_DECODE_NOALLOC_SCRATCH_BYTES) return RING_EINVAL;
+  void* ws = nullptr;
+  if (noalloc_scratch(&ws) != cudaSuccess) return RING_ECUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a{};
+  a.q = q; a.k = k; a.v = v; a.seqlens = seqlens;
+  a.partials = partials; a.part_lse = part_lse;
+  decode_workspace_split(ws, B, Hq, Hkv, Smax, D, P, &a.ws_part, &a.ws_count);
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Smax = Smax; a.D = D; a.P = P; a.scale = scale;
+  a.err = error_word();
+  // the arrival counters must start at zero; the previous call may have been cut short
+  if (cudaMemsetAsync(a.ws_count, 0, (size_t)B * Hkv * P * sizeof(unsigned int), st) != cudaSuccess)
+    return RING_ECUDA;
+  const cudaError_t e = launch_decode_partial(a, st);
+  if (e == cudaSuccess) return RING_OK;
+  return e == cudaErrorNotSupported ? RING_EUNSUPPORTED : RING_ECUDA;
+}

@@ -182,6 +182,36 @@ ring_status ring_attn_decode_partial(const void* q, const void* k, const void* v
 size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P);
 
 /*
+ * ring_attn_decode_partial_noalloc -- ring_attn_decode_partial without a
+ * workspace argument and without any allocation.  (The pages have no
+ * counterpart: this is an interface convenience of the library.)
+ *
+ * For callers that cannot call cudaMalloc or pass a workspace: a host program
+ * whose own allocator owns all device memory (a fixed budget, or a caching
+ * pool that must not be bypassed), or code on a latency-critical path where an
+ * allocation, which may synchronise the device, is not acceptable.
+ *
+ * The scratch lives in one fixed array of RING_DECODE_NOALLOC_SCRATCH_BYTES
+ * bytes inside the library, reserved on every GPU that loads the library and
+ * held until the process exits.  Sizes whose scratch need
+ * (ring_attn_decode_workspace_bytes) exceeds that maximum are rejected with
+ * RING_EINVAL before anything is launched; the B8 Hq32 Hkv8 D128 2^20-token,
+ * 32-chunk decode needs about 34 MB.  The first call on a device looks up the
+ * array's device address (with that device current); make that first call
+ * before any stream capture.  Each call clears the array's arrival counters
+ * on `stream`, then launches the same kernel as ring_attn_decode_partial.
+ * No call allocates: no cudaMalloc, cudaFree or allocating library routine.
+ * All calls share the one array, so calls that overlap on the GPU (other
+ * streams, other host threads) race and give wrong results: serialise them.
+ * Other arguments, outputs and errors as ring_attn_decode_partial.
+ */
+#define RING_DECODE_NOALLOC_SCRATCH_BYTES (40u << 20)
+ring_status ring_attn_decode_partial_noalloc(const void* q, const void* k, const void* v,
+                                             const int32_t* seqlens, float* partials, float* part_lse,
+                                             int B, int Hq, int Hkv, int Smax, int D, int P, float scale,
+                                             int dtype, void* stream);
+
+/*
  * ring_attn_merge -- combine P normalised partial results per (b, hq):
  *   lse = m* + ln sum_p exp(lse_p - m*),  m* = max_p lse_p
  *   out = sum_p exp(lse_p - lse) O_p
