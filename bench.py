@@ -365,8 +365,61 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- profiling cases
+PROFILE_CASES = {
+    # tensor-core ring, causal zig-zag MHA with 1% of keys x8: q/k/v 268 MB each (> L2), one launch ~11 ms
+    "tc": W.CFG3,
+    # the timed S=128k GQA workload (only for single-pass ncu metrics)
+    "tc_full": W.CFG4,
+    # split-KV decode on 4 x 65536-token sequences (K+V 1.07 GB > L2, lengths U[32k, 64k])
+    "decode": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),
+    "decode_full": W.CFG5,
+}
+
+
+def run_profile(args):
+    """Launch one kernel of the hot path `--steps` times after `--warmup`
+    launches, for ncu captures (-k <kernel> -s <warmup>).  Prints the mean
+    CUDA-event time per launch."""
+    import context_exact_attention_ring_b200 as ra
+    name = args.profile
+    cfg = PROFILE_CASES[name]
+    dev = torch.device("cuda", 0)
+    if isinstance(cfg, W.Prefill):
+        q, k, v = W.prefill_inputs(cfg, dev)
+        out = torch.empty_like(q)
+        lse = torch.empty((cfg.B, cfg.Hq, cfg.S), device=dev, dtype=torch.float32)
+        fn = lambda: ra.ring_attn_fwd(q, k, v, cfg.P, causal=cfg.causal, layout=cfg.layout, scale=cfg.scale,
+                                      out=out, lse=lse)
+        work, unit = cfg.flops() / 1e12, "TFLOP/s"
+    else:
+        q, k, v, sl = W.decode_inputs(cfg, dev)
+        lens = sl.cpu().numpy().astype(np.int64)
+        ws = ra.decode_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.capacity, cfg.D, cfg.P, dev)
+        part = torch.empty((cfg.B, cfg.Hq, cfg.P, cfg.D), device=dev, dtype=torch.float32)
+        plse = torch.empty((cfg.B, cfg.Hq, cfg.P), device=dev, dtype=torch.float32)
+        fn = lambda: ra.ring_attn_decode_partial(q, k, v, sl, cfg.P, cfg.scale, partials=part, part_lse=plse,
+                                                 workspace=ws)
+        work, unit = decode_bytes(cfg, lens) / 1e9, "GB/s"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    print(json.dumps({"profile": name, "workload": cfg.name, "ms_per_launch": round(ms, 3),
+                      "rate": round(work / (ms / 1e3), 1), "unit": unit}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", choices=sorted(PROFILE_CASES), default=None,
+                    help="launch one kernel of the hot path on a profiling workload (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -375,6 +428,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     if args.warmup < 3:
         print("note: warm-up raised to 3 steps", file=sys.stderr)
         args.warmup = 3

@@ -286,8 +286,10 @@ ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile
   for (int qs = 0; qs < nch; ++qs) {
     const int r = chunk_owner(p, qs);
     // pairs: the visiting order of rank r, filtered by the causal rule on chunks
-    for (int idx = 0; idx < p.nkc; ++idx) {
-      const int ks = kv_slot(p, qs, idx);
+    KvIter it;
+    kv_begin(p, qs, it);
+    for (; it.idx < p.nkc; kv_next_chunk(p, it)) {
+      const int ks = kv_cur_slot(p, it);
       if (!p.causal || ks <= qs) {
         if (per_rank_pairs) per_rank_pairs[r]++;
       }

@@ -82,9 +82,11 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(Plan p, const T* __restr
 #pragma unroll
   for (int j = 0; j < D / 4; ++j) o[j] = 0.f;
 
-  KvIter it{0, 0};
+  KvIter it;
+  kv_begin(p, qslot, it);
   KvTile t;
-  while (kv_next(p, qslot, qhi, BK, it, t)) {
+  const int tpc = cdiv(p.C, BK);
+  while (kv_next(p, qhi, BK, tpc, it, t)) {
     __syncthreads();
     for (int e = tid; e < BK * D; e += 256) {
       const int kk = e / D, d = e - kk * D;

@@ -53,6 +53,8 @@ constexpr int THREADS = 384;
 constexpr int SLAB = 128 * 64 * 2;   // one 128-row x 64-column bf16 box (16 KB, 128-byte swizzle)
 constexpr float LAZY = 8.f;
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int REG_LOW = 96, REG_HIGH = 184;
+constexpr int REG_NEED = (128 * REG_LOW + 256 * REG_HIGH + THREADS - 1) / THREADS;   // per thread at launch
 }  // namespace tc
 
 template <int D>
@@ -116,7 +118,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // Registers: the producer / MMA warpgroup needs few, the softmax warpgroups
+  // hold a 128-column score row each.  128*REG_LOW + 256*REG_HIGH must not
+  // exceed the 384 threads x registers the kernel was launched with (checked
+  // by the launcher before every launch).
 
+  if (warp < 4) {
+  setmaxnreg_dec<REG_LOW>();
   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
@@ -125,6 +133,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       tma_prefetch_desc(&tmV);
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
+      const int tpc = cdiv(p.C, BN);
       uint32_t kv_cnt = 0, n_items = 0;
       bool ok = true;
       for (int L = blockIdx.x; L < space.count && ok; L += gridDim.x, ++n_items) {
@@ -138,9 +147,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         for (int i = 0; i < 2; ++i)
           for (int sl = 0; sl < D / 64; ++sl)
             tma_load_4d(smem_u32(sm.q[i]) + sl * SLAB, &tmQ, qb, sl * 64, it.h[i], it.qrow0[i], it.b, pol_q);
-        KvIter iter{0, 0};
+        KvIter iter;
+        kv_begin(p, it.qslot, iter);
         KvTile t;
-        while (ok && kv_next(p, it.qslot, it.qhi, BN, iter, t)) {
+        while (ok && kv_next(p, it.qhi, BN, tpc, iter, t)) {
           for (int kind = 0; kind < 2; ++kind) {
             const int s = kv_cnt % NST;
             if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((kv_cnt / NST) & 1u) ^ 1u, abort_flag, kWaitKvEmpty, err)) {
@@ -168,22 +178,28 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
       const uint32_t tS[2] = {tmem, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      // descriptors built once; per MMA only a constant is added to the start address
+      const uint64_t dq[2] = {sw128_desc(smem_u32(sm.q[0]), 16, 1024), sw128_desc(smem_u32(sm.q[1]), 16, 1024)};
+      const uint64_t dk0 = sw128_desc(smem_u32(sm.kv[0]), 16, 1024);     // K tile, K-major
+      const uint64_t dv0 = sw128_desc(smem_u32(sm.kv[0]), SLAB, 1024);   // V tile, MN-major
+      constexpr uint32_t STAGE16 = (BN * D * 2) >> 4;                    // stage stride, 16-byte units
+      const int tpc = cdiv(p.C, BN);
       uint32_t kv_cnt = 0, n_items = 0, tiles_done = 0;
       bool ok = true;
 
-      auto issue_S = [&](int i, int s) {
-        const uint32_t qa = smem_u32(sm.q[i]), kb = smem_u32(sm.kv[s]);
+      auto issue_S = [&](int i, uint32_t s) {
+        const uint64_t a = dq[i], b = dk0 + s * STAGE16;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k / 4) * SLAB + (k % 4) * 32;
-          mma_ss(tS[i], sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_qk, k > 0);
+          const uint32_t off = ((k / 4) * SLAB + (k % 4) * 32) >> 4;
+          mma_ss(tS[i], a + off, b + off, idesc_qk, k > 0);
         }
       };
-      auto issue_PV = [&](int i, int s, bool acc) {
-        const uint32_t vb = smem_u32(sm.kv[s]);
+      auto issue_PV = [&](int i, uint32_t s, bool acc) {
+        const uint64_t b = dv0 + s * STAGE16;
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
-          mma_ts(tO[i], tS[i] + k * 8, sw128_desc(vb + k * 16 * 128, SLAB, 1024), idesc_pv, (acc || k > 0) ? 1u : 0u);
+          mma_ts(tO[i], tS[i] + k * 8, b + k * ((16 * 128) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
       };
       auto wait_stage = [&](uint32_t c) -> bool {
         if (!mbar_wait(smem_u32(&sm.kv_full[c % NST]), (c / NST) & 1u, abort_flag, kWaitKvFull, err)) return false;
@@ -193,16 +209,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 
       for (int L = blockIdx.x; L < space.count && ok; L += gridDim.x, ++n_items) {
         const Item it = item_at(p, space, BM, L);
+        const int n = kv_count(p, it.qslot, it.qhi, BN, tpc);
         if (!mbar_wait(smem_u32(&sm.q_full), n_items & 1u, abort_flag, kWaitQFull, err)) { ok = false; break; }
         tc_fence_after();
-        KvIter iter{0, 0};
-        KvTile t;
-        if (!kv_next(p, it.qslot, it.qhi, BN, iter, t)) {
+        if (n == 0) {
           mma_commit(smem_u32(&sm.q_empty));
           continue;
         }
         // S0(0), S1(0)
-        uint32_t sK = kv_cnt;
+        const uint32_t sK = kv_cnt;
         if (!wait_stage(sK)) { ok = false; break; }
         issue_S(0, sK % NST);
         mma_commit(smem_u32(&sm.s_full[0]));
@@ -210,10 +225,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         mma_commit(smem_u32(&sm.s_full[1]));
         mma_commit(smem_u32(&sm.kv_empty[sK % NST]));
         ++kv_cnt;
-        uint32_t j = 0;
-        for (;;) {
-          KvTile tn;
-          const bool has_next = kv_next(p, it.qslot, it.qhi, BN, iter, tn);
+        for (int j = 0; j < n; ++j) {
+          const bool has_next = j + 1 < n;
           const uint32_t sV = kv_cnt++;
           if (!wait_stage(sV)) { ok = false; break; }
           if (!mbar_wait(smem_u32(&sm.p_full[0]), (tiles_done + j) & 1u, abort_flag, kWaitPFull, err)) {
@@ -244,18 +257,18 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             mma_commit(smem_u32(&sm.kv_empty[sKn % NST]));
             ++kv_cnt;
           }
-          ++j;
-          if (!has_next) break;
         }
         if (!ok) break;
-        tiles_done += j;
+        tiles_done += n;
         mma_commit(smem_u32(&sm.q_empty));
       }
       // every MMA issued so far must be complete before tensor memory is freed
       mma_commit(smem_u32(&sm.teardown));
       mbar_wait(smem_u32(&sm.teardown), 0, nullptr, kWaitTeardown, err);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<REG_HIGH>();
     // ================================================================ softmax groups
     const int i = (warp - 4) >> 2;                 // query tile of this group
     const int wi = warp & 3;                       // tensor-memory lane quarter
@@ -264,6 +277,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const uint32_t tS = tmem + lane_off + i * 128;
     const uint32_t tO = tmem + lane_off + 256 + i * D;
     const float sl2 = prm.scale_log2;
+    const int tpc = cdiv(p.C, BN);
     uint32_t tiles_done = 0, items_with_tiles = 0;
     unsigned long long cnt_full = 0, cnt_part = 0;
     bool ok = true;
@@ -277,10 +291,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       // l: fp32 sum of p (gives lse); lt: sum of the bf16-rounded p that the PV
       // product actually used (normalises O, so the weights applied to V sum to 1)
       float m_run = -CUDART_INF_F, m_max = -CUDART_INF_F, l = 0.f, lt = 0.f;
-      KvIter iter{0, 0};
+      KvIter iter;
+      kv_begin(p, it.qslot, iter);
       KvTile t;
       uint32_t j = 0;
-      while (kv_next(p, it.qslot, it.qhi, BN, iter, t)) {
+      while (kv_next(p, it.qhi, BN, tpc, iter, t)) {
         if (prm.a.counters && row == 0 && nrows > 0) {
           const int cls = tile_class(p.causal, q0, q1, t.pos0, t.pos0 + t.nvalid - 1);
           if (cls == 0) ++cnt_full;
@@ -311,31 +326,51 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= t.nvalid || c > lim_causal) s[c] = -CUDART_INF_F;
         }
-        float mx = s[0];
+        // Row max first, then the exponentials against the (lazily moved) base.
+        const uint64_t sl2x2 = pack2(sl2, sl2);
+        float alpha = 1.f, rs = 0.f, rt = 0.f, mxs;
+        auto exp_pass = [&](float base) {
+          const uint64_t nbase2 = pack2(-base, -base);
+          uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull}, rt2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-        const float mxs = mx * sl2;
-        m_max = fmaxf(m_max, mxs);
-        float alpha = 1.f;
-        if (mxs > m_run + LAZY) {
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a0 = s[c * 32 + 2 * e], a1 = s[c * 32 + 2 * e + 1];
+              float x0, x1;
+              unpack2(ffma2(pack2(a0, a1), sl2x2, nbase2), x0, x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              rs2[e & 3] = fadd2(rs2[e & 3], pack2(p0, p1));
+              pk[e] = pack_bf16x2(p0, p1);
+              rt2[e & 3] = fadd2(rt2[e & 3], pack2(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xffff0000u)));
+            }
+            tmem_st16(tS + c * 16, pk);
+          }
+          rs = hsum2(fadd2(fadd2(rs2[0], rs2[1]), fadd2(rs2[2], rs2[3])));
+          rt = hsum2(fadd2(fadd2(rt2[0], rt2[1]), fadd2(rt2[2], rt2[3])));
+        };
+        auto row_max = [&]() -> float {
+          float mq[4];
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const float* sc = s + ch * 32;
+            float x = fmax3(sc[0], sc[1], sc[2]);
+#pragma unroll
+            for (int e = 3; e < 31; e += 2) x = fmax3(x, sc[e], sc[e + 1]);
+            mq[ch] = fmaxf(x, sc[31]);
+          }
+          return fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]);
+        };
+        // (exp_pass stores to tensor memory with warp-collective instructions; it
+        // runs unconditionally, by the whole warp)
+        mxs = row_max() * sl2;
+        if (mxs > m_run + LAZY) {   // always for a row without a base yet (m_run = -inf)
           alpha = (m_run == -CUDART_INF_F) ? 0.f : ex2(m_run - mxs);
           m_run = mxs;
         }
-        const float base = (m_run == -CUDART_INF_F) ? 0.f : m_run;
-        float rs = 0.f, rt = 0.f;
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(s[c * 32 + 2 * e], sl2, -base));
-            const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], sl2, -base));
-            rs += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-            rt += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
-          }
-          tmem_st16(tS + c * 16, pk);
-        }
+        exp_pass(m_run == -CUDART_INF_F ? 0.f : m_run);
+        m_max = fmaxf(m_max, mxs);
         l = l * alpha + rs;
         lt = lt * alpha + rt;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -471,6 +506,12 @@ static cudaError_t launch_tc_d(const Plan& p, const TcArgs& a, cudaStream_t st) 
   auto kern = attn_tc_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // the in-kernel register split needs this many registers per thread at launch;
+  // with fewer, setmaxnreg.inc would wait forever, so refuse instead
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs < tc::REG_NEED) return cudaErrorNotSupported;
   const int grid = prm.space.count < num_sms() ? prm.space.count : num_sms();
   kern<<<grid, tc::THREADS, smem, st>>>(tq, tk, tv, prm);
   return cudaGetLastError();

@@ -6,16 +6,19 @@
 // of one chunk.  A persistent grid (one CTA per SM) walks the units in chunk
 // order, so the always-full early chunks come first and the ragged tails of
 // the sequences last.  Per CTA:
-//   warp 0      TMA producer: 64-row K and V boxes into a 5-stage ring of
-//               shared memory (bounded waits on the stage barriers);
-//   warps 1..8  consumers: 32 groups of 8 lanes, each group owns two rows of a
-//               stage; a lane holds 16 of the 128 dims of the G query heads of
-//               the kv head (scaled by scale*log2 e), computes partial dot
-//               products, reduces them inside its group with shuffles, and
-//               folds the rows into a running (m, l, O) -- the online-softmax
-//               update of "Lesson 8: Context Parallelism", section 3 -- keeping
-//               a stale max until a score exceeds it by 2^8 (exact: the same
-//               base scales l and O).
+//   warp 0       TMA producer: 96-row K and V boxes into a 4-stage ring of
+//                shared memory (bounded waits on the stage barriers);
+//   warps 1..12  consumers: a half warp owns one K/V row per pass; a lane
+//                holds 8 of the 128 dims of every query head of the kv head
+//                (scaled by scale*log2 e), so each K/V element is widened to
+//                fp32 once; partial dot products (packed f32x2 FMA) are
+//                reduced by a transposing half-warp butterfly that leaves each
+//                lane the score of one head; that head's lanes fold the row
+//                into the running (m, l) -- the online-softmax update of
+//                "Lesson 8: Context Parallelism", section 3 -- keeping a stale
+//                max until a score exceeds it by 2^8 (exact: the same base
+//                scales l and O), and broadcast the weight to the other lanes
+//                for the PV update.
 // At the end of a unit the 32 group states are folded (shuffles, then shared
 // memory).  A chunk covered by one sub-split writes its partial directly;
 // otherwise every sub-split writes to the workspace and the last CTA to
@@ -32,12 +35,14 @@ namespace ra {
 
 namespace dec {
 constexpr int D = 128;
-constexpr int ROWS = 64;                    // rows per stage
-constexpr int NST = 5;                      // stages
-constexpr int RPS = 4096;                   // rows per sub-split
+constexpr int ROWS = 96;                    // rows per stage
+constexpr int NST = 4;                      // stages
+constexpr int RPS = 4032;                   // rows per sub-split (a multiple of ROWS)
 constexpr int STAGE_BYTES = 2 * ROWS * D * 2;
-constexpr int NCW = 8;                      // consumer warps
+constexpr int NCW = 12;                     // consumer warps
 constexpr int THREADS = 32 * (1 + NCW);
+static_assert(ROWS % (2 * NCW) == 0, "a stage is covered by whole passes of all consumer warps");
+static_assert(RPS % ROWS == 0, "stages never straddle two sub-splits");
 constexpr float LAZY = 8.f;                 // log2 of the largest tolerated growth before rescaling
 }  // namespace dec
 
@@ -54,6 +59,59 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float* f) {
     f[2 * i] = __uint_as_float(u[i] << 16);
     f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
   }
+}
+
+// 8 bf16 -> 4 packed pairs of float (exact widening)
+__device__ __forceinline__ void bf16x8_to_f32x2(const uint4 w, uint64_t* f2) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f2[i] = pack2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
+}
+
+// Sum over the 16 lanes of a half warp of G per-head partial sums, leaving
+// in every lane the full sum of one head, own_head(lane).  Transposing
+// butterfly: at each of the first log2(G) levels a lane keeps half of its
+// values and sends the other half, so G values need log2(G) + 4 - log2(G)
+// ... i.e. (G - 1) + (4 - log2 G) shuffles instead of 4 * G.
+template <int G>
+__device__ __forceinline__ float half_warp_transpose_sum(const float (&v)[G], int lane) {
+  if constexpr (G == 4) {
+    const bool hi = (lane >> 3) & 1;   // keeps heads {2,3} if set, else {0,1}
+    float k0 = (hi ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[2], 8);
+    float k1 = (hi ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, hi ? v[1] : v[3], 8);
+    const bool odd = (lane >> 2) & 1;  // keeps the odd head of the pair if set
+    float x = (odd ? k1 : k0) + __shfl_xor_sync(0xffffffffu, odd ? k0 : k1, 4);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    return x;
+  } else if constexpr (G == 2) {
+    const bool hi = (lane >> 3) & 1;
+    float x = (hi ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[1], 8);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    return x;
+  } else {
+    float x = v[0];
+#pragma unroll
+    for (int off = 8; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+  }
+}
+
+// The head whose full sum half_warp_transpose_sum leaves in `lane`, and the
+// lane (of the same half warp) holding head h.
+template <int G>
+__device__ __forceinline__ int own_head(int lane) {
+  if constexpr (G == 4) return ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+  else if constexpr (G == 2) return (lane >> 3) & 1;
+  else return 0;
+}
+template <int G>
+__device__ __forceinline__ int head_lane(int lane, int h) {
+  if constexpr (G == 4) return (lane & 16) | ((h >> 1) << 3) | ((h & 1) << 2);
+  else if constexpr (G == 2) return (lane & 16) | (h << 3);
+  else return lane & 16;
 }
 
 template <int G>
@@ -128,13 +186,22 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
   }
 
   // -------------------------------------------------------------- consumers
-  const int cw = warp - 1;                 // consumer warp 0..7
-  const int ctid = threadIdx.x - 32;       // 0..255
-  const int grp = lane >> 3, j = lane & 7;
-  const int gidx = cw * 4 + grp;           // row group 0..31 -> rows gidx, gidx + 32 of a stage
+  // Lane layout: each half warp (16 lanes) owns one K/V row per pass; lane
+  // (dh, j) holds dims [dh*64 + 8j, dh*64 + 8j + 8) of every one of the G
+  // query heads and of their output rows (the 16 lanes read the row's 256
+  // contiguous bytes).  Per row: partial dot products, a transposing
+  // half-warp reduction that leaves each lane the full score of one head,
+  // the online-softmax update done by that head's lanes, and a broadcast of
+  // the G weights p_h for the PV update.  Each K/V element is widened once.
+  const int cw = warp - 1;                 // consumer warp 0..NCW-1
+  const int ctid = threadIdx.x - 32;       // 0..32*NCW-1
+  const int half = lane >> 4;
+  const int dcol = ((lane >> 3) & 1) * 64 + (lane & 7) * 8;   // first dim of this lane
+  const int oh = own_head<G>(lane);
   const float qscale = a.scale * 1.4426950408889634f;
   uint32_t cnt = 0;
   const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(a.q);
+  constexpr int CT = 32 * NCW;
 
   for (int u = blockIdx.x; u < geo.units; u += gridDim.x) {
     int t = u;
@@ -151,7 +218,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
 
     if (nvalid_chunk == 0) {
       if (sub == 0) {
-        for (int e = ctid; e < G * D; e += 256) {
+        for (int e = ctid; e < G * D; e += CT) {
           const int h = e / D, d = e - h * D;
           a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = 0.f;
         }
@@ -161,26 +228,22 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     }
     if (r0 >= r1) continue;
 
-    // this lane's slice of the G query heads: dims [8j, 8j+8) and [64+8j, 64+8j+8)
-    float qf[G][16];
+    // this lane's 8 dims of the G query heads, scaled by scale * log2(e)
+    uint64_t q2[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const __nv_bfloat16* qh = qb + ((size_t)b * a.Hq + g * G + h) * D;
-      const uint4 w0 = *reinterpret_cast<const uint4*>(qh + 8 * j);
-      const uint4 w1 = *reinterpret_cast<const uint4*>(qh + 64 + 8 * j);
-      bf16x8_to_f32(w0, qf[h]);
-      bf16x8_to_f32(w1, qf[h] + 8);
+      float f[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + ((size_t)b * a.Hq + g * G + h) * D + dcol), f);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) qf[h][i] *= qscale;
+      for (int i = 0; i < 4; ++i) q2[h][i] = pack2(f[2 * i] * qscale, f[2 * i + 1] * qscale);
     }
-    float m[G], l[G], o[G][16];
+    // running state: m, l of head oh (this lane's owned head); O rows of all heads
+    float m = -CUDART_INF_F, l = 0.f;
+    uint64_t o2[G][4];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m[h] = -CUDART_INF_F;
-      l[h] = 0.f;
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o[h][i] = 0.f;
-    }
+      for (int i = 0; i < 4; ++i) o2[h][i] = 0ull;
 
     bool ok = true;
     for (int row = r0; row < r1 && ok; row += ROWS) {
@@ -189,119 +252,103 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, kWaitDecodeFull, a.err)) { ok = false; break; }
       const uint8_t* Ks = sm.stage[s];
       const uint8_t* Vs = Ks + ROWS * D * 2;
-      const bool vA = row + gidx < r1, vB = row + gidx + 32 < r1;
-      float kA[16], kB[16];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + gidx * 256 + 16 * j), kA);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + gidx * 256 + 128 + 16 * j), kA + 8);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + (gidx + 32) * 256 + 16 * j), kB);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Ks + (gidx + 32) * 256 + 128 + 16 * j), kB + 8);
-      float sA[G], sB[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float x = 0.f, y = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          x = fmaf(qf[h][i], kA[i], x);
-          y = fmaf(qf[h][i], kB[i], y);
-        }
-        sA[h] = x;
-        sB[h] = y;
-      }
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) {
+      for (int pass = 0; pass < ROWS / (2 * NCW); ++pass) {
+        const int rr = pass * 2 * NCW + cw * 2 + half;
+        const bool valid = row + rr < r1;
+        uint64_t x2[4];
+        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Ks + rr * 256 + dcol * 2), x2);
+        float part[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          sA[h] += __shfl_xor_sync(0xffffffffu, sA[h], off);
-          sB[h] += __shfl_xor_sync(0xffffffffu, sB[h], off);
+          const uint64_t acc = ffma2(q2[h][1], x2[1], ffma2(q2[h][0], x2[0], 0ull));
+          part[h] = hsum2(ffma2(q2[h][3], x2[3], ffma2(q2[h][2], x2[2], acc)));
+        }
+        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Vs + rr * 256 + dcol * 2), x2);
+        float sc = half_warp_transpose_sum<G>(part, lane);
+        if (!valid) sc = -CUDART_INF_F;
+        const bool moved = sc > m + LAZY;
+        if (__any_sync(0xffffffffu, moved)) {
+          float f = 1.f;
+          if (moved) {
+            f = (m == -CUDART_INF_F) ? 0.f : ex2(m - sc);
+            m = sc;
+            l *= f;
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float fh = __shfl_sync(0xffffffffu, f, head_lane<G>(lane, h));
+            const uint64_t f2 = pack2(fh, fh);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o2[h][i] = fmul2(o2[h][i], f2);
+          }
+        }
+        const float pw = (valid && m != -CUDART_INF_F) ? ex2(sc - m) : 0.f;
+        l += pw;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float ph_ = __shfl_sync(0xffffffffu, pw, head_lane<G>(lane, h));
+          const uint64_t p2 = pack2(ph_, ph_);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o2[h][i] = ffma2(p2, x2[i], o2[h][i]);
         }
       }
-      float vAf[16], vBf[16];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + gidx * 256 + 16 * j), vAf);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + gidx * 256 + 128 + 16 * j), vAf + 8);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + (gidx + 32) * 256 + 16 * j), vBf);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(Vs + (gidx + 32) * 256 + 128 + 16 * j), vBf + 8);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));   // this warp is done with the stage
       ++cnt;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        if (!vA) sA[h] = -CUDART_INF_F;
-        if (!vB) sB[h] = -CUDART_INF_F;
-        const float smax = fmaxf(sA[h], sB[h]);
-        if (smax > m[h] + LAZY) {
-          const float f = (m[h] == -CUDART_INF_F) ? 0.f : ex2(m[h] - smax);
-          l[h] *= f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[h][i] *= f;
-          m[h] = smax;
-        }
-        const bool live = m[h] != -CUDART_INF_F;
-        const float pA = (live && vA) ? ex2(sA[h] - m[h]) : 0.f;
-        const float pB = (live && vB) ? ex2(sB[h] - m[h]) : 0.f;
-        l[h] += pA + pB;
-        if (vA) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[h][i] = fmaf(pA, vAf[i], o[h][i]);
-        }
-        if (vB) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[h][i] = fmaf(pB, vBf[i], o[h][i]);
-        }
-      }
     }
     // (after an expired wait the unit still runs through every named barrier
     // below, so that all consumer warps leave the loop together)
 
-    // fold the 4 groups of this warp (lanes with equal j hold the same dims)
-#pragma unroll
-    for (int off = 8; off < 32; off <<= 1) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
-        const float mc = fmaxf(m[h], mo);
-        const float f = (m[h] == -CUDART_INF_F) ? 0.f : ex2(m[h] - mc);
-        l[h] *= f;
-        l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          o[h][i] *= f;
-          o[h][i] += __shfl_xor_sync(0xffffffffu, o[h][i], off);
-        }
-        m[h] = mc;
-      }
-    }
-    if (grp == 0) {
+    // fold the two half warps (same heads and dims, different rows)
+    {
+      const float mc = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      const float f = (m == -CUDART_INF_F) ? 0.f : ex2(m - mc);
+      l *= f;
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      m = mc;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
+        const float fh = __shfl_sync(0xffffffffu, f, head_lane<G>(lane, h));
+        const uint64_t f2 = pack2(fh, fh);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          sm.wpart[cw][h][8 * j + i] = o[h][i];
-          sm.wpart[cw][h][64 + 8 * j + i] = o[h][8 + i];
-        }
-        if (j == 0) {
-          sm.wm[cw][h] = m[h];
-          sm.wl[cw][h] = l[h];
+        for (int i = 0; i < 4; ++i) {
+          float x, y;
+          unpack2(fmul2(o2[h][i], f2), x, y);
+          x += __shfl_xor_sync(0xffffffffu, x, 16);
+          y += __shfl_xor_sync(0xffffffffu, y, 16);
+          o2[h][i] = pack2(x, y);
         }
       }
     }
-    named_bar_sync(1, 256);
+    if (half == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) unpack2(o2[h][i], sm.wpart[cw][h][dcol + 2 * i], sm.wpart[cw][h][dcol + 2 * i + 1]);
+      if ((lane & 3) == 0) {
+        sm.wm[cw][oh] = m;
+        sm.wl[cw][oh] = l;
+      }
+    }
+    named_bar_sync(1, CT);
 
-    // fold the 8 warps: thread -> (head, dim) pairs; natural-log lse at the end
+    // fold the consumer warps: thread -> (head, dim) pairs; natural-log lse at the end
     float* ws_unit = a.ws_part + ((((size_t)(b * a.Hkv + g) * a.P + p) * geo.nsub + sub) * G) * (D + 1);
-    for (int e = ctid; e < G * D; e += 256) {
+    for (int e = ctid; e < G * D; e += CT) {
       const int h = e / D, d = e - h * D;
       float mx = -CUDART_INF_F;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, sm.wm[w][h]);
-      float L = 0.f, acc = 0.f;
+      float Lsum = 0.f, acc = 0.f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) {
         const float f = (sm.wm[w][h] == -CUDART_INF_F) ? 0.f : ex2(sm.wm[w][h] - mx);
-        L = fmaf(sm.wl[w][h], f, L);
+        Lsum = fmaf(sm.wl[w][h], f, Lsum);
         acc = fmaf(sm.wpart[w][h][d], f, acc);
       }
-      const float od = acc / L;
-      const float lse = (mx + log2f(L)) * 0.6931471805599453f;
+      const float od = acc / Lsum;
+      const float lse = (mx + log2f(Lsum)) * 0.6931471805599453f;
       if (n_live == 1) {
         a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = od;
         if (d == 0) a.part_lse[(size_t)(b * a.Hq + g * G + h) * a.P + p] = lse;
@@ -312,7 +359,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     }
     if (n_live > 1) {
       __threadfence();
-      named_bar_sync(1, 256);
+      named_bar_sync(1, CT);
       if (ctid == 0) {
         unsigned int* ctr = a.ws_count + (size_t)(b * a.Hkv + g) * a.P + p;
         const unsigned int old = atomicAdd(ctr, 1u);
@@ -320,28 +367,28 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         if (last) atomicExch(ctr, 0u);       // leave the counter at zero for the next call
         sm.is_last = last;
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, CT);
       if (sm.is_last) {
         __threadfence();
         const float* ws_chunk = a.ws_part + (((size_t)(b * a.Hkv + g) * a.P + p) * geo.nsub) * G * (D + 1);
-        for (int e = ctid; e < G * D; e += 256) {
+        for (int e = ctid; e < G * D; e += CT) {
           const int h = e / D, d = e - h * D;
           float mx = -CUDART_INF_F;
           for (int s2 = 0; s2 < n_live; ++s2) mx = fmaxf(mx, __ldcg(ws_chunk + (s2 * G + h) * (D + 1) + D));
-          float L = 0.f, acc = 0.f;
+          float Lsum = 0.f, acc = 0.f;
           for (int s2 = 0; s2 < n_live; ++s2) {
             const float* r = ws_chunk + (s2 * G + h) * (D + 1);
             const float w = expf(__ldcg(r + D) - mx);
-            L += w;
+            Lsum += w;
             acc = fmaf(w, __ldcg(r + d), acc);
           }
-          a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = acc / L;
-          if (d == 0) a.part_lse[(size_t)(b * a.Hq + g * G + h) * a.P + p] = mx + logf(L);
+          a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = acc / Lsum;
+          if (d == 0) a.part_lse[(size_t)(b * a.Hq + g * G + h) * a.P + p] = mx + logf(Lsum);
         }
       }
     }
     // shared fold buffers are free again; leave together if any wait expired
-    if (named_bar_any(1, 256, !ok || *abort_flag)) break;
+    if (named_bar_any(1, CT, !ok || *abort_flag)) break;
   }
 }
 

@@ -62,40 +62,53 @@ RA_HD int rank_chunk(const Plan& p, int r, int j) {
 RA_HD int q_gid(const Plan& p, int slot) { return p.mode == kModeRing ? slot : p.qid[slot]; }
 RA_HD int kv_gid(const Plan& p, int slot) { return p.mode == kModeRing ? slot : p.kid[slot]; }
 
-// idx-th K/V slot visited by queries of Q slot `qslot`: ring order of the
-// owning rank in ring mode, buffer order in step mode.
-RA_HD int kv_slot(const Plan& p, int qslot, int idx) {
-  if (p.mode == kModeStep) return idx;
-  const int r = chunk_owner(p, qslot);
-  const int cpr = chunks_per_rank(p);
-  const int t = idx / cpr, j = idx - t * cpr;
-  int src = (r - t) % p.P;
-  if (src < 0) src += p.P;
-  return rank_chunk(p, src, j);
-}
-
 // One K/V tile: rows [row0, row0 + nvalid) of the K/V buffer, global
 // positions [pos0, pos0 + nvalid), chunk slot and global chunk id.
 struct KvTile {
   int row0, pos0, nvalid, slot, gid, first_in_chunk;
 };
 
+// Walks the K/V chunks met by the queries of one Q chunk, in the owning
+// rank's ring order (ring mode) or in buffer order (step mode), and the
+// tiles inside each chunk.  Incremental: no division per step.
 struct KvIter {
-  int idx, kt;
+  int idx;  // visited chunk index, 0 .. nkc-1
+  int kt;   // next tile inside the current chunk
+  int src;  // ring mode: the rank whose K/V block is held at this step
+  int j;    // ring mode: which of that rank's chunks
 };
 
-// Next K/V tile (of BN keys) for queries whose last valid global position is
-// qhi.  Tiles entirely after qhi are skipped when causal.
-RA_HD bool kv_next(const Plan& p, int qslot, int qhi, int BN, KvIter& it, KvTile& t) {
-  const int tiles = cdiv(p.C, BN);
+RA_HD void kv_begin(const Plan& p, int qslot, KvIter& it) {
+  it.idx = 0;
+  it.kt = 0;
+  it.j = 0;
+  it.src = p.mode == kModeRing ? chunk_owner(p, qslot) : 0;   // step 0: the rank's own block
+}
+
+RA_HD int kv_cur_slot(const Plan& p, const KvIter& it) {
+  return p.mode == kModeStep ? it.idx : rank_chunk(p, it.src, it.j);
+}
+
+RA_HD void kv_next_chunk(const Plan& p, KvIter& it) {
+  it.idx++;
+  it.kt = 0;
+  if (p.mode == kModeRing && ++it.j == chunks_per_rank(p)) {
+    it.j = 0;
+    it.src = it.src == 0 ? p.P - 1 : it.src - 1;   // next step: the block of rank (src - 1) mod P
+  }
+}
+
+// Next K/V tile (of BN keys; tpc = tiles per chunk) for queries whose last
+// valid global position is qhi.  Tiles entirely after qhi are skipped when
+// causal.
+RA_HD bool kv_next(const Plan& p, int qhi, int BN, int tpc, KvIter& it, KvTile& t) {
   while (it.idx < p.nkc) {
-    const int slot = kv_slot(p, qslot, it.idx);
+    const int slot = kv_cur_slot(p, it);
     const int gid = kv_gid(p, slot);
     const int k0 = it.kt * BN;
     const int pos0 = gid * p.C + k0;
-    if (it.kt >= tiles || (p.causal && pos0 > qhi)) {
-      it.idx++;
-      it.kt = 0;
+    if (it.kt >= tpc || (p.causal && pos0 > qhi)) {
+      kv_next_chunk(p, it);
       continue;
     }
     t.row0 = slot * p.C + k0;
@@ -108,6 +121,22 @@ RA_HD bool kv_next(const Plan& p, int qslot, int qhi, int BN, KvIter& it, KvTile
     return true;
   }
   return false;
+}
+
+// Number of tiles kv_next yields for these queries (one step per chunk).
+RA_HD int kv_count(const Plan& p, int qslot, int qhi, int BN, int tpc) {
+  KvIter it;
+  kv_begin(p, qslot, it);
+  int n = 0;
+  for (; it.idx < p.nkc; kv_next_chunk(p, it)) {
+    const int cpos = kv_gid(p, kv_cur_slot(p, it)) * p.C;
+    if (!p.causal) {
+      n += tpc;
+    } else if (cpos <= qhi) {
+      n += imin(tpc, (qhi - cpos) / BN + 1);
+    }
+  }
+  return n;
 }
 
 // Q slots ordered by decreasing global chunk id (longest work first).
