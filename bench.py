@@ -121,12 +121,19 @@ def barrier(dist):
         dist.barrier()
 
 
-def max_over_ranks(dist, x: float) -> float:
+def max_over_ranks(dist, x: float, device="cuda") -> float:
+    """The largest x over all ranks (timings are taken as the max over ranks)."""
     if dist is None:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(work_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job rate of `world` independent replicas, each doing `steps` steps
+    of `work_per_step`, timed as the max over ranks."""
+    return work_per_step * steps * world / (max_ms / 1e3)
 
 
 # --------------------------------------------------------------------------- the hot path
@@ -206,9 +213,9 @@ def run_ours(args):
     dec_sum = max_over_ranks(dist, sum(dec_ms))
 
     flops = cfg.flops()
-    value = flops * args.steps * world / (pre_sum / 1e3) / 1e12          # causal-adjusted TFLOP/s, all ranks
+    value = replica_throughput(flops, args.steps, world, pre_sum) / 1e12     # causal-adjusted TFLOP/s, all ranks
     dbytes = decode_bytes(dcfg, lens)
-    dvalue = dbytes * args.steps * world / (dec_sum / 1e3) / 1e9         # GB/s, all ranks
+    dvalue = replica_throughput(dbytes, args.steps, world, dec_sum) / 1e9    # GB/s, all ranks
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -294,12 +301,28 @@ def run_ours(args):
 
 
 def load_traffic():
-    """DRAM bytes per launch from the committed ncu summary (None if absent)."""
+    """DRAM bytes per launch of each kernel from the committed ncu summary
+    (profiles/traffic.json).  An entry whose kernel sources changed since the
+    counters were taken is reported as None."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(path):
-        with open(path) as f:
-            return json.load(f)
-    return {}
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        d = json.load(f)
+    out = {}
+    for k, e in d.items():
+        if not isinstance(e, dict):
+            continue
+        m = hashlib.sha256()
+        try:
+            for src in e["sources"]:
+                with open(os.path.join(ROOT, src), "rb") as g:
+                    m.update(g.read())
+        except OSError:
+            continue
+        out[k] = e["bytes"] if m.hexdigest()[:16] == e["source_sha256"] else None
+    return out
 
 
 # --------------------------------------------------------------------------- oracle on the host cores

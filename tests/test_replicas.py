@@ -1,0 +1,63 @@
+"""Multi-GPU runs of bench.py are independent replicas (no collective on the
+data path); only the timing is aggregated across ranks.  This checks that
+aggregation with two gloo ranks on the CPU: the max over ranks and the
+whole-job rate."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        local_ms = [120.0, 150.0][rank]
+        mx = bench.max_over_ranks(dist, local_ms, device="cpu")
+        rate = bench.replica_throughput(1.0e12, 4, world, mx)
+        q.put((rank, mx, rate))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_replicas_max_and_rate():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for _, mx, rate in res:
+        assert mx == 150.0                                  # max over ranks
+        assert rate == pytest.approx(1.0e12 * 4 * 2 / 0.150)  # all ranks' work / slowest rank's time
+
+
+def test_single_process_is_identity():
+    assert bench.max_over_ranks(None, 3.5) == 3.5
+    assert bench.replica_throughput(2.0, 3, 1, 1000.0) == pytest.approx(6.0)
+
+
+def test_cpu_baseline_small_sample():
+    import workloads as W
+    cfg = W.Prefill("tiny", "bf16", True, "zigzag", 1, 2, 1, 512, 64, 2, 3)
+    r = bench.cpu_baseline(cfg, seconds=0.2)
+    assert r["kind"] == "oracle" and r["cores"] >= 1 and r["value"] > 0 and r["unit"] == "TFLOP/s"
