@@ -30,9 +30,10 @@
 //   m_new = max(m, max_j x_j); the base m is only moved when m_new exceeds it
 //   by more than 8 (a factor 256), in which case l and the O row are rescaled
 //   by 2^(m - m_new) in place; p_j = 2^(x_j - m) is written as bf16 for the PV
-//   product, l += sum p_j in fp32 and lt += sum bf16(p_j).  Using a stale base
-//   is exact: l, lt and O share it.  out = O / lt (the weights that multiplied
-//   V sum to one), lse = (m + log2 l) * ln 2.
+//   product and l += sum p_j in fp32.  lt is l corrected by the bf16 rounding
+//   of each tile's largest weight (the error that does not average out when
+//   one key dominates).  Using a stale base is exact: l, lt and O share it.
+//   out = O / lt, lse = (m + log2 l) * ln 2.
 // Every wait is bounded; a wait that expires flags the device error word and
 // all roles unwind, let in-flight copies and MMAs finish, and free tensor
 // memory before the CTA exits.
@@ -178,33 +179,36 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
       const uint32_t tS[2] = {tmem, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
-      // descriptors built once; per MMA only a constant is added to the start address
-      const uint64_t dq[2] = {sw128_desc(smem_u32(sm.q[0]), 16, 1024), sw128_desc(smem_u32(sm.q[1]), 16, 1024)};
-      const uint64_t dk0 = sw128_desc(smem_u32(sm.kv[0]), 16, 1024);     // K tile, K-major
-      const uint64_t dv0 = sw128_desc(smem_u32(sm.kv[0]), SLAB, 1024);   // V tile, MN-major
-      constexpr uint32_t STAGE16 = (BN * D * 2) >> 4;                    // stage stride, 16-byte units
+      // descriptors built once: per MMA only a constant is added to a 32-bit low word
+      const uint32_t hi = (uint32_t)(sw128_desc(0, 16, 1024) >> 32);   // same for K- and MN-major here
+      const uint32_t lq[2] = {(uint32_t)sw128_desc(smem_u32(sm.q[0]), 16, 1024),
+                              (uint32_t)sw128_desc(smem_u32(sm.q[1]), 16, 1024)};
+      const uint32_t lk0 = (uint32_t)sw128_desc(smem_u32(sm.kv[0]), 16, 1024);     // K tile, K-major
+      const uint32_t lv0 = (uint32_t)sw128_desc(smem_u32(sm.kv[0]), SLAB, 1024);   // V tile, MN-major
+      constexpr uint32_t STAGE16 = (BN * D * 2) >> 4;                             // stage stride, 16-byte units
       const int tpc = cdiv(p.C, BN);
       uint32_t kv_cnt = 0, n_items = 0, tiles_done = 0;
       bool ok = true;
 
       auto issue_S = [&](int i, uint32_t s) {
-        const uint64_t a = dq[i], b = dk0 + s * STAGE16;
+        const uint32_t a = lq[i], b = lk0 + s * STAGE16;
+        mma_ss_lo_first(tS[i], a, b, hi, idesc_qk);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 1; k < D / 16; ++k) {
           const uint32_t off = ((k / 4) * SLAB + (k % 4) * 32) >> 4;
-          mma_ss(tS[i], a + off, b + off, idesc_qk, k > 0);
+          mma_ss_lo(tS[i], a + off, b + off, hi, idesc_qk);
         }
       };
       auto issue_PV = [&](int i, uint32_t s, bool acc) {
-        const uint64_t b = dv0 + s * STAGE16;
+        const uint32_t b = lv0 + s * STAGE16;
+        mma_ts_lo_pred(tO[i], tS[i], b, hi, idesc_pv, acc ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          mma_ts(tO[i], tS[i] + k * 8, b + k * ((16 * 128) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
+        for (int k = 1; k < BN / 16; ++k) mma_ts_lo(tO[i], tS[i] + k * 8, b + k * ((16 * 128) >> 4), hi, idesc_pv);
       };
+      // K/V tiles are written by TMA (async proxy) and published by the mbarrier's
+      // transaction count; no tcgen05 fence is needed to read them.
       auto wait_stage = [&](uint32_t c) -> bool {
-        if (!mbar_wait(smem_u32(&sm.kv_full[c % NST]), (c / NST) & 1u, abort_flag, kWaitKvFull, err)) return false;
-        tc_fence_after();
-        return true;
+        return mbar_wait(smem_u32(&sm.kv_full[c % NST]), (c / NST) & 1u, abort_flag, kWaitKvFull, err);
       };
 
       for (int L = blockIdx.x; L < space.count && ok; L += gridDim.x, ++n_items) {
@@ -288,8 +292,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const int q0 = it.qpos0[i], q1 = it.qpos0[i] + nrows - 1;
       const int qpos = it.qpos0[i] + row;
       const int rank = p.mode == kModeRing ? chunk_owner(p, it.qslot) : 0;
-      // l: fp32 sum of p (gives lse); lt: sum of the bf16-rounded p that the PV
-      // product actually used (normalises O, so the weights applied to V sum to 1)
+      // l: fp32 sum of p (gives lse); lt: l corrected by the bf16 rounding of
+      // each tile's largest weight (normalises O; see exp_pass)
       float m_run = -CUDART_INF_F, m_max = -CUDART_INF_F, l = 0.f, lt = 0.f;
       KvIter iter;
       kv_begin(p, it.qslot, iter);
@@ -328,10 +332,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
         // Row max first, then the exponentials against the (lazily moved) base.
         const uint64_t sl2x2 = pack2(sl2, sl2);
-        float alpha = 1.f, rs = 0.f, rt = 0.f, mxs;
+        float alpha = 1.f, rs = 0.f, rt = 0.f, mxs, mx_raw;
         auto exp_pass = [&](float base) {
           const uint64_t nbase2 = pack2(-base, -base);
-          uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull}, rt2[4] = {0ull, 0ull, 0ull, 0ull};
+          uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t pk[16];
@@ -343,12 +347,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
               const float p0 = ex2(x0), p1 = ex2(x1);
               rs2[e & 3] = fadd2(rs2[e & 3], pack2(p0, p1));
               pk[e] = pack_bf16x2(p0, p1);
-              rt2[e & 3] = fadd2(rt2[e & 3], pack2(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xffff0000u)));
             }
             tmem_st16(tS + c * 16, pk);
           }
           rs = hsum2(fadd2(fadd2(rs2[0], rs2[1]), fadd2(rs2[2], rs2[3])));
-          rt = hsum2(fadd2(fadd2(rt2[0], rt2[1]), fadd2(rt2[2], rt2[3])));
+          // The PV product uses bf16(p).  When one key dominates a row, the rounding of
+          // its weight is the one error that does not average out; folding it into
+          // the normaliser makes the weights applied to V sum to one in that case.
+          const float pm = ex2(fmaf(mx_raw, sl2, -base));
+          rt = rs + (__uint_as_float(pack_bf16x2(pm, pm) & 0xffff0000u) - pm);
         };
         auto row_max = [&]() -> float {
           float mq[4];
@@ -364,7 +371,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         };
         // (exp_pass stores to tensor memory with warp-collective instructions; it
         // runs unconditionally, by the whole warp)
-        mxs = row_max() * sl2;
+        mx_raw = row_max();
+        mxs = mx_raw * sl2;
         if (mxs > m_run + LAZY) {   // always for a row without a base yet (m_run = -inf)
           alpha = (m_run == -CUDART_INF_F) ? 0.f : ex2(m_run - mxs);
           m_run = mxs;
