@@ -41,7 +41,7 @@ constexpr int RPS = 4032;                   // rows per sub-split (a multiple of
 constexpr int STAGE_BYTES = 2 * ROWS * D * 2;
 constexpr int NCW = 12;                     // consumer warps
 constexpr int THREADS = 32 * (1 + NCW);
-static_assert(ROWS % (2 * NCW) == 0, "a stage is covered by whole passes of all consumer warps");
+static_assert(ROWS % (4 * NCW) == 0, "a stage is covered by whole pass pairs of all consumer warps");
 static_assert(RPS % ROWS == 0, "stages never straddle two sub-splits");
 constexpr float LAZY = 8.f;                 // log2 of the largest tolerated growth before rescaling
 }  // namespace dec
@@ -68,25 +68,39 @@ __device__ __forceinline__ void bf16x8_to_f32x2(const uint4 w, uint64_t* f2) {
   for (int i = 0; i < 4; ++i) f2[i] = pack2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
 }
 
-// Sum over the 16 lanes of a half warp of G per-head partial sums, leaving
-// in every lane the full sum of one head, own_head(lane).  Transposing
-// butterfly: at each of the first log2(G) levels a lane keeps half of its
-// values and sends the other half, so G values need log2(G) + 4 - log2(G)
-// ... i.e. (G - 1) + (4 - log2 G) shuffles instead of 4 * G.
+// Each lane keeps its G heads in a lane-dependent order (slot i holds head
+// head_of_slot(lane, i)) chosen so that the transposing half-warp sum below
+// needs no selects: at each of the first log2(G) butterfly levels a lane keeps
+// the first half of its remaining slots and sends the second half, which its
+// partner holds, in the same head order, in its own second half.
 template <int G>
-__device__ __forceinline__ float half_warp_transpose_sum(const float (&v)[G], int lane) {
+__device__ __forceinline__ int head_of_slot(int lane, int i) {
+  const int hi = (lane >> 3) & 1, odd = (lane >> 2) & 1;
   if constexpr (G == 4) {
-    const bool hi = (lane >> 3) & 1;   // keeps heads {2,3} if set, else {0,1}
-    float k0 = (hi ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[2], 8);
-    float k1 = (hi ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, hi ? v[1] : v[3], 8);
-    const bool odd = (lane >> 2) & 1;  // keeps the odd head of the pair if set
-    float x = (odd ? k1 : k0) + __shfl_xor_sync(0xffffffffu, odd ? k0 : k1, 4);
+    const int pair = (i >> 1) ? 1 - hi : hi;
+    const int mem = (i & 1) ? 1 - odd : odd;
+    return 2 * pair + mem;
+  } else if constexpr (G == 2) {
+    return i ? 1 - hi : hi;
+  } else {
+    return 0;
+  }
+}
+
+// Sum over the 16 lanes of a half warp of the G per-head partial sums (slot
+// order), leaving in every lane the full sum of head own_head(lane) = the head
+// of its slot 0.  G = 4 takes 5 shuffles instead of 16.
+template <int G>
+__device__ __forceinline__ float half_warp_transpose_sum(const float (&v)[G]) {
+  if constexpr (G == 4) {
+    const float k0 = v[0] + __shfl_xor_sync(0xffffffffu, v[2], 8);
+    const float k1 = v[1] + __shfl_xor_sync(0xffffffffu, v[3], 8);
+    float x = k0 + __shfl_xor_sync(0xffffffffu, k1, 4);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     return x;
   } else if constexpr (G == 2) {
-    const bool hi = (lane >> 3) & 1;
-    float x = (hi ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[1], 8);
+    float x = v[0] + __shfl_xor_sync(0xffffffffu, v[1], 8);
     x += __shfl_xor_sync(0xffffffffu, x, 4);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     x += __shfl_xor_sync(0xffffffffu, x, 1);
@@ -99,19 +113,12 @@ __device__ __forceinline__ float half_warp_transpose_sum(const float (&v)[G], in
   }
 }
 
-// The head whose full sum half_warp_transpose_sum leaves in `lane`, and the
-// lane (of the same half warp) holding head h.
+// Lane (xor distance) in the same half warp whose slot 0 holds the head of
+// this lane's slot i: the reduced score of a head is replicated in every lane
+// whose slot 0 is that head, so a butterfly shuffle reaches it.
 template <int G>
-__device__ __forceinline__ int own_head(int lane) {
-  if constexpr (G == 4) return ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-  else if constexpr (G == 2) return (lane >> 3) & 1;
-  else return 0;
-}
-template <int G>
-__device__ __forceinline__ int head_lane(int lane, int h) {
-  if constexpr (G == 4) return (lane & 16) | ((h >> 1) << 3) | ((h & 1) << 2);
-  else if constexpr (G == 2) return (lane & 16) | (h << 3);
-  else return lane & 16;
+__device__ __forceinline__ constexpr int slot_xor(int i) {
+  return G == 4 ? (i << 2) : G == 2 ? (i << 3) : 0;
 }
 
 template <int G>
@@ -197,7 +204,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
   const int ctid = threadIdx.x - 32;       // 0..32*NCW-1
   const int half = lane >> 4;
   const int dcol = ((lane >> 3) & 1) * 64 + (lane & 7) * 8;   // first dim of this lane
-  const int oh = own_head<G>(lane);
+  const int oh = head_of_slot<G>(lane, 0);   // the head whose running (m, l) this lane keeps
   const float qscale = a.scale * 1.4426950408889634f;
   uint32_t cnt = 0;
   const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(a.q);
@@ -229,11 +236,12 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     if (r0 >= r1) continue;
 
     // this lane's 8 dims of the G query heads, scaled by scale * log2(e)
-    uint64_t q2[G][4];
+    uint64_t q2[G][4];   // slot order (see head_of_slot)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float f[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + ((size_t)b * a.Hq + g * G + h) * D + dcol), f);
+      const int head = head_of_slot<G>(lane, h);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + ((size_t)b * a.Hq + g * G + head) * D + dcol), f);
 #pragma unroll
       for (int i = 0; i < 4; ++i) q2[h][i] = pack2(f[2 * i] * qscale, f[2 * i + 1] * qscale);
     }
@@ -252,45 +260,67 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, kWaitDecodeFull, a.err)) { ok = false; break; }
       const uint8_t* Ks = sm.stage[s];
       const uint8_t* Vs = Ks + ROWS * D * 2;
+      // two passes per iteration: their reductions and broadcasts interleave
 #pragma unroll
-      for (int pass = 0; pass < ROWS / (2 * NCW); ++pass) {
-        const int rr = pass * 2 * NCW + cw * 2 + half;
-        const bool valid = row + rr < r1;
-        uint64_t x2[4];
-        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Ks + rr * 256 + dcol * 2), x2);
-        float part[G];
+      for (int pass = 0; pass < ROWS / (2 * NCW); pass += 2) {
+        int rr[2];
+        bool valid[2];
+        uint64_t x2[2][4];
+        float part[2][G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const uint64_t acc = ffma2(q2[h][1], x2[1], ffma2(q2[h][0], x2[0], 0ull));
-          part[h] = hsum2(ffma2(q2[h][3], x2[3], ffma2(q2[h][2], x2[2], acc)));
+        for (int u = 0; u < 2; ++u) {
+          rr[u] = (pass + u) * 2 * NCW + cw * 2 + half;
+          valid[u] = row + rr[u] < r1;
+          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Ks + rr[u] * 256 + dcol * 2), x2[u]);
         }
-        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Vs + rr * 256 + dcol * 2), x2);
-        float sc = half_warp_transpose_sum<G>(part, lane);
-        if (!valid) sc = -CUDART_INF_F;
-        const bool moved = sc > m + LAZY;
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const uint64_t acc = ffma2(q2[h][1], x2[u][1], ffma2(q2[h][0], x2[u][0], 0ull));
+            part[u][h] = hsum2(ffma2(q2[h][3], x2[u][3], ffma2(q2[h][2], x2[u][2], acc)));
+          }
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Vs + rr[u] * 256 + dcol * 2), x2[u]);
+        float sc[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          sc[u] = half_warp_transpose_sum<G>(part[u]);
+          if (!valid[u]) sc[u] = -CUDART_INF_F;
+        }
+        // online update with both rows (the base moves at most once per row pair)
+        const float smax = fmaxf(sc[0], sc[1]);
+        const bool moved = smax > m + LAZY;
         if (__any_sync(0xffffffffu, moved)) {
           float f = 1.f;
           if (moved) {
-            f = (m == -CUDART_INF_F) ? 0.f : ex2(m - sc);
-            m = sc;
+            f = (m == -CUDART_INF_F) ? 0.f : ex2(m - smax);
+            m = smax;
             l *= f;
           }
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float fh = __shfl_sync(0xffffffffu, f, head_lane<G>(lane, h));
+            const float fh = __shfl_xor_sync(0xffffffffu, f, slot_xor<G>(h));
             const uint64_t f2 = pack2(fh, fh);
 #pragma unroll
             for (int i = 0; i < 4; ++i) o2[h][i] = fmul2(o2[h][i], f2);
           }
         }
-        const float pw = (valid && m != -CUDART_INF_F) ? ex2(sc - m) : 0.f;
-        l += pw;
+        const bool live = m != -CUDART_INF_F;
+        float pw[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          pw[u] = (valid[u] && live) ? ex2(sc[u] - m) : 0.f;
+          l += pw[u];
+        }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float ph_ = __shfl_sync(0xffffffffu, pw, head_lane<G>(lane, h));
-          const uint64_t p2 = pack2(ph_, ph_);
+          const float p0 = __shfl_xor_sync(0xffffffffu, pw[0], slot_xor<G>(h));
+          const float p1 = __shfl_xor_sync(0xffffffffu, pw[1], slot_xor<G>(h));
+          const uint64_t a2 = pack2(p0, p0), b2 = pack2(p1, p1);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) o2[h][i] = ffma2(p2, x2[i], o2[h][i]);
+          for (int i = 0; i < 4; ++i) o2[h][i] = ffma2(b2, x2[1][i], ffma2(a2, x2[0][i], o2[h][i]));
         }
       }
       __syncwarp();
@@ -309,7 +339,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       m = mc;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float fh = __shfl_sync(0xffffffffu, f, head_lane<G>(lane, h));
+        const float fh = __shfl_xor_sync(0xffffffffu, f, slot_xor<G>(h));
         const uint64_t f2 = pack2(fh, fh);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -323,9 +353,12 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     }
     if (half == 0) {
 #pragma unroll
-      for (int h = 0; h < G; ++h)
+      for (int h = 0; h < G; ++h) {
+        const int head = head_of_slot<G>(lane, h);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) unpack2(o2[h][i], sm.wpart[cw][h][dcol + 2 * i], sm.wpart[cw][h][dcol + 2 * i + 1]);
+        for (int i = 0; i < 4; ++i)
+          unpack2(o2[h][i], sm.wpart[cw][head][dcol + 2 * i], sm.wpart[cw][head][dcol + 2 * i + 1]);
+      }
       if ((lane & 3) == 0) {
         sm.wm[cw][oh] = m;
         sm.wl[cw][oh] = l;
