@@ -40,8 +40,9 @@ constexpr int NST = 4;                      // stages
 constexpr int RPS = 4032;                   // rows per sub-split (a multiple of ROWS)
 constexpr int STAGE_BYTES = 2 * ROWS * D * 2;
 constexpr int NCW = 12;                     // consumer warps
+constexpr int UPI = 4;                      // rows per half warp handled together
 constexpr int THREADS = 32 * (1 + NCW);
-static_assert(ROWS % (4 * NCW) == 0, "a stage is covered by whole pass pairs of all consumer warps");
+static_assert(ROWS % (2 * UPI * NCW) == 0, "a stage is covered by whole iterations of all consumer warps");
 static_assert(RPS % ROWS == 0, "stages never straddle two sub-splits");
 constexpr float LAZY = 8.f;                 // log2 of the largest tolerated growth before rescaling
 }  // namespace dec
@@ -260,37 +261,39 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, kWaitDecodeFull, a.err)) { ok = false; break; }
       const uint8_t* Ks = sm.stage[s];
       const uint8_t* Vs = Ks + ROWS * D * 2;
-      // two passes per iteration: their reductions and broadcasts interleave
+      // UPI passes per iteration: their reductions and broadcasts interleave
 #pragma unroll
-      for (int pass = 0; pass < ROWS / (2 * NCW); pass += 2) {
-        int rr[2];
-        bool valid[2];
-        uint64_t x2[2][4];
-        float part[2][G];
+      for (int pass = 0; pass < ROWS / (2 * NCW); pass += UPI) {
+        int rr[UPI];
+        bool valid[UPI];
+        uint64_t x2[UPI][4];
+        float part[UPI][G];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < UPI; ++u) {
           rr[u] = (pass + u) * 2 * NCW + cw * 2 + half;
           valid[u] = row + rr[u] < r1;
           bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Ks + rr[u] * 256 + dcol * 2), x2[u]);
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < UPI; ++u)
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const uint64_t acc = ffma2(q2[h][1], x2[u][1], ffma2(q2[h][0], x2[u][0], 0ull));
             part[u][h] = hsum2(ffma2(q2[h][3], x2[u][3], ffma2(q2[h][2], x2[u][2], acc)));
           }
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < UPI; ++u)
           bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Vs + rr[u] * 256 + dcol * 2), x2[u]);
-        float sc[2];
+        float sc[UPI];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < UPI; ++u) {
           sc[u] = half_warp_transpose_sum<G>(part[u]);
           if (!valid[u]) sc[u] = -CUDART_INF_F;
         }
-        // online update with both rows (the base moves at most once per row pair)
-        const float smax = fmaxf(sc[0], sc[1]);
+        // online update with the UPI rows (the base moves at most once per iteration)
+        float smax = sc[0];
+#pragma unroll
+        for (int u = 1; u < UPI; ++u) smax = fmaxf(smax, sc[u]);
         const bool moved = smax > m + LAZY;
         if (__any_sync(0xffffffffu, moved)) {
           float f = 1.f;
@@ -308,19 +311,21 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
           }
         }
         const bool live = m != -CUDART_INF_F;
-        float pw[2];
+        float pw[UPI];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < UPI; ++u) {
           pw[u] = (valid[u] && live) ? ex2(sc[u] - m) : 0.f;
           l += pw[u];
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float p0 = __shfl_xor_sync(0xffffffffu, pw[0], slot_xor<G>(h));
-          const float p1 = __shfl_xor_sync(0xffffffffu, pw[1], slot_xor<G>(h));
-          const uint64_t a2 = pack2(p0, p0), b2 = pack2(p1, p1);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) o2[h][i] = ffma2(b2, x2[1][i], ffma2(a2, x2[0][i], o2[h][i]));
+          for (int u = 0; u < UPI; ++u) {
+            const float pu = __shfl_xor_sync(0xffffffffu, pw[u], slot_xor<G>(h));
+            const uint64_t p2 = pack2(pu, pu);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o2[h][i] = ffma2(p2, x2[u][i], o2[h][i]);
+          }
         }
       }
       __syncwarp();
