@@ -21,6 +21,7 @@ same workload (the reference arm of this build).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -394,6 +395,13 @@ PROFILE_CASES = {
     "tc": W.CFG3,
     # the timed S=128k GQA workload (only for single-pass ncu metrics)
     "tc_full": W.CFG4,
+    # the same S=128k GQA workload under the other splits (same FLOPs, different tiles and order)
+    "tc_full_contiguous": dataclasses.replace(W.CFG4, layout="contiguous",
+                                              name="ring_bf16_causal_contiguous_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
+    "tc_full_zigzag4": dataclasses.replace(W.CFG4, layout="zigzag4",
+                                           name="ring_bf16_causal_zigzag4_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
+    "tc_full_striped": dataclasses.replace(W.CFG4, layout="striped",
+                                           name="ring_bf16_causal_striped_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
     # split-KV decode on 4 x 65536-token sequences (K+V 1.07 GB > L2, lengths U[32k, 64k])
     "decode": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),
     "decode_full": W.CFG5,

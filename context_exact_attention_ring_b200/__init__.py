@@ -26,9 +26,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libringattn_sm100a.so")
 
 RING_OK, RING_EINVAL, RING_EUNSUPPORTED, RING_ECUDA, RING_ETIMEOUT = 0, -1, -2, -3, -4
-RING_CONTIGUOUS, RING_ZIGZAG = 0, 1
+RING_CONTIGUOUS, RING_ZIGZAG, RING_STRIPED = 0, 1, 2
+RING_MAX_CHUNKS_PER_RANK = 8
 RING_BF16, RING_FP32 = 0, 1
-LAYOUTS = {"contiguous": RING_CONTIGUOUS, "zigzag": RING_ZIGZAG}
+LAYOUTS = {"contiguous": RING_CONTIGUOUS, "zigzag": RING_ZIGZAG, "striped": RING_STRIPED}
+
+
+def ring_split(split: str, k: int = 0) -> int:
+    """The C ABI's split code RING_SPLIT(split, k): k chunks per rank (0 = the split's default)."""
+    return LAYOUTS[split] | (int(k) << 8)
 
 EXPORTED = (
     "ring_attn_fwd", "ring_attn_fwd_counted", "ring_attn_fwd_simt", "ring_attn_state_init", "ring_attn_step",
@@ -45,8 +51,9 @@ class RingError(RuntimeError):
 
 
 class ChunkIds(ctypes.Structure):
-    _fields_ = [("n_q", ctypes.c_int32), ("q", ctypes.c_int32 * 2), ("n_kv", ctypes.c_int32),
-                ("kv", ctypes.c_int32 * 2), ("chunk_len", ctypes.c_int32), ("causal", ctypes.c_int32)]
+    _fields_ = [("n_q", ctypes.c_int32), ("q", ctypes.c_int32 * RING_MAX_CHUNKS_PER_RANK),
+                ("n_kv", ctypes.c_int32), ("kv", ctypes.c_int32 * RING_MAX_CHUNKS_PER_RANK),
+                ("chunk_len", ctypes.c_int32), ("causal", ctypes.c_int32), ("stripes", ctypes.c_int32)]
 
 
 _lib = None
@@ -130,7 +137,15 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _layout(layout) -> int:
-    return LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    """A split code from 'contiguous' | 'zigzag' | 'striped', optionally with the
+    chunks per rank appended ('zigzag4', 'contiguous2'), or an int code."""
+    if not isinstance(layout, str):
+        return int(layout)
+    name = layout.rstrip("0123456789")
+    k = layout[len(name):]
+    if name not in LAYOUTS:
+        raise ValueError(f"unknown split {layout!r}")
+    return ring_split(name, int(k) if k else 0)
 
 
 def _prefill(name, q, k, v, P, causal, layout, scale, out, lse, extra=()):
@@ -185,12 +200,16 @@ def new_state(B, Hq, S_loc, D, device="cuda"):
     return m, l, O
 
 
-def ring_attn_step(q_shard, kchunk, vchunk, m, l, O, q_ids, kv_ids, chunk_len, causal=True, scale=None):
+def ring_attn_step(q_shard, kchunk, vchunk, m, l, O, q_ids, kv_ids, chunk_len, causal=True, scale=None, stripes=0):
     """One ring hop: fold the held K/V chunks (global ids kv_ids) into the
-    state of the query shard (global chunk ids q_ids), in place."""
+    state of the query shard (global chunk ids q_ids), in place.  With
+    stripes=P the shard and the block are stripes of the striped split and
+    q_ids / kv_ids hold the two ranks."""
     _cuda(q_shard, kchunk, vchunk, m, l, O)
     B, Sq, Hq, D = q_shard.shape
     Hkv = kchunk.shape[2]
+    if not (1 <= len(q_ids) <= RING_MAX_CHUNKS_PER_RANK and 1 <= len(kv_ids) <= RING_MAX_CHUNKS_PER_RANK):
+        raise ValueError(f"1..{RING_MAX_CHUNKS_PER_RANK} chunk ids expected")
     ids = ChunkIds()
     ids.n_q = len(q_ids)
     ids.n_kv = len(kv_ids)
@@ -200,6 +219,7 @@ def ring_attn_step(q_shard, kchunk, vchunk, m, l, O, q_ids, kv_ids, chunk_len, c
         ids.kv[i] = int(c)
     ids.chunk_len = int(chunk_len)
     ids.causal = int(bool(causal))
+    ids.stripes = int(stripes)
     if Sq != len(q_ids) * chunk_len or kchunk.shape[1] != len(kv_ids) * chunk_len:
         raise ValueError("shard / chunk buffers do not match the chunk ids")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)

@@ -57,6 +57,21 @@ bool make_tmap_bhsd(CUtensorMap* m, const void* base, int B, int rows, int heads
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_striped(CUtensorMap* m, const void* base, int B, int S, int P, int heads, int D, int box_d,
+                       int box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc || P < 1 || S % P) return false;
+  const cuuint64_t row = (cuuint64_t)heads * D * 2;   // bytes per token
+  const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)P, (cuuint64_t)(S / P), (cuuint64_t)B};
+  const cuuint64_t strides[4] = {(cuuint64_t)D * 2, row, row * P, row * S};
+  const cuuint32_t box[5] = {(cuuint32_t)box_d, 1, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
@@ -98,28 +113,59 @@ ring_status from_cuda(cudaError_t e) {
 
 bool good_scale(float s) { return std::isfinite(s) && s > 0.f; }
 
+// Split code of the `layout` argument: low byte the split, next byte the
+// chunks per rank (0 = the split's default).  Returns false if out of range.
+bool decode_layout(int layout, int* kind, int* cpr) {
+  if (layout < 0 || (layout >> 16)) return false;
+  const int kd = layout & 0xff, k = (layout >> 8) & 0xff;
+  if (kd == RING_CONTIGUOUS) {
+    *cpr = k ? k : 1;
+    if (*cpr > RING_MAX_CHUNKS_PER_RANK) return false;
+  } else if (kd == RING_ZIGZAG) {
+    *cpr = k ? k : 2;
+    if (*cpr < 2 || *cpr > RING_MAX_CHUNKS_PER_RANK) return false;
+  } else if (kd == RING_STRIPED) {
+    if (k > 1) return false;
+    *cpr = 1;
+  } else {
+    return false;
+  }
+  *kind = kd == RING_ZIGZAG ? kLayoutZigzag : kd == RING_STRIPED ? kLayoutStriped : kLayoutContiguous;
+  return true;
+}
+
+// Ring-mode plan of a split (no pointers, no shapes beyond the sequence).
+bool ring_split(int S, int P, int layout, Plan* pl) {
+  int kind = 0, cpr = 1;
+  if (S < 1 || P < 1 || !decode_layout(layout, &kind, &cpr)) return false;
+  const long long nchunks = (long long)P * cpr;
+  if (nchunks > (1LL << 30) || S % nchunks) return false;
+  pl->mode = kModeRing;
+  pl->layout = kind;
+  pl->P = P;
+  pl->cpr = cpr;
+  pl->striped = kind == kLayoutStriped;
+  pl->strided = pl->striped;
+  pl->nqc = pl->nkc = (int)nchunks;
+  pl->C = (int)(S / nchunks);
+  pl->Sq = pl->Skv = S;
+  return true;
+}
+
 // Shared checks of the prefill entry points; fills the ring-mode plan.
 ring_status ring_plan(const void* q, const void* k, const void* v, const void* out, const void* lse, int B, int Hq,
                       int Hkv, int S, int D, int P, int causal, int layout, float scale, int dtype, Plan* p) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return RING_EINVAL;
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || P < 1 || D < 1) return RING_EINVAL;
   if (Hq % Hkv) return RING_EINVAL;
-  if (layout != RING_CONTIGUOUS && layout != RING_ZIGZAG) return RING_EINVAL;
   if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
   if (!good_scale(scale)) return RING_EINVAL;
-  const long long nchunks = layout == RING_ZIGZAG ? 2LL * P : (long long)P;
-  if (S % nchunks) return RING_EINVAL;
+  Plan pl{};
+  if (!ring_split(S, P, layout, &pl)) return RING_EINVAL;
   if ((long long)B * S * Hq * D >= (1LL << 40)) return RING_EINVAL;
   if (D != 64 && D != 128) return RING_EUNSUPPORTED;
-  Plan pl{};
   pl.B = B; pl.Hq = Hq; pl.Hkv = Hkv; pl.D = D;
   pl.causal = causal ? 1 : 0;
-  pl.mode = kModeRing;
-  pl.layout = layout == RING_ZIGZAG ? kLayoutZigzag : kLayoutContiguous;
-  pl.P = P;
-  pl.nqc = pl.nkc = (int)nchunks;
-  pl.C = (int)(S / nchunks);
-  pl.Sq = pl.Skv = S;
   *p = pl;
   return RING_OK;
 }
@@ -171,30 +217,51 @@ ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* 
       !aligned16(O))
     return RING_EINVAL;
   if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv) return RING_EINVAL;
-  if (ids->n_q < 1 || ids->n_q > 2 || ids->n_kv < 1 || ids->n_kv > 2 || ids->chunk_len < 1) return RING_EINVAL;
+  if (ids->n_q < 1 || ids->n_q > RING_MAX_CHUNKS_PER_RANK || ids->n_kv < 1 ||
+      ids->n_kv > RING_MAX_CHUNKS_PER_RANK || ids->chunk_len < 1 || ids->stripes < 0)
+    return RING_EINVAL;
   for (int i = 0; i < ids->n_q; ++i)
     if (ids->q[i] < 0) return RING_EINVAL;
   for (int i = 0; i < ids->n_kv; ++i)
     if (ids->kv[i] < 0) return RING_EINVAL;
   if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
   if (!good_scale(scale)) return RING_EINVAL;
-  const long long maxgid = 2147483647LL / ids->chunk_len;
-  for (int i = 0; i < ids->n_q; ++i)
-    if (ids->q[i] + 1LL > maxgid) return RING_EINVAL;
-  for (int i = 0; i < ids->n_kv; ++i)
-    if (ids->kv[i] + 1LL > maxgid) return RING_EINVAL;
+  if (ids->stripes > 0) {
+    // striped split: one stripe of queries against one stripe of keys
+    if (ids->n_q != 1 || ids->n_kv != 1 || ids->q[0] >= ids->stripes || ids->kv[0] >= ids->stripes)
+      return RING_EINVAL;
+  } else {
+    const long long maxgid = 2147483647LL / ids->chunk_len;
+    for (int i = 0; i < ids->n_q; ++i)
+      if (ids->q[i] + 1LL > maxgid) return RING_EINVAL;
+    for (int i = 0; i < ids->n_kv; ++i)
+      if (ids->kv[i] + 1LL > maxgid) return RING_EINVAL;
+  }
+  if ((long long)ids->n_q * ids->chunk_len > 2147483647LL || (long long)ids->n_kv * ids->chunk_len > 2147483647LL)
+    return RING_EINVAL;
   if (D != 64 && D != 128) return RING_EUNSUPPORTED;
   Plan p{};
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.D = D;
   p.causal = ids->causal ? 1 : 0;
   p.mode = kModeStep;
-  p.layout = kLayoutContiguous;
-  p.P = 1;
+  p.layout = ids->stripes > 0 ? kLayoutStriped : kLayoutContiguous;
+  p.P = ids->stripes > 0 ? ids->stripes : 1;
+  p.cpr = 1;
+  p.striped = ids->stripes > 0;
+  p.strided = 0;   // the buffers are the shards themselves
   p.C = ids->chunk_len;
   p.nqc = ids->n_q;
   p.nkc = ids->n_kv;
-  p.qid[0] = ids->q[0]; p.qid[1] = ids->n_q > 1 ? ids->q[1] : 0;
-  p.kid[0] = ids->kv[0]; p.kid[1] = ids->n_kv > 1 ? ids->kv[1] : 0;
+  for (int i = 0; i < p.nqc; ++i) p.qid[i] = ids->q[i];
+  for (int i = 0; i < p.nkc; ++i) p.kid[i] = ids->kv[i];
+  // Q slots by decreasing chunk id (the longest rows first)
+  for (int i = 0; i < p.nqc; ++i) p.qorder[i] = i;
+  for (int i = 1; i < p.nqc; ++i)
+    for (int j = i; j > 0 && p.qid[p.qorder[j]] > p.qid[p.qorder[j - 1]]; --j) {
+      const int t = p.qorder[j];
+      p.qorder[j] = p.qorder[j - 1];
+      p.qorder[j - 1] = t;
+    }
   p.Sq = p.nqc * p.C;
   p.Skv = p.nkc * p.C;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -267,36 +334,29 @@ ring_status ring_attn_merge(const float* partials, const float* part_lse, void* 
 ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile_q, int tile_k,
                                   int64_t* per_rank_pairs, int64_t* full, int64_t* partial, int64_t* skipped) {
   if (S < 1 || P < 1 || tile_q < 1 || tile_k < 1) return RING_EINVAL;
-  if (layout != RING_CONTIGUOUS && layout != RING_ZIGZAG) return RING_EINVAL;
-  const int nch = layout == RING_ZIGZAG ? 2 * P : P;
-  if (S % nch) return RING_EINVAL;
   Plan p{};
+  if (!ring_split(S, P, layout, &p)) return RING_EINVAL;
   p.B = 1; p.Hq = 1; p.Hkv = 1; p.D = 128;
   p.causal = causal ? 1 : 0;
-  p.mode = kModeRing;
-  p.layout = layout == RING_ZIGZAG ? kLayoutZigzag : kLayoutContiguous;
-  p.P = P;
-  p.C = S / nch;
-  p.nqc = p.nkc = nch;
-  p.Sq = p.Skv = S;
   int64_t f = 0, pa = 0, sk = 0;
   if (per_rank_pairs)
     for (int r = 0; r < P; ++r) per_rank_pairs[r] = 0;
   const int tq = cdiv(p.C, tile_q), tk = cdiv(p.C, tile_k);
-  for (int qs = 0; qs < nch; ++qs) {
+  for (int qs = 0; qs < p.nqc; ++qs) {
     const int r = chunk_owner(p, qs);
+    const int qb = q_pos_base(p, qs);
     // pairs: the visiting order of rank r, filtered by the causal rule on chunks
     KvIter it;
     kv_begin(p, qs, it);
     for (; it.idx < p.nkc; kv_next_chunk(p, it)) {
-      const int ks = kv_cur_slot(p, it);
-      if (!p.causal || ks <= qs) {
+      const int kb = kv_pos_base(p, it.qg, kv_cur_slot(p, it));
+      if (!p.causal || kb <= qb + p.C - 1) {
         if (per_rank_pairs) per_rank_pairs[r]++;
       }
       for (int a = 0; a < tq; ++a) {
-        const int q0 = qs * p.C + a * tile_q, q1 = qs * p.C + imin((a + 1) * tile_q, p.C) - 1;
+        const int q0 = qb + a * tile_q, q1 = qb + imin((a + 1) * tile_q, p.C) - 1;
         for (int b = 0; b < tk; ++b) {
-          const int k0 = ks * p.C + b * tile_k, k1 = ks * p.C + imin((b + 1) * tile_k, p.C) - 1;
+          const int k0 = kb + b * tile_k, k1 = kb + imin((b + 1) * tile_k, p.C) - 1;
           const int c = tile_class(p.causal, q0, q1, k0, k1);
           if (c == 0) ++f; else if (c == 1) ++pa; else ++sk;
         }

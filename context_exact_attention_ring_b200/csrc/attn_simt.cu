@@ -3,9 +3,10 @@
 //
 // The SIMT kernel serves the float32 path, whose tolerance (1e-5) rules out
 // the tensor cores, and is the GPU cross-check of the bf16 tensor-core path.
-// It follows the same ring scheduler (ring_sched.h): for a 64-row query tile of one
-// head it folds 64-key K/V tiles in the rank's ring order into the running
-// (m, l, O) of "Lesson 8: Context Parallelism", section 3, then writes
+// It follows the same ring scheduler (ring_sched.h), for every split: for a
+// 64-row query tile of one head it folds 64-key K/V tiles in the rank's ring
+// order into the running (m, l, O) of "Lesson 8: Context Parallelism",
+// section 3, then writes
 // out = O / l and lse = m + ln l (ring mode) or folds its block result into
 // the caller's state (step mode).
 #include <cuda_bf16.h>
@@ -65,8 +66,8 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(Plan p, const T* __restr
   const int g = h / (p.Hq / p.Hkv);
   const int q_off = qt * BQ;
   const int nrows = imin(BQ, p.C - q_off);
-  const int qrow0 = qslot * p.C + q_off;
-  const int qpos0 = q_gid(p, qslot) * p.C + q_off;
+  const int qrow0 = buf_row(p, qslot, q_off);
+  const int qpos0 = q_pos_base(p, qslot) + q_off;
   const int qhi = qpos0 + nrows - 1;
   const int tid = threadIdx.x, r = tid >> 2, sub = tid & 3;
   const int qpos = qpos0 + r;
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(Plan p, const T* __restr
   for (int e = tid; e < BQ * D; e += 256) {
     const int rr = e / D, d = e - rr * D;
     float x = 0.f;
-    if (rr < nrows) x = ld_val(q + (((size_t)b * p.Sq + qrow0 + rr) * p.Hq + h) * D + d);
+    if (rr < nrows) x = ld_val(q + (((size_t)b * p.Sq + buf_row(p, qslot, q_off + rr)) * p.Hq + h) * D + d);
     Qs[rr * DP + d] = x;
   }
 
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(Plan p, const T* __restr
       const int kk = e / D, d = e - kk * D;
       float xk = 0.f, xv = 0.f;
       if (kk < t.nvalid) {
-        const size_t off = (((size_t)b * p.Skv + t.row0 + kk) * p.Hkv + g) * D + d;
+        const size_t off = (((size_t)b * p.Skv + buf_row(p, t.slot, t.k0 + kk)) * p.Hkv + g) * D + d;
         xk = ld_val(k + off);
         xv = ld_val(v + off);
       }
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(Plan p, const T* __restr
   }
 
   const bool active = r < nrows;
-  const int row = qrow0 + r;
+  const int row = buf_row(p, qslot, q_off + r);
   if (p.mode == kModeRing) {
     if (!active) return;
     const float inv = l > 0.f ? 1.f / l : 0.f;

@@ -147,7 +147,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         mbar_arrive_expect_tx(qb, 2 * BM * D * 2);
         for (int i = 0; i < 2; ++i)
           for (int sl = 0; sl < D / 64; ++sl)
-            tma_load_4d(smem_u32(sm.q[i]) + sl * SLAB, &tmQ, qb, sl * 64, it.h[i], it.qrow0[i], it.b, pol_q);
+            if (p.strided)
+              tma_load_5d(smem_u32(sm.q[i]) + sl * SLAB, &tmQ, qb, sl * 64, it.h[i], it.qslot, it.qoff[i], it.b,
+                          pol_q);
+            else
+              tma_load_4d(smem_u32(sm.q[i]) + sl * SLAB, &tmQ, qb, sl * 64, it.h[i], it.qrow0[i], it.b, pol_q);
         KvIter iter;
         kv_begin(p, it.qslot, iter);
         KvTile t;
@@ -160,9 +164,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
             const uint32_t fb = smem_u32(&sm.kv_full[s]);
             mbar_arrive_expect_tx(fb, BN * D * 2);
-            for (int sl = 0; sl < D / 64; ++sl)
-              tma_load_4d(smem_u32(sm.kv[s]) + sl * SLAB, kind == 0 ? (const void*)&tmK : (const void*)&tmV, fb,
-                          sl * 64, it.hkv, t.row0, it.b, pol_kv);
+            const void* tm = kind == 0 ? (const void*)&tmK : (const void*)&tmV;
+            for (int sl = 0; sl < D / 64; ++sl) {
+              if (p.strided)
+                tma_load_5d(smem_u32(sm.kv[s]) + sl * SLAB, tm, fb, sl * 64, it.hkv, t.slot, t.k0, it.b, pol_kv);
+              else
+                tma_load_4d(smem_u32(sm.kv[s]) + sl * SLAB, tm, fb, sl * 64, it.hkv, t.row0, it.b, pol_kv);
+            }
             ++kv_cnt;
           }
         }
@@ -409,7 +417,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       ++items_with_tiles;
       tc_fence_after();
       const bool active = row < nrows;
-      const int qr = it.qrow0[i] + row;
+      const int qr = p.strided ? (it.qoff[i] + row) * p.P + it.qslot : it.qrow0[i] + row;
       const int h = it.h[i];
       const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
       if (p.mode == kModeRing) {
@@ -500,10 +508,16 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 template <int D>
 static cudaError_t launch_tc_d(const Plan& p, const TcArgs& a, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_bhsd(&tq, a.q, p.B, p.Sq, p.Hq, D, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_bhsd(&tk, a.k, p.B, p.Skv, p.Hkv, D, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_bhsd(&tv, a.v, p.B, p.Skv, p.Hkv, D, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (p.strided) {
+    if (!make_tmap_striped(&tq, a.q, p.B, p.Sq, p.P, p.Hq, D, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_striped(&tk, a.k, p.B, p.Skv, p.P, p.Hkv, D, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_striped(&tv, a.v, p.B, p.Skv, p.P, p.Hkv, D, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else if (!make_tmap_bhsd(&tq, a.q, p.B, p.Sq, p.Hq, D, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+             !make_tmap_bhsd(&tk, a.k, p.B, p.Skv, p.Hkv, D, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+             !make_tmap_bhsd(&tv, a.v, p.B, p.Skv, p.Hkv, D, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B)) {
     return cudaErrorInvalidValue;
+  }
   TcParams prm;
   prm.p = p;
   prm.space = item_space(p, tc::BM);

@@ -68,6 +68,12 @@ EncodeTiledFn get_encode_tiled();
 bool make_tmap_bhsd(CUtensorMap* m, const void* base, int B, int rows, int heads, int D, int box_d, int box_rows,
                     CUtensorMapSwizzle swz);
 
+// 5-D bf16 tensor map over a [B, S, heads, D] tensor viewed as
+// [B, S/P, P, heads, D] (token x*P + c at coordinates (c, x)) with box
+// {box_d, 1, 1, box_rows, 1}: one box holds box_rows tokens of stripe c.
+bool make_tmap_striped(CUtensorMap* m, const void* base, int B, int S, int P, int heads, int D, int box_d,
+                       int box_rows, CUtensorMapSwizzle swz);
+
 int num_sms();
 
 // Device address of the library's error word on the current device.

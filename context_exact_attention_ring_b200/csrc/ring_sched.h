@@ -2,8 +2,16 @@
 //
 // Ownership of chunks, the ring visiting order and the causal tile filter of
 // "Lesson 8: Context Parallelism":
-//   * section 4A -- contiguous split: P chunks, rank r owns chunk r;
+//   * section 4A -- contiguous split: rank r owns chunk r (with k chunks per
+//                   rank, the sequential assignment of the worked example:
+//                   chunks r*k .. r*k+k-1);
 //   * section 4B -- zig-zag split: 2P chunks, rank r owns chunks r, 2P-1-r;
+//                   the code exercise generalises it to k chunks per rank
+//                   (even slots count up from the front of the sequence,
+//                   odd slots down from the back);
+//   * "Sequence parallelism and ring attention", outlook -- the striped
+//                   split, read as: token t belongs to rank t mod P, so the
+//                   shard of rank r is the stripe r, r+P, r+2P, ...;
 //   * section 2  -- at ring step t rank r holds the K/V block that started on
 //                   rank (r - t) mod P;
 //   * section 4  -- causal rule: query position i sees key position j <= i,
@@ -14,6 +22,13 @@
 // needs no memory of its own.  Work items are handed out longest-first
 // (queries at later positions meet more keys), which balances the
 // persistent CTAs.
+//
+// Mask positions.  Chunked splits compare global token positions.  The
+// striped split compares shard-local row indices instead: query row x of
+// stripe r sits at x*P + r and key row y of stripe s at y*P + s, and
+// y*P + s <= x*P + r  <=>  y + [s > r] <= x, so key rows are shifted by one
+// when the key's stripe comes after the query's.  Both give the same
+// "key position <= query position" test, tile filter and element mask.
 #pragma once
 #include <cstdint>
 
@@ -25,8 +40,9 @@
 
 namespace ra {
 
-enum { kLayoutContiguous = 0, kLayoutZigzag = 1 };
+enum { kLayoutContiguous = 0, kLayoutZigzag = 1, kLayoutStriped = 2 };
 enum { kModeRing = 0, kModeStep = 1 };
+enum { kMaxChunksPerRank = 8 };
 
 struct Plan {
   int B, Hq, Hkv, D;
@@ -34,10 +50,14 @@ struct Plan {
   int mode;      // kModeRing: buffers hold the whole sequence; kModeStep: one hop
   int layout;    // ring mode: split of the sequence
   int P;         // ring mode: virtual ranks
-  int C;         // tokens per chunk
+  int cpr;       // ring mode: chunks per rank
+  int striped;   // striped split: chunk c is stripe c (step mode: ids are ranks)
+  int strided;   // ring mode + striped: row x of stripe c is buffer row x*P + c
+  int C;         // tokens per chunk (per stripe when striped)
   int nqc, nkc;  // chunks held in the Q buffer and in the K/V buffer
-  int qid[2];    // step mode: global chunk index of each Q-buffer chunk
-  int kid[2];    // step mode: global chunk index of each K/V-buffer chunk
+  int qid[kMaxChunksPerRank];     // step mode: global chunk index of each Q-buffer chunk
+  int kid[kMaxChunksPerRank];     // step mode: global chunk index of each K/V-buffer chunk
+  int qorder[kMaxChunksPerRank];  // step mode: Q slots by decreasing chunk index
   int Sq, Skv;   // rows of the Q buffer / K/V buffer (nqc*C, nkc*C)
 };
 
@@ -45,27 +65,46 @@ RA_HD int imin(int a, int b) { return a < b ? a : b; }
 RA_HD int imax(int a, int b) { return a > b ? a : b; }
 RA_HD int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-RA_HD int chunks_per_rank(const Plan& p) { return p.layout == kLayoutZigzag ? 2 : 1; }
+RA_HD int chunks_per_rank(const Plan& p) { return p.cpr; }
 
 // Owner rank of global chunk c (ring mode).
 RA_HD int chunk_owner(const Plan& p, int c) {
-  if (p.layout == kLayoutZigzag) return c < p.P ? c : 2 * p.P - 1 - c;
-  return c;
+  if (p.layout == kLayoutZigzag) {
+    const int m = c / p.P;                                 // block of P chunks
+    return m < (p.cpr + 1) / 2 ? c - m * p.P              // counted from the front
+                               : (m + 1) * p.P - 1 - c;   // counted from the back
+  }
+  if (p.layout == kLayoutContiguous) return c / p.cpr;
+  return c;                                                // striped
 }
 
 // j-th chunk (j < chunks_per_rank) owned by rank r.
 RA_HD int rank_chunk(const Plan& p, int r, int j) {
-  if (p.layout == kLayoutZigzag) return j == 0 ? r : 2 * p.P - 1 - r;
+  if (p.layout == kLayoutZigzag) {
+    const int i = j >> 1;
+    return (j & 1) ? p.cpr * p.P - 1 - i * p.P - r : i * p.P + r;
+  }
+  if (p.layout == kLayoutContiguous) return r * p.cpr + j;
   return r;
 }
 
 RA_HD int q_gid(const Plan& p, int slot) { return p.mode == kModeRing ? slot : p.qid[slot]; }
 RA_HD int kv_gid(const Plan& p, int slot) { return p.mode == kModeRing ? slot : p.kid[slot]; }
 
-// One K/V tile: rows [row0, row0 + nvalid) of the K/V buffer, global
-// positions [pos0, pos0 + nvalid), chunk slot and global chunk id.
+// Mask position of row 0 of a Q chunk / of a K/V chunk met by Q chunk qg.
+RA_HD int q_pos_base(const Plan& p, int qslot) { return p.striped ? 0 : q_gid(p, qslot) * p.C; }
+RA_HD int kv_pos_base(const Plan& p, int qg, int kslot) {
+  return p.striped ? (kv_gid(p, kslot) > qg ? 1 : 0) : kv_gid(p, kslot) * p.C;
+}
+
+// Buffer row of row x of chunk slot c.
+RA_HD int buf_row(const Plan& p, int slot, int x) { return p.strided ? x * p.P + slot : slot * p.C + x; }
+
+// One K/V tile: rows k0 .. k0 + nvalid - 1 of chunk slot `slot` (buffer row
+// row0 for the first when rows are not strided), mask positions
+// [pos0, pos0 + nvalid), and the chunk's global id.
 struct KvTile {
-  int row0, pos0, nvalid, slot, gid, first_in_chunk;
+  int row0, k0, pos0, nvalid, slot, gid, first_in_chunk;
 };
 
 // Walks the K/V chunks met by the queries of one Q chunk, in the owning
@@ -76,12 +115,14 @@ struct KvIter {
   int kt;   // next tile inside the current chunk
   int src;  // ring mode: the rank whose K/V block is held at this step
   int j;    // ring mode: which of that rank's chunks
+  int qg;   // global id of the Q chunk (mask positions of the striped split)
 };
 
 RA_HD void kv_begin(const Plan& p, int qslot, KvIter& it) {
   it.idx = 0;
   it.kt = 0;
   it.j = 0;
+  it.qg = q_gid(p, qslot);
   it.src = p.mode == kModeRing ? chunk_owner(p, qslot) : 0;   // step 0: the rank's own block
 }
 
@@ -106,12 +147,13 @@ RA_HD bool kv_next(const Plan& p, int qhi, int BN, int tpc, KvIter& it, KvTile& 
     const int slot = kv_cur_slot(p, it);
     const int gid = kv_gid(p, slot);
     const int k0 = it.kt * BN;
-    const int pos0 = gid * p.C + k0;
+    const int pos0 = kv_pos_base(p, it.qg, slot) + k0;
     if (it.kt >= tpc || (p.causal && pos0 > qhi)) {
       kv_next_chunk(p, it);
       continue;
     }
-    t.row0 = slot * p.C + k0;
+    t.row0 = buf_row(p, slot, k0);
+    t.k0 = k0;
     t.pos0 = pos0;
     t.nvalid = imin(BN, p.C - k0);
     t.slot = slot;
@@ -129,7 +171,7 @@ RA_HD int kv_count(const Plan& p, int qslot, int qhi, int BN, int tpc) {
   kv_begin(p, qslot, it);
   int n = 0;
   for (; it.idx < p.nkc; kv_next_chunk(p, it)) {
-    const int cpos = kv_gid(p, kv_cur_slot(p, it)) * p.C;
+    const int cpos = kv_pos_base(p, it.qg, kv_cur_slot(p, it));
     if (!p.causal) {
       n += tpc;
     } else if (cpos <= qhi) {
@@ -140,12 +182,7 @@ RA_HD int kv_count(const Plan& p, int qslot, int qhi, int BN, int tpc) {
 }
 
 // Q slots ordered by decreasing global chunk id (longest work first).
-RA_HD int q_slot_by_rank(const Plan& p, int k) {
-  if (p.mode == kModeRing) return p.nqc - 1 - k;
-  if (p.nqc == 1) return 0;
-  const bool first_later = p.qid[0] > p.qid[1];
-  return (k == 0) == first_later ? 0 : 1;
-}
+RA_HD int q_slot_by_rank(const Plan& p, int k) { return p.mode == kModeRing ? p.nqc - 1 - k : p.qorder[k]; }
 
 // ---------------------------------------------------------------------------
 // Work items of the tensor-core kernel: two 128-row query tiles that share
@@ -156,8 +193,9 @@ RA_HD int q_slot_by_rank(const Plan& p, int k) {
 struct Item {
   int b, hkv, h[2];
   int qslot;
-  int qrow0[2];  // first row of tile i in the Q buffer
-  int qpos0[2];  // global position of that row
+  int qoff[2];   // first row of tile i inside its chunk
+  int qrow0[2];  // buffer row of that row (when rows are not strided)
+  int qpos0[2];  // mask position of that row
   int nrows[2];  // valid rows of tile i (0..BM)
   int qlo, qhi;  // first / last valid global position over both tiles
   int tile_in_chunk[2];
@@ -213,15 +251,15 @@ RA_HD Item item_at(const Plan& p, const ItemSpace& s, int BM, int L) {
     t0 = 2 * within;
     t1 = 2 * within + 1;
   }
-  const int cbase_row = it.qslot * p.C;
-  const int cbase_pos = q_gid(p, it.qslot) * p.C;
+  const int cbase_pos = q_pos_base(p, it.qslot);
   const int ts[2] = {t0, t1};
   it.qlo = 0x7fffffff;
   it.qhi = -1;
   for (int i = 0; i < 2; ++i) {
     const int off = ts[i] * BM;
     it.tile_in_chunk[i] = ts[i];
-    it.qrow0[i] = cbase_row + off;
+    it.qoff[i] = off;
+    it.qrow0[i] = buf_row(p, it.qslot, off);
     it.qpos0[i] = cbase_pos + off;
     it.nrows[i] = ts[i] < s.tq ? imin(BM, p.C - off) : 0;
     if (it.nrows[i] > 0) {

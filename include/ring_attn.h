@@ -12,7 +12,8 @@
  * softmax(scale * Q K^T) V (section 1; "Sequence parallelism and ring
  * attention", FAQ).  Causal masking follows section 4 (query i sees keys
  * j <= i, global positions); the contiguous split is section 4A, the zig-zag
- * split (2P chunks, rank r owns chunks r and 2P-1-r) section 4B.  The decode
+ * split (2P chunks, rank r owns chunks r and 2P-1-r) section 4B, with k
+ * chunks per rank and the striped split as variants (see ring_layout).  The decode
  * entry points shard the KV cache of one-token queries along the sequence
  * ("NVIDIA unveils Helix Parallelism", Phase 1, KV parallelism) and merge the
  * per-shard partial results.
@@ -53,17 +54,38 @@ typedef enum {
   RING_ETIMEOUT = -4       /* a bounded wait inside a kernel expired */
 } ring_status;
 
-typedef enum { RING_CONTIGUOUS = 0, RING_ZIGZAG = 1 } ring_layout; /* how the sequence is split */
+/*
+ * How the sequence is split among the P virtual ranks (the `layout` argument):
+ *   RING_CONTIGUOUS  P*k chunks; rank r owns chunks r*k .. r*k+k-1 (section 4A
+ *                    of "Lesson 8" for k = 1; the worked example's sequential
+ *                    assignment for k > 1).
+ *   RING_ZIGZAG      P*k chunks; slot j of rank r is chunk (j/2)*P + r for
+ *                    even j and P*k-1-(j/2)*P-r for odd j (section 4B for
+ *                    k = 2, chunks r and 2P-1-r; the code exercise for any k).
+ *   RING_STRIPED     token t belongs to rank t mod P ("Sequence parallelism and
+ *                    ring attention", outlook, which names the striped variant;
+ *                    the token rule is this library's reading).
+ * The low byte selects the split; RING_SPLIT(split, k) adds the chunks per
+ * rank k (1..RING_MAX_CHUNKS_PER_RANK; zig-zag needs k >= 2, striped k = 1).
+ * A bare RING_CONTIGUOUS means k = 1, a bare RING_ZIGZAG k = 2.
+ */
+typedef enum { RING_CONTIGUOUS = 0, RING_ZIGZAG = 1, RING_STRIPED = 2 } ring_layout;
+#define RING_MAX_CHUNKS_PER_RANK 8
+#define RING_SPLIT(split, k) ((int)(split) | ((int)(k) << 8))
 typedef enum { RING_BF16 = 0, RING_FP32 = 1 } ring_dtype;
 
-/* Global chunk indices carried by one ring step (see ring_attn_step). */
+/* The chunks carried by one ring step (see ring_attn_step). */
 typedef struct {
-  int32_t n_q;        /* query chunks in the shard: 1 (contiguous) or 2 (zig-zag) */
-  int32_t q[2];       /* their global chunk indices, in shard order            */
-  int32_t n_kv;       /* K/V chunks in the block: 1 or 2                        */
-  int32_t kv[2];      /* their global chunk indices, in buffer order            */
-  int32_t chunk_len;  /* tokens per chunk (all chunks have this length)        */
-  int32_t causal;     /* 1: key at global position j is allowed for query i iff j <= i */
+  int32_t n_q;        /* query chunks in the shard: 1..RING_MAX_CHUNKS_PER_RANK  */
+  int32_t q[RING_MAX_CHUNKS_PER_RANK];   /* their chunk indices, in shard order  */
+  int32_t n_kv;       /* K/V chunks in the block: 1..RING_MAX_CHUNKS_PER_RANK    */
+  int32_t kv[RING_MAX_CHUNKS_PER_RANK];  /* their chunk indices, in buffer order */
+  int32_t chunk_len;  /* rows per chunk (all chunks have this length)            */
+  int32_t causal;     /* 1: key at position j is allowed for query i iff j <= i  */
+  int32_t stripes;    /* 0: chunked split, row x of chunk c is position c*chunk_len + x.
+                         P > 0: striped split over P ranks; q[0] and kv[0] are
+                         ranks (< P), row x of rank c's stripe is position
+                         x*P + c, and n_q = n_kv = 1.                           */
 } ring_chunk_ids;
 
 /*
@@ -72,15 +94,16 @@ typedef struct {
  *
  * q [B,S,Hq,D], k/v [B,S,Hkv,D] in natural token order; out [B,S,Hq,D] (same
  * dtype as q), lse [B,Hq,S] float.  The sequence is split into P chunks
- * (layout RING_CONTIGUOUS, chunk length S/P) or 2P chunks (RING_ZIGZAG,
- * chunk length S/(2P)).  For every rank and every query tile the kernel folds
+ * (layout RING_CONTIGUOUS, chunk length S/P), 2P chunks (RING_ZIGZAG, chunk
+ * length S/(2P)), P*k chunks (RING_SPLIT(..., k)) or P stripes of S/P
+ * tokens (RING_STRIPED).  For every rank and every query tile the kernel folds
  * K/V tiles into the on-chip (m, l, O) state in the rank's ring order,
  * skipping tiles that the causal mask removes entirely; the state never
  * leaves the chip between ring steps.
  *
  * Returns RING_EINVAL for a null or misaligned pointer, B/Hq/Hkv/S/P < 1,
- * Hq % Hkv != 0, S not divisible by the number of chunks, layout or dtype out
- * of range, or a non-finite / non-positive scale; RING_EUNSUPPORTED for
+ * Hq % Hkv != 0, S not divisible by the number of chunks (or stripes), layout
+ * or dtype out of range, or a non-finite / non-positive scale; RING_EUNSUPPORTED for
  * D not in {64, 128}; RING_ECUDA if a launch fails.
  */
 ring_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -127,16 +150,19 @@ ring_status ring_attn_state_init(float* m, float* l, float* O, int B, int Hq, in
  *
  * q_shard [B, n_q*C, Hq, D]: the rank's query chunks ids->q[0..n_q) stacked in
  * that order (C = ids->chunk_len); kchunk, vchunk [B, n_kv*C, Hkv, D]: the
- * held K/V chunks ids->kv[0..n_kv) stacked in that order.  State, read and
- * written in place:  m, l [B, Hq, n_q*C] float (m is the running max of the
- * scaled scores, natural units; l = sum exp(s - m)) and O [B, n_q*C, Hq, D]
- * float, normalised (O = sum exp(s - m) v / l), as in section 3.  Rows whose
- * block has no allowed key keep their state.  Fully masked tiles are skipped.
+ * held K/V chunks ids->kv[0..n_kv) stacked in that order.  For the striped
+ * split (ids->stripes = P) the shard is rank ids->q[0]'s stripe in token
+ * order and the block is rank ids->kv[0]'s stripe.  State, read and written
+ * in place:  m, l [B, Hq, n_q*C] float (m is the running max of the scaled
+ * scores, natural units; l = sum exp(s - m)) and O [B, n_q*C, Hq, D] float,
+ * normalised (O = sum exp(s - m) v / l), as in section 3.  Rows whose block
+ * has no allowed key keep their state.  Fully masked tiles are skipped.
  *
  * Returns RING_EINVAL for null/misaligned pointers, ids == NULL, n_q or n_kv
- * outside {1,2}, chunk_len < 1, negative chunk ids, Hq % Hkv != 0, bad dtype
- * or scale; RING_EUNSUPPORTED for D not in {64,128}; RING_ECUDA on launch
- * failure.
+ * outside 1..RING_MAX_CHUNKS_PER_RANK, chunk_len < 1, negative chunk ids,
+ * stripes < 0, a striped step with n_q or n_kv != 1 or a rank >= stripes,
+ * Hq % Hkv != 0, bad dtype or scale; RING_EUNSUPPORTED for D not in {64,128};
+ * RING_ECUDA on launch failure.
  */
 ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* vchunk,
                            float* m, float* l, float* O, const ring_chunk_ids* ids,
@@ -240,9 +266,10 @@ ring_status ring_attn_decode(const void* q, const void* k, const void* v, const 
  * ring_attn_sched_stats -- the scheduler's host-side view of one (batch, head)
  * of a causal or full ring, without running anything: per-rank unmasked
  * chunk pairs (a diagonal pair counts once; "Lesson 8", section 4B: 2P+1 per
- * zig-zag rank, section 4A: r+1 per contiguous rank) and tile classes for
- * tile_q x tile_k tiles cut inside each chunk pair (full: no mask needed;
- * partial: masked; skipped: fully masked, never issued).
+ * zig-zag rank, section 4A: r+1 per contiguous rank; a striped pair counts
+ * if any key precedes a query) and tile classes for tile_q x tile_k tiles
+ * cut inside each chunk pair (full: no mask needed; partial: masked;
+ * skipped: fully masked, never issued).  `layout` as for ring_attn_fwd.
  * per_rank_pairs has room for P values.  Any output pointer may be NULL.
  */
 ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile_q, int tile_k,

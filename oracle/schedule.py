@@ -15,6 +15,8 @@ Sources (each function cites the passage it follows):
     (q + 1) over its query chunks.
   * same lesson, code exercise: the general zig-zag rule for k chunks per rank
     (even slots count up from the front, odd slots down from the back).
+  * "Sequence parallelism and ring attention", outlook: names the striped
+    variant; read here as token t belonging to rank t mod P.
 
 Nothing here is closed-form: the closed forms printed on the page (2P+1 pairs
 per zig-zag rank, i+1 per contiguous rank) are *pins* checked against these
@@ -23,6 +25,22 @@ enumerations in tests/test_oracle_schedule.py.
 from __future__ import annotations
 
 from dataclasses import dataclass
+
+import numpy as np
+
+_DEFAULT_K = {"contiguous": 1, "zigzag": 2, "striped": 1}
+
+
+def parse_layout(layout: str) -> tuple[str, int]:
+    """Split name and chunks per rank: 'contiguous' | 'zigzag' | 'striped',
+    optionally followed by k ('zigzag4' = four chunks per rank)."""
+    name = layout.rstrip("0123456789")
+    if name not in _DEFAULT_K:
+        raise ValueError(layout)
+    k = int(layout[len(name):]) if layout != name else _DEFAULT_K[name]
+    if (name == "zigzag" and k < 2) or (name == "striped" and k != 1) or k < 1:
+        raise ValueError(layout)
+    return name, k
 
 
 def sequential_assignment(P: int, chunks_per_rank: int) -> dict[int, list[int]]:
@@ -50,14 +68,34 @@ def zigzag_assignment(P: int, chunks_per_rank: int = 2) -> dict[int, list[int]]:
     return out
 
 
+def striped_tokens(S: int, P: int) -> dict[int, list[int]]:
+    """Striped split: rank r holds tokens r, r+P, r+2P, ... in that order."""
+    return {r: list(range(r, S, P)) for r in range(P)}
+
+
 def layout_assignment(P: int, layout: str) -> dict[int, list[int]]:
-    """The two splits of the hot path: 'contiguous' (one chunk per rank,
-    section 4A) and 'zigzag' (two chunks per rank, section 4B)."""
-    if layout == "contiguous":
-        return sequential_assignment(P, 1)
-    if layout == "zigzag":
-        return zigzag_assignment(P, 2)
-    raise ValueError(layout)
+    """Chunks owned by each rank: 'contiguous' (section 4A; with k chunks per
+    rank the sequential assignment), 'zigzag' (section 4B; k per rank from the
+    code exercise).  For 'striped' the one "chunk" of rank r is its stripe,
+    numbered r."""
+    name, k = parse_layout(layout)
+    if name == "contiguous":
+        return sequential_assignment(P, k)
+    if name == "zigzag":
+        return zigzag_assignment(P, k)
+    return {r: [r] for r in range(P)}
+
+
+def chunk_positions(S: int, P: int, layout: str) -> dict[int, list[int]]:
+    """Global token positions of every chunk, in the chunk's row order."""
+    name, _ = parse_layout(layout)
+    if name == "striped":
+        if S % P:
+            raise ValueError("S must divide into the stripes")
+        return striped_tokens(S, P)
+    C = chunk_len(S, P, layout)
+    n = S // C
+    return {c: list(range(c * C, (c + 1) * C)) for c in range(n)}
 
 
 def causal_workload(assign: dict[int, list[int]]) -> dict[int, int]:
@@ -85,16 +123,28 @@ class Pair:
     kind: str       # 'full' | 'diag' | 'skip'
 
 
-def ring_pairs(P: int, layout: str, causal: bool) -> list[Pair]:
+def ring_pairs(P: int, layout: str, causal: bool, S: int | None = None) -> list[Pair]:
     """Every (rank, step, q chunk, kv chunk) the ring loop meets, classified
-    under the causal rule (kv < q full, kv == q diagonal, kv > q skipped)."""
+    under the causal rule.  Chunked splits: kv < q full, kv == q diagonal,
+    kv > q skipped.  Striped split (S needed): from the token positions, full
+    if every key precedes every query, skipped if none does, else 'diag'."""
     own = layout_assignment(P, layout)
+    striped = parse_layout(layout)[0] == "striped"
+    pos = chunk_positions(S, P, layout) if striped else None
     out = []
     for r in range(P):
         for t, src in enumerate(ring_rotation(P, r)):
             for qc in own[r]:
                 for kc in own[src]:
-                    if not causal or kc < qc:
+                    if striped:
+                        qp, kp = pos[qc], pos[kc]
+                        if not causal or max(kp) <= min(qp):
+                            kind = "full"
+                        elif min(kp) > max(qp):
+                            kind = "skip"
+                        else:
+                            kind = "diag"
+                    elif not causal or kc < qc:
                         kind = "full"
                     elif kc == qc:
                         kind = "diag"
@@ -104,17 +154,19 @@ def ring_pairs(P: int, layout: str, causal: bool) -> list[Pair]:
     return out
 
 
-def per_rank_pairs(P: int, layout: str, causal: bool) -> list[int]:
+def per_rank_pairs(P: int, layout: str, causal: bool, S: int | None = None) -> list[int]:
     """Unmasked chunk pairs per rank (a diagonal pair counts as one)."""
     cnt = [0] * P
-    for p in ring_pairs(P, layout, causal):
+    for p in ring_pairs(P, layout, causal, S):
         if p.kind != "skip":
             cnt[p.rank] += 1
     return cnt
 
 
 def chunk_len(S: int, P: int, layout: str) -> int:
-    n = P if layout == "contiguous" else 2 * P
+    """Rows per chunk (per stripe for the striped split)."""
+    name, k = parse_layout(layout)
+    n = P * k
     if S % n:
         raise ValueError("S must divide into the chunks")
     return S // n
@@ -124,29 +176,38 @@ def tile_classes(S: int, P: int, layout: str, causal: bool, tile_q: int, tile_k:
     """Tile classes for one (batch, head), enumerated tile by tile.
 
     Each chunk pair met by the ring is cut into tiles of tile_q query rows and
-    tile_k keys (the last tile of a chunk may be shorter).  With global first
-    and last positions [q0,q1] x [k0,k1] a tile is 'full' if k1 <= q0,
-    'skip' if k0 > q1, else 'partial' (causal); all tiles are full otherwise.
+    tile_k key rows in the chunks' row order (the last tile of a chunk may be
+    shorter).  From the global token positions of the tile's rows a tile is
+    'full' if its last key precedes its first query (max key <= min query),
+    'skip' if its first key follows its last query (min key > max query),
+    else 'partial' (causal); all tiles are full otherwise.
     Returns (full, partial, skipped, per_rank_processed[P]) where processed
     counts full + partial tiles by the rank owning the queries.
     """
-    C = chunk_len(S, P, layout)
+    pos = {c: np.asarray(v, dtype=np.int64) for c, v in chunk_positions(S, P, layout).items()}
+
+    def spans(x, t):
+        lo = np.array([x[a:a + t].min() for a in range(0, len(x), t)])
+        hi = np.array([x[a:a + t].max() for a in range(0, len(x), t)])
+        return lo, hi
+
+    qspan = {c: spans(x, tile_q) for c, x in pos.items()}
+    kspan = {c: spans(x, tile_k) for c, x in pos.items()}
     full = partial = skipped = 0
     per_rank = [0] * P
-    for pr in ring_pairs(P, layout, causal):
-        qbase, kbase = pr.q_chunk * C, pr.kv_chunk * C
-        for qa in range(0, C, tile_q):
-            q0, q1 = qbase + qa, qbase + min(qa + tile_q, C) - 1
-            for ka in range(0, C, tile_k):
-                k0, k1 = kbase + ka, kbase + min(ka + tile_k, C) - 1
-                if not causal or k1 <= q0:
-                    full += 1
-                    per_rank[pr.rank] += 1
-                elif k0 > q1:
-                    skipped += 1
-                else:
-                    partial += 1
-                    per_rank[pr.rank] += 1
+    for pr in ring_pairs(P, layout, causal, S):
+        q0, q1 = qspan[pr.q_chunk]
+        k0, k1 = kspan[pr.kv_chunk]
+        if not causal:
+            f, sk = q0.size * k0.size, 0
+        else:
+            f = int(np.sum(k1[None, :] <= q0[:, None]))
+            sk = int(np.sum(k0[None, :] > q1[:, None]))
+        pa = q0.size * k0.size - f - sk
+        full += f
+        partial += pa
+        skipped += sk
+        per_rank[pr.rank] += f + pa
     return full, partial, skipped, per_rank
 
 

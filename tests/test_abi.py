@@ -71,6 +71,13 @@ def fwd(**kw):
     (dict(layout=1, S=260), ra.RING_EINVAL), (dict(layout=7), ra.RING_EINVAL), (dict(dtype=5), ra.RING_EINVAL),
     (dict(scale=0.0), ra.RING_EINVAL), (dict(scale=float("nan")), ra.RING_EINVAL), (dict(P=0), ra.RING_EINVAL),
     (dict(D=96), ra.RING_EUNSUPPORTED), (dict(D=256), ra.RING_EUNSUPPORTED),
+    # split codes: zig-zag needs 2..8 chunks per rank, striped exactly one, S divisible by the chunks
+    (dict(layout=ra.ring_split("zigzag", 1)), ra.RING_EINVAL), (dict(layout=ra.ring_split("zigzag", 9)), ra.RING_EINVAL),
+    (dict(layout=ra.ring_split("striped", 2)), ra.RING_EINVAL), (dict(layout=ra.ring_split("contiguous", 9)), ra.RING_EINVAL),
+    (dict(layout=ra.ring_split("zigzag", 3), S=260), ra.RING_EINVAL), (dict(layout=2, S=258), ra.RING_EINVAL),
+    (dict(layout=1 << 16), ra.RING_EINVAL), (dict(layout=-1), ra.RING_EINVAL),
+    (dict(layout=ra.ring_split("zigzag", 4), D=96), ra.RING_EUNSUPPORTED),
+    (dict(layout=ra.ring_split("striped", 1), D=96), ra.RING_EUNSUPPORTED),
 ])
 def test_fwd_argument_checks(kw, code):
     assert fwd(**kw) == code
@@ -83,13 +90,28 @@ def test_step_argument_checks():
     ids.q[0], ids.kv[0] = 0, 0
     args = lambda i, D=64: (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(i), 1, 2, 2, D, 0.125, 1, None)
     assert L.ring_attn_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 64, 0.125, 1, None) == ra.RING_EINVAL
-    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.n_q = 3
-    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
     bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.kv[0] = -1
     assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
     bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.chunk_len = 0
     assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
+    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.n_q = ra.RING_MAX_CHUNKS_PER_RANK + 1
+    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
+    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.stripes = -1
+    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
+    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.stripes = 4; bad.kv[0] = 4   # rank outside the stripes
+    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
+    bad = ra.ChunkIds(); ctypes.pointer(bad)[0] = ids; bad.stripes = 4; bad.n_q = 2      # one stripe per shard
+    assert L.ring_attn_step(*args(bad)) == ra.RING_EINVAL
     assert L.ring_attn_step(*args(ids, D=80)) == ra.RING_EUNSUPPORTED
+    ok = ra.ChunkIds(); ctypes.pointer(ok)[0] = ids; ok.n_q = ok.n_kv = 8; ok.chunk_len = 8
+    assert L.ring_attn_step(*args(ok, D=80)) == ra.RING_EUNSUPPORTED   # 8 chunks pass the id checks
+
+
+def test_chunk_ids_struct_matches_header():
+    # n_q, q[8], n_kv, kv[8], chunk_len, causal, stripes: 21 int32
+    text = open(HEADER).read()
+    assert "#define RING_MAX_CHUNKS_PER_RANK 8" in text
+    assert ctypes.sizeof(ra.ChunkIds) == 4 * (3 + 2 * ra.RING_MAX_CHUNKS_PER_RANK + 2)
 
 
 def test_decode_and_merge_argument_checks():
@@ -121,12 +143,15 @@ def test_decode_and_merge_argument_checks():
     (256, 4, "contiguous", False, 64, 64), (8192, 8, "contiguous", True, 128, 128),
     (32768, 8, "zigzag", True, 128, 128), (131072, 16, "zigzag", True, 128, 128),
     (1536, 3, "zigzag", True, 128, 128), (1000, 4, "zigzag", True, 128, 128), (960, 5, "contiguous", True, 64, 128),
+    (3072, 4, "zigzag3", True, 128, 128), (131072, 16, "zigzag4", True, 128, 128), (4000, 2, "zigzag8", True, 64, 128),
+    (8192, 4, "contiguous2", True, 128, 128), (131072, 16, "striped", True, 128, 128), (4096, 8, "striped", True, 128, 64),
+    (1000, 4, "striped", True, 128, 128), (2048, 4, "striped", False, 128, 128), (1200, 3, "zigzag5", False, 64, 64),
 ])
 def test_sched_stats_equals_oracle_enumeration(S, P, layout, causal, tq, tk):
     per, full, partial, skipped = ra.ring_attn_sched_stats(S, P, causal, layout, tq, tk)
     o_full, o_partial, o_skipped, _ = sch.tile_classes(S, P, layout, causal, tq, tk)
     assert (full, partial, skipped) == (o_full, o_partial, o_skipped)
-    assert per == sch.per_rank_pairs(P, layout, causal)
+    assert per == sch.per_rank_pairs(P, layout, causal, S)
 
 
 def test_sched_stats_zigzag_closed_form():

@@ -57,15 +57,18 @@ def test_bf16_simt(cfg):
 
 
 def ring_by_steps(q, k, v, P, layout, causal, scale, order_fn=None, checkpoint_at=None):
-    """Drive ring_attn_step rank by rank; returns (out, lse) in natural order."""
+    """Drive ring_attn_step rank by rank; returns (out, lse) in natural order.
+    Each rank's shard is gathered from its chunks (its stripe when striped)."""
     B, S, Hq, D = q.shape
     own = sch.layout_assignment(P, layout)
+    pos = sch.chunk_positions(S, P, layout)
     C = sch.chunk_len(S, P, layout)
+    stripes = P if layout.startswith("striped") else 0
     out = torch.empty_like(q)
     lse = torch.empty((B, Hq, S), device=q.device, dtype=torch.float32)
     for r in range(P):
         qc = own[r]
-        rows = torch.cat([torch.arange(c * C, (c + 1) * C) for c in qc]).to(q.device)
+        rows = torch.tensor([t for c in qc for t in pos[c]], device=q.device)
         qs = q[:, rows].contiguous()
         m, l, O = ra.new_state(B, Hq, len(rows), D)
         srcs = sch.ring_rotation(P, r)
@@ -73,9 +76,9 @@ def ring_by_steps(q, k, v, P, layout, causal, scale, order_fn=None, checkpoint_a
             srcs = order_fn(srcs)
         for t, src in enumerate(srcs):
             kc = own[src]
-            krows = torch.cat([torch.arange(c * C, (c + 1) * C) for c in kc]).to(q.device)
+            krows = torch.tensor([t_ for c in kc for t_ in pos[c]], device=q.device)
             ra.ring_attn_step(qs, k[:, krows].contiguous(), v[:, krows].contiguous(), m, l, O, qc, kc, C,
-                              causal=causal, scale=scale)
+                              causal=causal, scale=scale, stripes=stripes)
             if checkpoint_at is not None and t == checkpoint_at:
                 # checkpoint / resume: the state is the only thing carried between steps
                 saved = [x.cpu().clone() for x in (m, l, O)]

@@ -98,3 +98,95 @@ def test_kv_visit_order_covers_all_chunks_once():
                 assert sorted(order) == list(range(n))
                 # step 0 is the rank's own K/V
                 assert order[: n // P] == sch.layout_assignment(P, layout)[r]
+
+
+# --------------------------------------------------------------------------- split variants
+@pytest.mark.parametrize("P,k", [(p, k) for p in (1, 2, 3, 4, 8) for k in (2, 3, 4, 5, 8)])
+def test_general_zigzag_is_a_partition(P, k):
+    own = sch.zigzag_assignment(P, k)
+    assert sorted(c for cs in own.values() for c in cs) == list(range(P * k))
+    # slot 0 counts up from the front, slot 1 down from the back (the section 4B pair for k = 2)
+    for r in range(P):
+        assert own[r][0] == r and own[r][1] == P * k - 1 - r
+
+
+@pytest.mark.parametrize("P,k", [(p, k) for p in (1, 2, 3, 4, 8, 16) for k in (2, 4, 6, 8)])
+def test_general_zigzag_even_k_balanced_closed_form(P, k):
+    # slots 2i and 2i+1 hold chunks iP+r and (k-i)P-1-r: (iP+r+1) + ((k-i)P-r) = kP+1 pairs,
+    # so each rank does (k/2)(kP+1) causal chunk pairs whatever its index
+    expect = [(k // 2) * (k * P + 1)] * P
+    assert list(sch.causal_workload(sch.zigzag_assignment(P, k)).values()) == expect
+    assert sch.per_rank_pairs(P, f"zigzag{k}", True) == expect
+
+
+@pytest.mark.parametrize("P,k", [(2, 3), (4, 3), (3, 5)])
+def test_general_zigzag_odd_k_near_balanced(P, k):
+    # odd k: the unpaired last slot (a front chunk) leaves a spread of at most P-1 pairs
+    w = sch.per_rank_pairs(P, f"zigzag{k}", True)
+    assert max(w) - min(w) == P - 1
+
+
+@pytest.mark.parametrize("P,k", [(2, 2), (4, 3), (3, 4)])
+def test_sequential_k_per_rank_pairs(P, k):
+    # rank r holds chunks rk .. rk+k-1, chunk c meets c+1 chunks: sum = k(rk) + k(k+1)/2
+    assert sch.per_rank_pairs(P, f"contiguous{k}", True) == [k * r * k + k * (k + 1) // 2 for r in range(P)]
+
+
+@pytest.mark.parametrize("S,P", [(64, 4), (96, 3), (1024, 8)])
+def test_striped_tokens_partition(S, P):
+    st = sch.striped_tokens(S, P)
+    assert sorted(t for ts in st.values() for t in ts) == list(range(S))
+    assert all(t % P == r for r, ts in st.items() for t in ts)
+
+
+@pytest.mark.parametrize("S,P", [(64, 4), (4096, 8), (8192, 16)])
+def test_striped_every_pair_meets_keys(S, P):
+    # every rank's stripe has keys before some query of every other stripe
+    assert sch.per_rank_pairs(P, "striped", True, S) == [P] * P
+
+
+@pytest.mark.parametrize("S,P,T", [(4096, 4, 128), (8192, 8, 128), (2048, 2, 64), (131072, 16, 128)])
+def test_striped_tile_totals_closed_form(S, P, T):
+    # stripes of n = S/(P*T) tiles: pair (r, s) keeps key tile b for query tile a iff b < a (full) or
+    # b == a (partial: the diagonal, shifted by one row when s > r), so each of the P^2 pairs is a
+    # lower triangle of n(n-1)/2 full, n partial, n(n-1)/2 skipped tiles
+    full, partial, skipped, per_rank = sch.tile_classes(S, P, "striped", True, T, T)
+    n = S // (P * T)
+    assert (full, partial, skipped) == (P * P * n * (n - 1) // 2, P * P * n, P * P * n * (n - 1) // 2)
+    assert len(set(per_rank)) == 1
+
+
+def _brute_tile_classes(S, P, layout, tq, tk):
+    """Element by element: a tile is full if every (query, key) pair is allowed, skipped if none is."""
+    pos = sch.chunk_positions(S, P, layout)
+    own = sch.layout_assignment(P, layout)
+    out = [0, 0, 0]
+    for r in range(P):
+        for src in range(P):
+            for qc in own[r]:
+                for kc in own[src]:
+                    qp, kp = pos[qc], pos[kc]
+                    for a in range(0, len(qp), tq):
+                        for b in range(0, len(kp), tk):
+                            ok = [kk <= qq for qq in qp[a:a + tq] for kk in kp[b:b + tk]]
+                            out[0 if all(ok) else 2 if not any(ok) else 1] += 1
+    return tuple(out)
+
+
+@pytest.mark.parametrize("S,P,layout,tq,tk", [
+    (48, 3, "striped", 4, 4), (64, 4, "striped", 5, 3), (60, 2, "zigzag3", 4, 4), (64, 2, "zigzag4", 3, 5),
+    (48, 4, "contiguous2", 4, 4), (40, 2, "zigzag", 4, 3), (30, 3, "contiguous", 4, 4),
+])
+def test_tile_classes_brute_force(S, P, layout, tq, tk):
+    full, partial, skipped, _ = sch.tile_classes(S, P, layout, True, tq, tk)
+    assert (full, partial, skipped) == _brute_tile_classes(S, P, layout, tq, tk)
+
+
+def test_kv_visit_order_general_splits():
+    for P in (1, 2, 3, 4):
+        for layout in ("zigzag3", "zigzag4", "contiguous2", "striped"):
+            k = sch.parse_layout(layout)[1]
+            for r in range(P):
+                order = sch.kv_visit_order(P, layout, r)
+                assert sorted(order) == list(range(P * k))
+                assert order[:k] == sch.layout_assignment(P, layout)[r]

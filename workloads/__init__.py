@@ -29,7 +29,7 @@ class Prefill:
     name: str
     dtype: str            # "fp32" | "bf16"
     causal: bool
-    layout: str           # "contiguous" | "zigzag"
+    layout: str           # "contiguous" | "zigzag" | "striped", optionally + chunks per rank ("zigzag4")
     B: int
     Hq: int
     Hkv: int
@@ -46,7 +46,10 @@ class Prefill:
 
     @property
     def n_chunks(self) -> int:
-        return self.P if self.layout == "contiguous" else 2 * self.P
+        """Chunks of the split (stripes for the striped split)."""
+        name = self.layout.rstrip("0123456789")
+        per_rank = int(self.layout[len(name):] or (2 if name == "zigzag" else 1))
+        return self.P * per_rank
 
     @property
     def chunk(self) -> int:
@@ -122,7 +125,7 @@ def prefill_inputs(cfg: Prefill, device="cpu"):
 
 def sample_rows(cfg: Prefill, n: int | None = None, seed_offset: int = 1000) -> np.ndarray:
     """Query rows checked against the oracle at large S: for every (b, hq),
-    rows 0 and S-1, the first and last row of every chunk, and seeded uniform
+    rows 0 and S-1, the first and last row of every chunk (stripe), and seeded uniform
     rows up to ``n`` (default cfg.sample_rows) per head.  Returns [N,3] int32
     (b, h, i); with n == 0 every row."""
     n = cfg.sample_rows if n is None else n
@@ -131,9 +134,14 @@ def sample_rows(cfg: Prefill, n: int | None = None, seed_offset: int = 1000) -> 
         return np.stack([b.ravel(), h.ravel(), i.ravel()], 1).astype(np.int32)
     rng = np.random.default_rng(cfg.seed + seed_offset)
     fixed = {0, cfg.S - 1}
-    for c in range(cfg.n_chunks):
-        fixed.add(c * cfg.chunk)
-        fixed.add((c + 1) * cfg.chunk - 1)
+    if cfg.layout.startswith("striped"):
+        # first and last token of every stripe (token t belongs to stripe t mod P)
+        fixed.update(range(cfg.P))
+        fixed.update(range(cfg.S - cfg.P, cfg.S))
+    else:
+        for c in range(cfg.n_chunks):
+            fixed.add(c * cfg.chunk)
+            fixed.add((c + 1) * cfg.chunk - 1)
     out = []
     for b in range(cfg.B):
         for h in range(cfg.Hq):
