@@ -404,7 +404,10 @@ PROFILE_CASES = {
                                            name="ring_bf16_causal_striped_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
     # split-KV decode on 4 x 65536-token sequences (K+V 1.07 GB > L2, lengths U[32k, 64k])
     "decode": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),
+    "decode_fused": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),
     "decode_full": W.CFG5,
+    # the same decode in one launch (partials plus the last-CTA merge)
+    "decode_full_fused": W.CFG5,
 }
 
 
@@ -429,8 +432,14 @@ def run_profile(args):
         ws = ra.decode_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.capacity, cfg.D, cfg.P, dev)
         part = torch.empty((cfg.B, cfg.Hq, cfg.P, cfg.D), device=dev, dtype=torch.float32)
         plse = torch.empty((cfg.B, cfg.Hq, cfg.P), device=dev, dtype=torch.float32)
-        fn = lambda: ra.ring_attn_decode_partial(q, k, v, sl, cfg.P, cfg.scale, partials=part, part_lse=plse,
-                                                 workspace=ws)
+        if name.endswith("_fused"):
+            out = torch.empty((cfg.B, cfg.Hq, cfg.D), device=dev, dtype=torch.bfloat16)
+            olse = torch.empty((cfg.B, cfg.Hq), device=dev, dtype=torch.float32)
+            fn = lambda: ra.ring_attn_decode_fused(q, k, v, cfg.P, seqlens=sl, scale=cfg.scale, partials=part,
+                                                   part_lse=plse, out=out, out_lse=olse, workspace=ws)
+        else:
+            fn = lambda: ra.ring_attn_decode_partial(q, k, v, sl, cfg.P, cfg.scale, partials=part, part_lse=plse,
+                                                     workspace=ws)
         work, unit = decode_bytes(cfg, lens) / 1e9, "GB/s"
     for _ in range(args.warmup):
         fn()

@@ -11,8 +11,8 @@ Names follow the C ABI:
   ring_attn_fwd, ring_attn_fwd_counted, ring_attn_fwd_simt,
   ring_attn_state_init, ring_attn_step, ring_attn_state_finalize,
   ring_attn_decode_partial, ring_attn_merge, ring_attn_decode,
-  ring_attn_decode_workspace_bytes, ring_attn_sched_stats,
-  ring_attn_device_error.
+  ring_attn_decode_workspace_bytes, ring_attn_decode_fused,
+  ring_attn_kv_append, ring_attn_sched_stats, ring_attn_device_error.
 """
 from __future__ import annotations
 
@@ -25,7 +25,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libringattn_sm100a.so")
 
-RING_OK, RING_EINVAL, RING_EUNSUPPORTED, RING_ECUDA, RING_ETIMEOUT = 0, -1, -2, -3, -4
+RING_OK, RING_EINVAL, RING_EUNSUPPORTED, RING_ECUDA, RING_ETIMEOUT, RING_ECAPACITY = 0, -1, -2, -3, -4, -5
 RING_CONTIGUOUS, RING_ZIGZAG, RING_STRIPED = 0, 1, 2
 RING_MAX_CHUNKS_PER_RANK = 8
 RING_BF16, RING_FP32 = 0, 1
@@ -41,6 +41,7 @@ EXPORTED = (
     "ring_attn_state_finalize", "ring_attn_decode_partial", "ring_attn_decode_workspace_bytes", "ring_attn_decode",
     "ring_attn_merge", "ring_attn_sched_stats", "ring_attn_device_error", "ring_attn_strerror",
     "ring_attn_version", "ring_attn_built_arch", "ring_attn_selftest_wait", "ring_attn_decode_partial_noalloc",
+    "ring_attn_decode_fused", "ring_attn_kv_append",
 )
 
 
@@ -79,6 +80,9 @@ def lib():
         "ring_attn_decode_partial": [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz, vp],
         "ring_attn_decode": [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz, vp],
         "ring_attn_decode_partial_noalloc": [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp],
+        "ring_attn_decode_fused": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz,
+                                   vp],
+        "ring_attn_kv_append": [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp],
         "ring_attn_merge": [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp],
         "ring_attn_sched_stats": [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp],
         "ring_attn_device_error": [ctypes.POINTER(ctypes.c_int)],
@@ -331,6 +335,59 @@ def ring_attn_decode(q, k, v, seqlens, P, scale=None, partials=None, part_lse=No
                                 workspace.numel(), _stream())
     _check(st, "ring_attn_decode")
     return out, out_lse
+
+
+def ring_attn_decode_fused(q, k, v, P, seqlens=None, shard_lens=None, scale=None, partials=None, part_lse=None,
+                           out=None, out_lse=None, workspace=None):
+    """Split-KV decode in one launch (partials plus the last-CTA merge).  Valid
+    rows come from `seqlens` [B] (whole-cache lengths) or `shard_lens` [B,P]
+    (per-chunk fill counts, e.g. after ring_attn_kv_append).  Returns (out, out_lse)."""
+    if (seqlens is None) == (shard_lens is None):
+        raise ValueError("give exactly one of seqlens / shard_lens")
+    _cuda(q, k, v, seqlens, shard_lens, partials, part_lse, out, out_lse, workspace)
+    B, Hq, D = q.shape
+    _, Smax, Hkv, _ = k.shape
+    lens = seqlens if seqlens is not None else shard_lens
+    if lens.dtype != torch.int32 or lens.shape != ((B,) if seqlens is not None else (B, int(P))):
+        raise ValueError("seqlens must be int32 [B], shard_lens int32 [B,P]")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dev = q.device
+    if partials is None:
+        partials = torch.empty((B, Hq, P, D), device=dev, dtype=torch.float32)
+    if part_lse is None:
+        part_lse = torch.empty((B, Hq, P), device=dev, dtype=torch.float32)
+    if out is None:
+        out = torch.empty((B, Hq, D), device=dev, dtype=torch.bfloat16)
+    if out_lse is None:
+        out_lse = torch.empty((B, Hq), device=dev, dtype=torch.float32)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, Smax, D, P, dev)
+    st = lib().ring_attn_decode_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), _ptr(shard_lens), _ptr(partials),
+                                      _ptr(part_lse), _ptr(out), _ptr(out_lse), B, Hq, Hkv, Smax, D, int(P), scale,
+                                      _dtype_code(q), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, "ring_attn_decode_fused")
+    return out, out_lse
+
+
+def ring_attn_kv_append(k_cache, v_cache, k_new, v_new, shard_lens, n_appended, P, block):
+    """Append k_new / v_new [B,T,Hkv,D] to the P-way sharded cache [B,Smax,Hkv,D],
+    round-robin by blocks of `block` tokens; shard_lens [B,P] and n_appended [B]
+    (int32, device) advance in place."""
+    _cuda(k_cache, v_cache, k_new, v_new, shard_lens, n_appended)
+    B, Smax, Hkv, D = k_cache.shape
+    T = k_new.shape[1]
+    if k_new.shape != (B, T, Hkv, D) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("k_new/v_new [B,T,Hkv,D] and caches [B,Smax,Hkv,D] expected")
+    if k_new.dtype != k_cache.dtype or v_new.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise ValueError("one dtype for caches and new tokens")
+    if shard_lens.dtype != torch.int32 or shard_lens.shape != (B, int(P)):
+        raise ValueError("shard_lens must be int32 [B,P]")
+    if n_appended.dtype != torch.int32 or n_appended.shape != (B,):
+        raise ValueError("n_appended must be int32 [B]")
+    st = lib().ring_attn_kv_append(_ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(shard_lens),
+                                   _ptr(n_appended), B, T, Hkv, Smax, D, int(P), int(block),
+                                   _dtype_code(k_cache), _stream())
+    _check(st, "ring_attn_kv_append")
 
 
 def ring_attn_sched_stats(S, P, causal, layout, tile_q=128, tile_k=128):

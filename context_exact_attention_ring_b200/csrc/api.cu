@@ -170,6 +170,36 @@ ring_status ring_plan(const void* q, const void* k, const void* v, const void* o
   return RING_OK;
 }
 
+// Shared checks of the decode entry points; fills the kernel arguments.
+ring_status decode_args(const void* q, const void* k, const void* v, const int32_t* seqlens,
+                        const int32_t* shard_lens, float* partials, float* part_lse, int B, int Hq, int Hkv,
+                        int Smax, int D, int P, float scale, int dtype, void* workspace, size_t workspace_bytes,
+                        DecodeArgs* out, DecodeExtra* extra) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !(seqlens || shard_lens) || !aligned16(partials) ||
+      !aligned16(part_lse))
+    return RING_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Smax < 1 || P < 1 || D < 1 || Hq % Hkv || Smax % P) return RING_EINVAL;
+  if (!good_scale(scale)) return RING_EINVAL;
+  if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
+  if ((long long)B * Smax * Hkv * D >= (1LL << 42)) return RING_EINVAL;
+  if (dtype != RING_BF16 || D != 128) return RING_EUNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4) return RING_EUNSUPPORTED;
+  const size_t need = decode_workspace_bytes(B, Hq, Hkv, Smax, D, P);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need) return RING_EINVAL;
+  DecodeArgs a{};
+  DecodeExtra x{};
+  a.q = q; a.k = k; a.v = v; a.seqlens = seqlens;
+  x.shard_lens = shard_lens;
+  a.partials = partials; a.part_lse = part_lse;
+  decode_workspace_split(workspace, B, Hq, Hkv, Smax, D, P, &a.ws_part, &a.ws_count, &x.ws_done);
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Smax = Smax; a.D = D; a.P = P; a.scale = scale;
+  a.err = error_word();
+  *out = a;
+  *extra = x;
+  return RING_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -288,24 +318,48 @@ size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D,
 ring_status ring_attn_decode_partial(const void* q, const void* k, const void* v, const int32_t* seqlens,
                                      float* partials, float* part_lse, int B, int Hq, int Hkv, int Smax, int D, int P,
                                      float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !seqlens || !aligned16(partials) || !aligned16(part_lse))
-    return RING_EINVAL;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Smax < 1 || P < 1 || D < 1 || Hq % Hkv || Smax % P) return RING_EINVAL;
-  if (!good_scale(scale)) return RING_EINVAL;
-  if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
-  if ((long long)B * Smax * Hkv * D >= (1LL << 42)) return RING_EINVAL;
-  if (dtype != RING_BF16 || D != 128) return RING_EUNSUPPORTED;
-  const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4) return RING_EUNSUPPORTED;
-  const size_t need = decode_workspace_bytes(B, Hq, Hkv, Smax, D, P);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need) return RING_EINVAL;
   DecodeArgs a{};
-  a.q = q; a.k = k; a.v = v; a.seqlens = seqlens;
-  a.partials = partials; a.part_lse = part_lse;
-  decode_workspace_split(workspace, B, Hq, Hkv, Smax, D, P, &a.ws_part, &a.ws_count);
-  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Smax = Smax; a.D = D; a.P = P; a.scale = scale;
+  DecodeExtra x{};
+  ring_status rs = decode_args(q, k, v, seqlens, nullptr, partials, part_lse, B, Hq, Hkv, Smax, D, P, scale, dtype,
+                               workspace, workspace_bytes, &a, &x);
+  if (rs != RING_OK) return rs;
+  return from_cuda(launch_decode_partial(a, x, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ring_status ring_attn_decode_fused(const void* q, const void* k, const void* v, const int32_t* seqlens,
+                                   const int32_t* shard_lens, float* partials, float* part_lse, void* out,
+                                   float* out_lse, int B, int Hq, int Hkv, int Smax, int D, int P, float scale,
+                                   int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if ((seqlens == nullptr) == (shard_lens == nullptr)) return RING_EINVAL;   // exactly one source of lengths
+  if (!aligned16(out)) return RING_EINVAL;
+  if (out_lse && (reinterpret_cast<uintptr_t>(out_lse) & 3u)) return RING_EINVAL;
+  DecodeArgs a{};
+  DecodeExtra x{};
+  ring_status rs = decode_args(q, k, v, seqlens, shard_lens, partials, part_lse, B, Hq, Hkv, Smax, D, P, scale,
+                               dtype, workspace, workspace_bytes, &a, &x);
+  if (rs != RING_OK) return rs;
+  x.out = out;
+  x.out_lse = out_lse;
+  return from_cuda(launch_decode_partial(a, x, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ring_status ring_attn_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                                int32_t* shard_lens, int32_t* n_appended, int B, int T, int Hkv, int Smax, int D,
+                                int P, int block, int dtype, void* stream) {
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new) || !shard_lens ||
+      !n_appended)
+    return RING_EINVAL;
+  if (B < 1 || T < 1 || Hkv < 1 || Smax < 1 || D < 1 || P < 1 || block < 1 || Smax % P) return RING_EINVAL;
+  if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
+  const int eb = dtype == RING_BF16 ? 2 : 4;
+  if (((long long)Hkv * D * eb) % 16) return RING_EUNSUPPORTED;   // rows are copied in 16-byte pieces
+  if ((long long)B * Smax * Hkv * D >= (1LL << 42) || (long long)B * T * Hkv * D >= (1LL << 42)) return RING_EINVAL;
+  AppendArgs a{};
+  a.k_cache = k_cache; a.v_cache = v_cache; a.k_new = k_new; a.v_new = v_new;
+  a.shard_lens = shard_lens; a.n_appended = n_appended;
+  a.B = B; a.T = T; a.Hkv = Hkv; a.Smax = Smax; a.D = D; a.P = P; a.block = block; a.elem_bytes = eb;
   a.err = error_word();
-  return from_cuda(launch_decode_partial(a, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ring_status ring_attn_merge(const float* partials, const float* part_lse, void* out, float* out_lse, int B, int Hq,
@@ -378,7 +432,7 @@ ring_status ring_attn_device_error(int* where) {
   if (word) {
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return RING_ECUDA;
     if (where) *where = (int)word;
-    return RING_ETIMEOUT;
+    return word == kFaultCapacity ? RING_ECAPACITY : RING_ETIMEOUT;
   }
   return RING_OK;
 }
@@ -397,6 +451,7 @@ const char* ring_attn_strerror(ring_status s) {
     case RING_EUNSUPPORTED: return "unsupported configuration";
     case RING_ECUDA: return "CUDA error";
     case RING_ETIMEOUT: return "a bounded wait inside a kernel expired";
+    case RING_ECAPACITY: return "a KV append found its shard full";
   }
   return "unknown status";
 }

@@ -23,8 +23,15 @@
 // memory).  A chunk covered by one sub-split writes its partial directly;
 // otherwise every sub-split writes to the workspace and the last CTA to
 // arrive (atomic counter, reset by that CTA) folds them into the chunk's
-// partial.  The kernel is HBM-bound: each valid K/V byte is read once.
+// partial.  With an output buffer the merge runs in the same launch: the CTA
+// that finishes the last of the P chunks of a (sequence, kv head) -- a second
+// counter, reset the same way -- combines the P partials into out and lse.
+// The valid rows of a chunk come from the sequence length (chunk p holds
+// positions [p*C, (p+1)*C)) or, for a cache filled by the round-robin append
+// of "NVIDIA unveils Helix Parallelism" (KV cache growth), from the chunk's
+// own fill count.  The kernel is HBM-bound: each valid K/V byte is read once.
 #include <cuda_bf16.h>
+#include <type_traits>
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -52,6 +59,23 @@ struct DecGeom {
   int nsub;    // sub-splits per chunk
   int units;
 };
+
+// Valid rows of chunk p of sequence b (always in [0, Cd]; out-of-range
+// lengths are clamped, never trusted): from the chunk's own fill count
+// (kShard) or from the sequence length.
+template <bool kShard>
+__device__ __forceinline__ int chunk_rows(const DecodeArgs& a, const DecodeExtra& x, int Cd, int b, int p) {
+  if constexpr (kShard) return min(max(x.shard_lens[b * a.P + p], 0), Cd);
+  const int len = min(max(a.seqlens[b], 0), a.Smax);
+  return max(0, min(len - p * Cd, Cd));
+}
+// One past the last valid row of chunk p (a row index of the whole cache).
+template <bool kShard>
+__device__ __forceinline__ int chunk_end(const DecodeArgs& a, const DecodeExtra& x, int Cd, int b, int p) {
+  if constexpr (kShard) return p * Cd + min(max(x.shard_lens[b * a.P + p], 0), Cd);
+  const int len = min(max(a.seqlens[b], 0), a.Smax);
+  return min(len, (p + 1) * Cd);
+}
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float* f) {
   const uint32_t u[4] = {w.x, w.y, w.z, w.w};
@@ -130,14 +154,114 @@ struct DecSmem {
   float wl[dec::NCW][G];
   alignas(8) uint64_t full[dec::NST];
   alignas(8) uint64_t empty[dec::NST];
-  int is_last;
+  int is_last;      // set by one thread between two consumer barriers, read by all after the second
   int abort_flag;
 };
 
+// Counts one finished chunk of (b, kv head g) with an acquire-release atomic
+// (after a barrier that follows the CTA's writes of that chunk's partial, so
+// the release publishes them).  True for the arrival that completes the P
+// chunks; that arrival resets the counter for the next call.
+__device__ __forceinline__ bool count_chunk(const DecodeArgs& a, const DecodeExtra& x, int b, int g) {
+  unsigned int* ctr = x.ws_done + (size_t)b * a.Hkv + g;
+  const bool last = atom_add_acq_rel_gpu(ctr, 1u) == (unsigned int)(a.P - 1);
+  if (last) atomicExch(ctr, 0u);
+  return last;
+}
+
+// The merge of the P partials of (b, kv head g) for its G query heads, done
+// by one warp of the CTA whose arrival completed the count of finished chunks
+// (that arrival's acquire, followed by __syncwarp, makes every chunk's partial
+// visible here).  The update of "Lesson 8: Context Parallelism", section 3,
+// applied to whole partial states:
+//   lse = m* + ln sum_p e^(lse_p - m*),  out = sum_p e^(lse_p - lse) O_p.
 template <int G>
+__device__ __noinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
+  constexpr int D = dec::D;
+  __syncwarp();   // lane 0's acquire covers the warp from here on
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(x.out);
+  const size_t bh0 = (size_t)b * a.Hq + g * G;
+  // lse of chunk (q0 + lane) of every head; the first 32 chunks stay in registers
+  auto lse_at = [&](int h, int q) { return q < a.P ? __ldcg(a.part_lse + (bh0 + h) * a.P + q) : -CUDART_INF_F; };
+  float lv[G], mx[G], L[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) mx[h] = lv[h] = lse_at(h, lane);
+  for (int q0 = 32; q0 < a.P; q0 += 32)
+#pragma unroll
+    for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], lse_at(h, q0 + lane));
+#pragma unroll
+  for (int off = 16; off; off >>= 1)
+#pragma unroll
+    for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
+#pragma unroll
+  for (int h = 0; h < G; ++h) L[h] = mx[h] == -CUDART_INF_F ? 0.f : expf(lv[h] - mx[h]);
+  for (int q0 = 32; q0 < a.P; q0 += 32)
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      if (mx[h] != -CUDART_INF_F) L[h] += expf(lse_at(h, q0 + lane) - mx[h]);
+#pragma unroll
+  for (int off = 16; off; off >>= 1)
+#pragma unroll
+    for (int h = 0; h < G; ++h) L[h] += __shfl_xor_sync(0xffffffffu, L[h], off);
+  float inv[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    inv[h] = L[h] > 0.f ? 1.f / L[h] : 0.f;
+    if (lane == 0 && x.out_lse) x.out_lse[bh0 + h] = L[h] > 0.f ? mx[h] + logf(L[h]) : -CUDART_INF_F;
+  }
+  // lane owns dims lane + 32k of every head; the weights of 32 chunks at a time sit
+  // one per lane and reach the others by shuffles; the loads of a chunk are independent
+  float acc[G][D / 32];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) acc[h][k] = 0.f;
+  for (int q0 = 0; q0 < a.P; q0 += 32) {
+    float w[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float v = q0 == 0 ? lv[h] : lse_at(h, q0 + lane);
+      w[h] = inv[h] > 0.f && v != -CUDART_INF_F ? expf(v - mx[h]) * inv[h] : 0.f;
+    }
+    const int n = min(32, a.P - q0);
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float wj = __shfl_sync(0xffffffffu, w[h], j);
+        const float* row = a.partials + ((bh0 + h) * a.P + q0 + j) * D + lane;
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) acc[h][k] = fmaf(wj, __ldcg(row + 32 * k), acc[h][k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) out[(bh0 + h) * D + lane + 32 * k] = __float2bfloat16_rn(acc[h][k]);
+}
+
+// Called by consumer warp 0 (all lanes) after the CTA's writes of a chunk's
+// final partial and a consumer barrier: one lane counts the chunk; the warp
+// that completes the count of (b, g) merges it.  The other consumer warps do
+// not wait.
+template <int G>
+__device__ __forceinline__ void chunk_final_count(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
+  int last = 0;
+  if (lane == 0) last = count_chunk(a, x, b, g);
+  if (__shfl_sync(0xffffffffu, last, 0)) {
+    __syncwarp();   // lane 0's acquire covers the warp
+    merge_bg<G>(a, x, b, g, lane);
+  }
+}
+
+// kMerge: the launch also merges the partials (a.out != null); kShard: valid
+// rows come from per-chunk fill counts (a.shard_lens != null).  Separate
+// instantiations, so that the plain partial kernel carries none of their code.
+template <int G, bool kMerge, bool kShard>
 __global__ void __launch_bounds__(dec::THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DecodeArgs a,
-                  DecGeom geo) {
+                  DecGeom geo, DecodeExtra x) {
   using namespace dec;
   extern __shared__ uint8_t smem_raw[];
   DecSmem<G>& sm = *reinterpret_cast<DecSmem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,9 +293,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         const int g = t % a.Hkv; t /= a.Hkv;
         const int b = t % a.B;
         const int p = t / a.B;
-        const int len = min(max(a.seqlens[b], 0), a.Smax);
         const int r0 = p * geo.Cd + sub * RPS;
-        const int r1 = min(r0 + RPS, min(len, (p + 1) * geo.Cd));
+        const int r1 = min(r0 + RPS, chunk_end<kShard>(a, x, geo.Cd, b, p));
         for (int row = r0; row < r1; row += ROWS) {
           const int s = cnt % NST;
           const uint32_t ph = (cnt / NST) & 1u;
@@ -217,9 +340,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     const int g = t % a.Hkv; t /= a.Hkv;
     const int b = t % a.B;
     const int p = t / a.B;
-    const int len = min(max(a.seqlens[b], 0), a.Smax);
     const int c0 = p * geo.Cd;
-    const int nvalid_chunk = max(0, min(len - c0, geo.Cd));
+    const int nvalid_chunk = chunk_rows<kShard>(a, x, geo.Cd, b, p);
     const int n_live = (nvalid_chunk + RPS - 1) / RPS;
     const int r0 = c0 + sub * RPS;
     const int r1 = min(r0 + RPS, c0 + nvalid_chunk);
@@ -231,6 +353,10 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
           a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = 0.f;
         }
         if (ctid < G) a.part_lse[(size_t)(b * a.Hq + g * G + ctid) * a.P + p] = -CUDART_INF_F;
+        if constexpr (kMerge) {
+          named_bar_sync(1, CT);   // the chunk's partial is written before it is counted
+          if (cw == 0) chunk_final_count<G>(a, x, b, g, lane);
+        }
       }
       continue;
     }
@@ -396,18 +522,16 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       }
     }
     if (n_live > 1) {
-      __threadfence();
       named_bar_sync(1, CT);
       if (ctid == 0) {
         unsigned int* ctr = a.ws_count + (size_t)(b * a.Hkv + g) * a.P + p;
-        const unsigned int old = atomicAdd(ctr, 1u);
+        const unsigned int old = atom_add_acq_rel_gpu(ctr, 1u);
         const int last = (old == (unsigned int)(n_live - 1));
         if (last) atomicExch(ctr, 0u);       // leave the counter at zero for the next call
         sm.is_last = last;
       }
       named_bar_sync(1, CT);
       if (sm.is_last) {
-        __threadfence();
         const float* ws_chunk = a.ws_part + (((size_t)(b * a.Hkv + g) * a.P + p) * geo.nsub) * G * (D + 1);
         for (int e = ctid; e < G * D; e += CT) {
           const int h = e / D, d = e - h * D;
@@ -425,10 +549,18 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         }
       }
     }
+    // this CTA wrote the chunk's final partial: directly, or as the last sub-split to arrive
+    const bool chunk_final = n_live == 1 || sm.is_last;
     // shared fold buffers are free again; leave together if any wait expired
     if (named_bar_any(1, CT, !ok || *abort_flag)) break;
+    if constexpr (kMerge)
+      if (chunk_final && cw == 0) chunk_final_count<G>(a, x, b, g, lane);
   }
 }
+
+// Workspace: sub-split results | per-chunk arrival counters | per-(b, kv head)
+// finished-chunk counters, each part 256-byte aligned.
+static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P) {
   if (B < 1 || Hq < 1 || Hkv < 1 || P < 1 || Smax < P || D < 1 || Hq % Hkv) return 0;
@@ -436,25 +568,26 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P) {
   const int Cd = Smax / P;
   const int nsub = (Cd + dec::RPS - 1) / dec::RPS;
   const size_t chunks = (size_t)B * Hkv * P;
-  size_t part = chunks * nsub * G * (D + 1) * sizeof(float);
-  part = (part + 255) & ~size_t(255);
-  return part + ((chunks * sizeof(unsigned int) + 255) & ~size_t(255));
+  return round256(chunks * nsub * G * (D + 1) * sizeof(float)) + round256(chunks * sizeof(unsigned int)) +
+         round256((size_t)B * Hkv * sizeof(unsigned int));
 }
 
 void decode_workspace_split(void* ws, int B, int Hq, int Hkv, int Smax, int D, int P, float** part,
-                            unsigned int** count) {
+                            unsigned int** count, unsigned int** done) {
   const int G = Hq / Hkv;
   const int Cd = Smax / P;
   const int nsub = (Cd + dec::RPS - 1) / dec::RPS;
   const size_t chunks = (size_t)B * Hkv * P;
-  size_t bytes = chunks * nsub * G * (D + 1) * sizeof(float);
-  bytes = (bytes + 255) & ~size_t(255);
-  *part = reinterpret_cast<float*>(ws);
-  *count = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) + bytes);
+  const size_t b_part = round256(chunks * nsub * G * (D + 1) * sizeof(float));
+  const size_t b_count = round256(chunks * sizeof(unsigned int));
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  *part = reinterpret_cast<float*>(base);
+  *count = reinterpret_cast<unsigned int*>(base + b_part);
+  *done = reinterpret_cast<unsigned int*>(base + b_part + b_count);
 }
 
-template <int G>
-static cudaError_t launch_decode_g(const DecodeArgs& a, cudaStream_t st) {
+template <int G, bool kMerge, bool kShard>
+static cudaError_t launch_decode_g(const DecodeArgs& a, const DecodeExtra& x, cudaStream_t st) {
   CUtensorMap tk, tv;
   if (!make_tmap_bhsd(&tk, a.k, a.B, a.Smax, a.Hkv, a.D, dec::D, dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_tmap_bhsd(&tv, a.v, a.B, a.Smax, a.Hkv, a.D, dec::D, dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -466,22 +599,30 @@ static cudaError_t launch_decode_g(const DecodeArgs& a, cudaStream_t st) {
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
   geo.units = (int)units;
   const size_t smem = sizeof(DecSmem<G>) + 1024;
-  auto kern = decode_kernel<G>;
+  auto kern = decode_kernel<G, kMerge, kShard>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = num_sms();
-  kern<<<grid, dec::THREADS, smem, st>>>(tk, tv, a, geo);
+  kern<<<grid, dec::THREADS, smem, st>>>(tk, tv, a, geo, x);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_partial(const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_decode_partial(const DecodeArgs& a, const DecodeExtra& x, cudaStream_t st) {
   const int G = a.Hq / a.Hkv;
-  switch (G) {
-    case 1: return launch_decode_g<1>(a, st);
-    case 2: return launch_decode_g<2>(a, st);
-    case 4: return launch_decode_g<4>(a, st);
-    default: return cudaErrorNotSupported;
-  }
+  if (G != 1 && G != 2 && G != 4) return cudaErrorNotSupported;
+  const int mode = (x.out != nullptr ? 2 : 0) + (x.shard_lens != nullptr ? 1 : 0);
+  auto pick = [&](auto g) -> cudaError_t {
+    constexpr int GG = decltype(g)::value;
+    switch (mode) {
+      case 0: return launch_decode_g<GG, false, false>(a, x, st);
+      case 1: return launch_decode_g<GG, false, true>(a, x, st);
+      case 2: return launch_decode_g<GG, true, false>(a, x, st);
+      default: return launch_decode_g<GG, true, true>(a, x, st);
+    }
+  };
+  if (G == 1) return pick(std::integral_constant<int, 1>{});
+  if (G == 2) return pick(std::integral_constant<int, 2>{});
+  return pick(std::integral_constant<int, 4>{});
 }
 
 }  // namespace ra
@@ -552,13 +693,14 @@ extern "C" ring_status ring_attn_decode_partial_noalloc(const void* q, const voi
   DecodeArgs a{};
   a.q = q; a.k = k; a.v = v; a.seqlens = seqlens;
   a.partials = partials; a.part_lse = part_lse;
-  decode_workspace_split(ws, B, Hq, Hkv, Smax, D, P, &a.ws_part, &a.ws_count);
+  DecodeExtra x{};
+  decode_workspace_split(ws, B, Hq, Hkv, Smax, D, P, &a.ws_part, &a.ws_count, &x.ws_done);
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Smax = Smax; a.D = D; a.P = P; a.scale = scale;
   a.err = error_word();
   // the arrival counters must start at zero; the previous call may have been cut short
   if (cudaMemsetAsync(a.ws_count, 0, (size_t)B * Hkv * P * sizeof(unsigned int), st) != cudaSuccess)
     return RING_ECUDA;
-  const cudaError_t e = launch_decode_partial(a, st);
+  const cudaError_t e = launch_decode_partial(a, x, st);
   if (e == cudaSuccess) return RING_OK;
   return e == cudaErrorNotSupported ? RING_EUNSUPPORTED : RING_ECUDA;
 }

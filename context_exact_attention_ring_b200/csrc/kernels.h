@@ -40,9 +40,9 @@ cudaError_t launch_merge(const float* part, const float* plse, void* out, float*
 // Split-KV decode.
 struct DecodeArgs {
   const void* q;        // [B,Hq,D] bf16
-  const void* k;        // [B,Smax,Hkv,D] bf16
+  const void* k;        // [B,Smax,Hkv,D] bf16; chunk p = rows [p*Smax/P, (p+1)*Smax/P)
   const void* v;
-  const int32_t* seqlens;
+  const int32_t* seqlens;  // [B]: rows < seqlens[b] are valid (unless DecodeExtra::shard_lens)
   float* partials;      // [B,Hq,P,D]
   float* part_lse;      // [B,Hq,P]
   float* ws_part;       // sub-split results
@@ -51,10 +51,32 @@ struct DecodeArgs {
   float scale;
   unsigned int* err;    // device error word
 };
+// Arguments of the fused / shard-length decode, kept out of DecodeArgs (a
+// separate kernel parameter leaves the register allocation of the plain
+// partial kernel as it was).
+struct DecodeExtra {
+  const int32_t* shard_lens;  // [B,P] or null: the first shard_lens[b,p] rows of chunk p are valid
+  void* out;                  // null, or [B,Hq,D] bf16: merge the P partials in the same launch
+  float* out_lse;             // [B,Hq] or null (with out)
+  unsigned int* ws_done;      // per-(b, kv head) finished-chunk counters (zero between calls)
+};
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P);
 void decode_workspace_split(void* ws, int B, int Hq, int Hkv, int Smax, int D, int P, float** part,
-                            unsigned int** count);
-cudaError_t launch_decode_partial(const DecodeArgs& a, cudaStream_t st);
+                            unsigned int** count, unsigned int** done);
+cudaError_t launch_decode_partial(const DecodeArgs& a, const DecodeExtra& x, cudaStream_t st);
+
+// Round-robin KV append (one CTA per sequence).
+struct AppendArgs {
+  void* k_cache;        // [B,Smax,Hkv,D]
+  void* v_cache;
+  const void* k_new;    // [B,T,Hkv,D]
+  const void* v_new;
+  int32_t* shard_lens;  // [B,P], read and advanced
+  int32_t* n_appended;  // [B], read and advanced
+  int B, T, Hkv, Smax, D, P, block, elem_bytes;
+  unsigned int* err;    // device error word (capacity overflow)
+};
+cudaError_t launch_kv_append(const AppendArgs& a, cudaStream_t st);
 
 // Driver entry point for building TMA descriptors (resolved at run time, so
 // the library does not link libcuda).

@@ -20,6 +20,8 @@ enum WaitSite : unsigned int {
   kWaitSFull = 5, kWaitPFull = 6, kWaitOFinal = 7, kWaitTeardown = 8,
   kWaitDecodeFull = 9, kWaitDecodeEmpty = 10, kWaitSelftest = 11,
 };
+// Not a wait: a KV append found the target shard full and dropped the token.
+constexpr unsigned int kFaultCapacity = 0x100;
 
 // Two seconds: far above any legitimate wait inside these kernels.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -372,6 +374,17 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Arrival on a GPU-scope counter, acquire-release.  Pattern: every thread of
+// the CTA writes its results, the CTA synchronises (bar.sync), one thread
+// arrives; the release is cumulative, so it publishes the whole CTA's
+// writes.  The arriver that sees the final count has acquired every earlier
+// arriver's writes and hands them to its CTA with another bar.sync.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

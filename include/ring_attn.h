@@ -51,7 +51,8 @@ typedef enum {
   RING_EINVAL = -1,        /* bad argument: null/misaligned pointer, shape not divisible, ... */
   RING_EUNSUPPORTED = -2,  /* valid but not built: head dim, dtype combination */
   RING_ECUDA = -3,         /* a CUDA runtime / driver call or a launch failed */
-  RING_ETIMEOUT = -4       /* a bounded wait inside a kernel expired */
+  RING_ETIMEOUT = -4,      /* a bounded wait inside a kernel expired */
+  RING_ECAPACITY = -5      /* a KV append found its shard full (see ring_attn_kv_append) */
 } ring_status;
 
 /*
@@ -263,6 +264,64 @@ ring_status ring_attn_decode(const void* q, const void* k, const void* v, const 
                              int P, float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * ring_attn_decode_fused -- the whole split-KV decode in ONE launch: the
+ * per-chunk partials of ring_attn_decode_partial, and the merge of
+ * ring_attn_merge done by the CTA that finishes the last of the P chunks of
+ * each (sequence, kv head) ("NVIDIA unveils Helix Parallelism", Phase 1: the
+ * KV-parallel partial results are combined once per token; the combine is
+ * the section-3 update of "Lesson 8" applied to whole partial states).
+ *
+ * Valid rows come from exactly one of:
+ *   seqlens [B] int32     rows j < seqlens[b] of the whole cache (chunk p
+ *                         covers rows [p*Smax/P, (p+1)*Smax/P)), as in
+ *                         ring_attn_decode_partial;
+ *   shard_lens [B,P] int32  the first shard_lens[b*P+p] rows of chunk p (a
+ *                         cache filled shard by shard, e.g. by
+ *                         ring_attn_kv_append); other rows are ignored.
+ * Pass the other pointer as NULL.  Lengths outside their range are clamped.
+ * partials [B,Hq,P,D] / part_lse [B,Hq,P] float receive the per-chunk results
+ * as in ring_attn_decode_partial (caller buffers, also read by the merge);
+ * out [B,Hq,D] bf16 and out_lse [B,Hq] float (may be NULL) the merged
+ * result.  The workspace is ring_attn_decode_workspace_bytes(...) bytes,
+ * 256-byte aligned; its counters must be zero before the first call on it and
+ * every call leaves them zero.  Calls that share a workspace must not overlap
+ * on the GPU.  Errors as ring_attn_decode_partial, plus RING_EINVAL unless
+ * exactly one of seqlens / shard_lens is given, or for a null or misaligned
+ * out.
+ */
+ring_status ring_attn_decode_fused(const void* q, const void* k, const void* v, const int32_t* seqlens,
+                                   const int32_t* shard_lens, float* partials, float* part_lse, void* out,
+                                   float* out_lse, int B, int Hq, int Hkv, int Smax, int D, int P, float scale,
+                                   int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ring_attn_kv_append -- append T new tokens per sequence to a KV cache
+ * sharded over P KV-parallel ranks, round-robin by blocks ("NVIDIA unveils
+ * Helix Parallelism", on growing the KV cache: the first block of new tokens
+ * goes to rank 0, the next to rank 1, and so on, so that every rank's share
+ * grows evenly).
+ *
+ * k_cache, v_cache [B,Smax,Hkv,D]: rank p's shard is rows [p*C, (p+1)*C),
+ * C = Smax/P, of which the first shard_lens[b*P+p] are filled.  k_new, v_new
+ * [B,T,Hkv,D] hold the new tokens in order.  n_appended [B] counts the tokens
+ * appended to each sequence so far (0 after the prompt).  Token j of sequence
+ * b has append index n = n_appended[b] + j and goes to rank (n / block) mod P,
+ * at row shard_lens[b*P+p] of that shard (after the earlier tokens of this
+ * call that went there).  On return shard_lens and n_appended have advanced.
+ * All of these are device buffers; lengths outside [0, C] (counts below 0)
+ * are clamped.  A token whose shard is full is not written, the shard's
+ * count stays at C, and the next ring_attn_device_error() reports
+ * RING_ECAPACITY; nothing is written outside the shard.
+ * dtype RING_BF16 or RING_FP32 (the element type of cache and tokens).
+ * Returns RING_EINVAL for null/misaligned pointers, sizes < 1, Smax % P != 0,
+ * block < 1; RING_EUNSUPPORTED if a token row (Hkv*D elements) is not a
+ * multiple of 16 bytes; RING_ECUDA on launch failure.
+ */
+ring_status ring_attn_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                                int32_t* shard_lens, int32_t* n_appended, int B, int T, int Hkv, int Smax,
+                                int D, int P, int block, int dtype, void* stream);
+
+/*
  * ring_attn_sched_stats -- the scheduler's host-side view of one (batch, head)
  * of a causal or full ring, without running anything: per-rank unmasked
  * chunk pairs (a diagonal pair counts once; "Lesson 8", section 4B: 2P+1 per
@@ -279,9 +338,10 @@ ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile
 /*
  * ring_attn_device_error -- synchronise the current device and read-and-clear
  * the library's device error word.  Returns RING_ETIMEOUT if a bounded wait
- * in any kernel expired since the last call, RING_ECUDA if the device
- * reports an error, else RING_OK.  `where` (may be NULL) receives a code of
- * the wait that expired (0 if none).
+ * in any kernel expired since the last call, RING_ECAPACITY if a KV append
+ * dropped a token because its shard was full, RING_ECUDA if the device
+ * reports an error, else RING_OK.  `where` (may be NULL) receives the code
+ * of the site that recorded the error (0 if none).
  */
 ring_status ring_attn_device_error(int* where);
 

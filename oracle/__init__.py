@@ -17,6 +17,9 @@ Contents
                 blockwise recurrence reaches the oracle's value.
   merge.py      the direct formula for combining normalised partial
                 attention results (O_p, lse_p).
+  helix.py      the round-robin placement of appended KV tokens across
+                KV-parallel ranks ("NVIDIA unveils Helix Parallelism"),
+                simulated one token at a time.
 
 Parity pins for every function live in ``tests/test_oracle_*.py``; none of
 them is "parity unpinned".

@@ -1,0 +1,46 @@
+"""Round-robin placement of appended KV tokens across KV-parallel ranks.
+
+TEST INFRASTRUCTURE (see the package docstring).
+
+Source: "NVIDIA unveils Helix Parallelism", on growing the KV cache during
+decoding: writing every new token to one GPU would make a memory hotspot, so
+new tokens are dealt out by blocks -- the first block to GPU 0, the next to
+GPU 1, and so on -- and every KV-parallel rank's share grows evenly.
+
+Reading: "and so on" wraps around after the last rank (block i goes to rank
+i mod P), a block is `block` consecutive appended tokens of one sequence, and
+inside a rank's shard tokens keep their arrival order.
+
+Everything here is a step-by-step simulation (one token at a time); no closed
+form is used, so the closed forms in the tests pin it.
+"""
+from __future__ import annotations
+
+
+def append_rank(n: int, block: int, P: int) -> int:
+    """Rank that receives the n-th appended token (n = 0, 1, ...): block
+    n // block, dealt to the ranks in turn."""
+    return (n // block) % P
+
+
+def simulate_appends(shards: list[list], n_appended: int, tokens: list, block: int, P: int, capacity: int):
+    """Append `tokens` one by one to `shards` (a list of P lists, each the
+    shard's rows in order), starting at append index `n_appended`.
+
+    A token whose shard already holds `capacity` rows is dropped.  Returns
+    (shards, n_appended_after, placements, dropped), where placements[j] is
+    (rank, row) for token j, or None if it was dropped.
+    """
+    shards = [list(s) for s in shards]
+    placements, dropped = [], 0
+    n = n_appended
+    for tok in tokens:
+        p = append_rank(n, block, P)
+        if len(shards[p]) < capacity:
+            placements.append((p, len(shards[p])))
+            shards[p].append(tok)
+        else:
+            placements.append(None)
+            dropped += 1
+        n += 1
+    return shards, n, placements, dropped
