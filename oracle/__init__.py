@@ -7,7 +7,9 @@ imports it, and it imports nothing from the product: the two share no code.
 
 Contents
   attn_fp64.c   the definition of (causal / GQA / variable-length) attention
-                in fp64, threaded over query rows          -> ``attention_rows``
+                in fp64, threaded over query rows          -> ``attention_rows``;
+                and its gradients (the calculus of that
+                definition; the pages give no backward)    -> ``attention_bwd``
   brute.py      a second, independent numpy fp64 oracle that materialises the
                 whole score matrix (tiny shapes only)     -> ``brute``
   schedule.py   the chunk assignment / ring rotation / causal workload
@@ -61,6 +63,12 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_double,
             ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         lib.oracle_cores.restype = ctypes.c_int
+        lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_attn_bwd.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -111,6 +119,37 @@ def attention_rows(q, k, v, rows, *, scale: float, causal: bool,
     if rc != 0:
         raise ValueError(f"oracle_attn_rows failed with code {rc}")
     return out, lse
+
+
+def attention_bwd(q, k, v, dout, *, scale: float, causal: bool, qpos=None, kpos=None, threads: int = 0):
+    """fp64 gradients of L = sum(dout * out) with respect to q, k, v (the
+    calculus of the attention definition; see attn_fp64.c).
+
+    q, dout [B,Sq,Hq,D], k/v [B,Skv,Hkv,D] (read as float32).  Returns
+    (dq [B,Sq,Hq,D], dk [B,Skv,Hkv,D], dv [B,Skv,Hkv,D]) float64.
+    """
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, Sq, Hq, D = q.shape
+    Bk, Skv, Hkv, Dk = k.shape
+    assert Bk == B and Dk == D and v.shape == k.shape and dout.shape == q.shape and Hq % Hkv == 0
+    dq = np.zeros(q.shape, dtype=np.float64)
+    dk = np.zeros(k.shape, dtype=np.float64)
+    dv = np.zeros(k.shape, dtype=np.float64)
+    keep = []
+
+    def ptr(a):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+        keep.append(a)
+        return a.ctypes.data
+
+    rc = _load().oracle_attn_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, B, Sq, Skv, Hq,
+                                 Hkv, D, ptr(qpos), ptr(kpos), int(bool(causal)), float(scale), dq.ctypes.data,
+                                 dk.ctypes.data, dv.ctypes.data, int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd failed with code {rc}")
+    return dq, dk, dv
 
 
 def all_rows(B: int, H: int, S: int) -> np.ndarray:

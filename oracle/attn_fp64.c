@@ -132,6 +132,7 @@ int oracle_attn_rows(const float *q, const float *k, const float *v,
   }
   if (nthreads <= 0) nthreads = oracle_cores();
   if (nthreads > nrows) nthreads = nrows > 0 ? (int)nrows : 1;
+  if (nthreads < 1) nthreads = 1;
   job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
   pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
   if (!jobs || !th) { free(jobs); free(th); return 2; }
@@ -145,6 +146,126 @@ int oracle_attn_rows(const float *q, const float *k, const float *v,
     J->r0 = nrows * t / nthreads; J->r1 = nrows * (t + 1) / nthreads;
     J->out = out; J->lse = lse;
     if (pthread_create(&th[t], NULL, worker, J) != 0) { J->r1 = J->r0; err = 3; th[t] = 0; }
+  }
+  for (int t = 0; t < nthreads; ++t) {
+    if (th[t]) pthread_join(th[t], NULL);
+    if (jobs[t].err) err = 2;
+  }
+  free(jobs); free(th);
+  return err;
+}
+
+/*
+ * Backward of the same attention: the gradients of L = sum(dout * out) with
+ * respect to q, k and v.  The pages give no backward; this is the calculus of
+ * the definition above, written out with the whole score row materialised:
+ *
+ *   for each query row (b, h, i), g = h / (Hq/Hkv), over its allowed keys J:
+ *     s_j    = scale * q_i . k_j ,  lse = log sum_j exp(s_j)
+ *     p_j    = exp(s_j - lse)                    (the softmax weights)
+ *     dp_j   = dout_i . v_j
+ *     delta  = sum_j p_j dp_j                    (= dout_i . out_i)
+ *     ds_j   = p_j (dp_j - delta)                (derivative through softmax)
+ *     dq_i   = scale * sum_j ds_j k_j
+ *     dk_j  += scale * ds_j q_i                  (summed over rows and the
+ *     dv_j  += p_j dout_i                         query heads of group g)
+ *
+ * Layouts as above; dout [B, Sq, Hq, D]; dq [B, Sq, Hq, D] and dk, dv
+ * [B, Skv, Hkv, D] are double and are overwritten.  Threads split the
+ * (b, kv head) pairs, so the dk / dv sums need no locks.
+ */
+typedef struct {
+  const float *q, *k, *v, *dout;
+  int B, Sq, Skv, Hq, Hkv, D;
+  const int64_t *qpos, *kpos;
+  int causal;
+  double scale;
+  double *dq, *dk, *dv;
+  int t, nthreads, err;
+} bjob_t;
+
+static void *bwd_worker(void *arg) {
+  bjob_t *J = (bjob_t *)arg;
+  const int G = J->Hq / J->Hkv, D = J->D;
+  double *s = (double *)malloc(sizeof(double) * (size_t)(J->Skv > 0 ? J->Skv : 1));
+  double *dp = (double *)malloc(sizeof(double) * (size_t)(J->Skv > 0 ? J->Skv : 1));
+  if (!s || !dp) { free(s); free(dp); J->err = 1; return NULL; }
+  for (int bg = J->t; bg < J->B * J->Hkv; bg += J->nthreads) {
+    const int b = bg / J->Hkv, g = bg % J->Hkv;
+    for (int h = g * G; h < (g + 1) * G; ++h) {
+      for (int i = 0; i < J->Sq; ++i) {
+        const float *qi = J->q + (((int64_t)b * J->Sq + i) * J->Hq + h) * D;
+        const float *oi = J->dout + (((int64_t)b * J->Sq + i) * J->Hq + h) * D;
+        const int64_t qp = J->qpos ? J->qpos[i] : i;
+        double m = -INFINITY;
+        for (int j = 0; j < J->Skv; ++j) {
+          const int64_t kp = J->kpos ? J->kpos[j] : j;
+          if (J->causal && kp > qp) { s[j] = -INFINITY; continue; }
+          const float *kj = J->k + (((int64_t)b * J->Skv + j) * J->Hkv + g) * D;
+          double acc = 0.0;
+          for (int d = 0; d < D; ++d) acc += (double)qi[d] * (double)kj[d];
+          s[j] = J->scale * acc;
+          if (s[j] > m) m = s[j];
+        }
+        double *dqi = J->dq + (((int64_t)b * J->Sq + i) * J->Hq + h) * D;
+        for (int d = 0; d < D; ++d) dqi[d] = 0.0;
+        if (m == -INFINITY) continue;              /* no allowed key: no gradient */
+        double Z = 0.0;
+        for (int j = 0; j < J->Skv; ++j)
+          if (s[j] != -INFINITY) Z += exp(s[j] - m);
+        const double lse = m + log(Z);
+        double delta = 0.0;
+        for (int j = 0; j < J->Skv; ++j) {
+          if (s[j] == -INFINITY) { dp[j] = 0.0; continue; }
+          const float *vj = J->v + (((int64_t)b * J->Skv + j) * J->Hkv + g) * D;
+          double acc = 0.0;
+          for (int d = 0; d < D; ++d) acc += (double)oi[d] * (double)vj[d];
+          dp[j] = acc;
+          delta += exp(s[j] - lse) * acc;
+        }
+        for (int j = 0; j < J->Skv; ++j) {
+          if (s[j] == -INFINITY) continue;
+          const double p = exp(s[j] - lse);
+          const double ds = p * (dp[j] - delta);
+          const float *kj = J->k + (((int64_t)b * J->Skv + j) * J->Hkv + g) * D;
+          double *dkj = J->dk + (((int64_t)b * J->Skv + j) * J->Hkv + g) * D;
+          double *dvj = J->dv + (((int64_t)b * J->Skv + j) * J->Hkv + g) * D;
+          for (int d = 0; d < D; ++d) {
+            dqi[d] += J->scale * ds * (double)kj[d];
+            dkj[d] += J->scale * ds * (double)qi[d];
+            dvj[d] += p * (double)oi[d];
+          }
+        }
+      }
+    }
+  }
+  free(s);
+  free(dp);
+  return NULL;
+}
+
+/* Returns 0 on success, nonzero on a bad argument or an allocation failure. */
+int oracle_attn_bwd(const float *q, const float *k, const float *v, const float *dout,
+                    int B, int Sq, int Skv, int Hq, int Hkv, int D,
+                    const int64_t *qpos, const int64_t *kpos, int causal, double scale,
+                    double *dq, double *dk, double *dv, int nthreads) {
+  if (B <= 0 || Sq <= 0 || Skv < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return 1;
+  for (int64_t e = 0; e < (int64_t)B * Skv * Hkv * D; ++e) { dk[e] = 0.0; dv[e] = 0.0; }
+  if (nthreads <= 0) nthreads = oracle_cores();
+  if (nthreads > B * Hkv) nthreads = B * Hkv;
+  if (nthreads < 1) nthreads = 1;
+  bjob_t *jobs = (bjob_t *)calloc((size_t)nthreads, sizeof(bjob_t));
+  pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+  if (!jobs || !th) { free(jobs); free(th); return 2; }
+  int err = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    bjob_t *J = &jobs[t];
+    J->q = q; J->k = k; J->v = v; J->dout = dout;
+    J->B = B; J->Sq = Sq; J->Skv = Skv; J->Hq = Hq; J->Hkv = Hkv; J->D = D;
+    J->qpos = qpos; J->kpos = kpos; J->causal = causal; J->scale = scale;
+    J->dq = dq; J->dk = dk; J->dv = dv;
+    J->t = t; J->nthreads = nthreads;
+    if (pthread_create(&th[t], NULL, bwd_worker, J) != 0) { err = 3; th[t] = 0; }
   }
   for (int t = 0; t < nthreads; ++t) {
     if (th[t]) pthread_join(th[t], NULL);
