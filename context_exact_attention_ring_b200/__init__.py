@@ -41,7 +41,8 @@ EXPORTED = (
     "ring_attn_state_finalize", "ring_attn_decode_partial", "ring_attn_decode_workspace_bytes", "ring_attn_decode",
     "ring_attn_merge", "ring_attn_sched_stats", "ring_attn_device_error", "ring_attn_strerror",
     "ring_attn_version", "ring_attn_built_arch", "ring_attn_selftest_wait", "ring_attn_decode_partial_noalloc",
-    "ring_attn_decode_fused", "ring_attn_kv_append",
+    "ring_attn_decode_fused", "ring_attn_kv_append", "ring_attn_bwd", "ring_attn_bwd_delta",
+    "ring_attn_bwd_workspace_bytes", "ring_attn_step_bwd",
 )
 
 
@@ -83,6 +84,9 @@ def lib():
         "ring_attn_decode_fused": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz,
                                    vp],
         "ring_attn_kv_append": [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp],
+        "ring_attn_bwd": [vp] * 9 + [i32] * 8 + [f32, i32, vp, sz, vp],
+        "ring_attn_bwd_delta": [vp, vp, vp, i32, i32, i32, i32, i32, vp],
+        "ring_attn_step_bwd": [vp] * 9 + [ctypes.POINTER(ChunkIds), i32, i32, i32, i32, f32, i32, vp],
         "ring_attn_merge": [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp],
         "ring_attn_sched_stats": [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp],
         "ring_attn_device_error": [ctypes.POINTER(ctypes.c_int)],
@@ -98,6 +102,8 @@ def lib():
     L.ring_attn_strerror.restype = ctypes.c_char_p
     L.ring_attn_decode_workspace_bytes.argtypes = [i32] * 6
     L.ring_attn_decode_workspace_bytes.restype = sz
+    L.ring_attn_bwd_workspace_bytes.argtypes = [i32] * 3
+    L.ring_attn_bwd_workspace_bytes.restype = sz
     _lib = L
     return L
 
@@ -188,6 +194,72 @@ def ring_attn_fwd_simt(q, k, v, P, causal=True, layout="zigzag", scale=None, out
     return _prefill("ring_attn_fwd_simt", q, k, v, P, causal, layout, scale, out, lse)
 
 
+def ring_attn_bwd_delta(out, dout, delta=None):
+    """delta [B,Hq,S] = rowsum(dout * out) for out, dout [B,S,Hq,D]."""
+    _cuda(out, dout, delta)
+    B, S, Hq, D = out.shape
+    if delta is None:
+        delta = torch.empty((B, Hq, S), device=out.device, dtype=torch.float32)
+    _check(lib().ring_attn_bwd_delta(_ptr(out), _ptr(dout), _ptr(delta), B, Hq, S, D, _dtype_code(out), _stream()),
+           "ring_attn_bwd_delta")
+    return delta
+
+
+def ring_attn_bwd(q, k, v, out, lse, dout, P, causal=True, layout="zigzag", scale=None, dq=None, dk=None, dv=None,
+                  workspace=None):
+    """Gradients (dq, dk, dv) of the whole ring for the output gradient dout."""
+    _cuda(q, k, v, out, lse, dout, dq, dk, dv, workspace)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out.shape != q.shape or dout.shape != q.shape or dout.dtype != q.dtype or out.dtype != q.dtype:
+        raise ValueError("out and dout must match q")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(int(lib().ring_attn_bwd_workspace_bytes(B, Hq, S)), device=q.device,
+                                dtype=torch.uint8)
+    st = lib().ring_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                             _ptr(dv), B, Hq, Hkv, S, D, int(P), int(bool(causal)), _layout(layout), scale,
+                             _dtype_code(q), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, "ring_attn_bwd")
+    return dq, dk, dv
+
+
+def ring_attn_step_bwd(q_shard, kchunk, vchunk, dout_shard, lse, delta, dq_acc, dk_acc, dv_acc, q_ids, kv_ids,
+                       chunk_len, causal=True, scale=None, stripes=0):
+    """One backward hop: add this block's share to dq_acc and the shard's share
+    to dk_acc, dv_acc (float32, in place)."""
+    _cuda(q_shard, kchunk, vchunk, dout_shard, lse, delta, dq_acc, dk_acc, dv_acc)
+    B, Sq, Hq, D = q_shard.shape
+    Hkv = kchunk.shape[2]
+    ids = _chunk_ids(q_ids, kv_ids, chunk_len, causal, stripes)
+    if Sq != len(q_ids) * chunk_len or kchunk.shape[1] != len(kv_ids) * chunk_len:
+        raise ValueError("shard / chunk buffers do not match the chunk ids")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = lib().ring_attn_step_bwd(_ptr(q_shard), _ptr(kchunk), _ptr(vchunk), _ptr(dout_shard), _ptr(lse),
+                                  _ptr(delta), _ptr(dq_acc), _ptr(dk_acc), _ptr(dv_acc), ctypes.byref(ids), B, Hq,
+                                  Hkv, D, scale, _dtype_code(q_shard), _stream())
+    _check(st, "ring_attn_step_bwd")
+
+
+def _chunk_ids(q_ids, kv_ids, chunk_len, causal, stripes):
+    if not (1 <= len(q_ids) <= RING_MAX_CHUNKS_PER_RANK and 1 <= len(kv_ids) <= RING_MAX_CHUNKS_PER_RANK):
+        raise ValueError(f"1..{RING_MAX_CHUNKS_PER_RANK} chunk ids expected")
+    ids = ChunkIds()
+    ids.n_q = len(q_ids)
+    ids.n_kv = len(kv_ids)
+    for i, c in enumerate(q_ids):
+        ids.q[i] = int(c)
+    for i, c in enumerate(kv_ids):
+        ids.kv[i] = int(c)
+    ids.chunk_len = int(chunk_len)
+    ids.causal = int(bool(causal))
+    ids.stripes = int(stripes)
+    return ids
+
+
 def ring_attn_state_init(m, l, O):
     _cuda(m, l, O)
     B, Hq, S = m.shape
@@ -212,18 +284,7 @@ def ring_attn_step(q_shard, kchunk, vchunk, m, l, O, q_ids, kv_ids, chunk_len, c
     _cuda(q_shard, kchunk, vchunk, m, l, O)
     B, Sq, Hq, D = q_shard.shape
     Hkv = kchunk.shape[2]
-    if not (1 <= len(q_ids) <= RING_MAX_CHUNKS_PER_RANK and 1 <= len(kv_ids) <= RING_MAX_CHUNKS_PER_RANK):
-        raise ValueError(f"1..{RING_MAX_CHUNKS_PER_RANK} chunk ids expected")
-    ids = ChunkIds()
-    ids.n_q = len(q_ids)
-    ids.n_kv = len(kv_ids)
-    for i, c in enumerate(q_ids):
-        ids.q[i] = int(c)
-    for i, c in enumerate(kv_ids):
-        ids.kv[i] = int(c)
-    ids.chunk_len = int(chunk_len)
-    ids.causal = int(bool(causal))
-    ids.stripes = int(stripes)
+    ids = _chunk_ids(q_ids, kv_ids, chunk_len, causal, stripes)
     if Sq != len(q_ids) * chunk_len or kchunk.shape[1] != len(kv_ids) * chunk_len:
         raise ValueError("shard / chunk buffers do not match the chunk ids")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)

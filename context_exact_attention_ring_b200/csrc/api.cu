@@ -200,52 +200,11 @@ ring_status decode_args(const void* q, const void* k, const void* v, const int32
   return RING_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-ring_status ring_attn_fwd_counted(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
-                                  int Hkv, int S, int D, int P, int causal, int layout, float scale, int dtype,
-                                  unsigned long long* counters, void* stream) {
-  Plan p;
-  ring_status rs = ring_plan(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, &p);
-  if (rs != RING_OK) return rs;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == RING_FP32)
-    return from_cuda(launch_attn_simt(p, false, q, k, v, out, lse, nullptr, nullptr, nullptr, scale, st));
-  TcArgs a{q, k, v, out, lse, nullptr, nullptr, nullptr, counters, scale, error_word()};
-  return from_cuda(launch_attn_tc(p, a, st));
-}
-
-ring_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
-                          int S, int D, int P, int causal, int layout, float scale, int dtype, void* stream) {
-  return ring_attn_fwd_counted(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, nullptr,
-                               stream);
-}
-
-ring_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
-                               int Hkv, int S, int D, int P, int causal, int layout, float scale, int dtype,
-                               void* stream) {
-  Plan p;
-  ring_status rs = ring_plan(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, &p);
-  if (rs != RING_OK) return rs;
-  return from_cuda(launch_attn_simt(p, dtype == RING_BF16, q, k, v, out, lse, nullptr, nullptr, nullptr, scale,
-                                    reinterpret_cast<cudaStream_t>(stream)));
-}
-
-ring_status ring_attn_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D, void* stream) {
-  if (!aligned16(m) || !aligned16(l) || !aligned16(O)) return RING_EINVAL;
-  if (B < 1 || Hq < 1 || S_loc < 1 || D < 1 || D % 4) return RING_EINVAL;
-  return from_cuda(launch_state_init(m, l, O, B, Hq, S_loc, D, reinterpret_cast<cudaStream_t>(stream)));
-}
-
-ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* vchunk, float* m, float* l, float* O,
-                           const ring_chunk_ids* ids, int B, int Hq, int Hkv, int D, float scale, int dtype,
-                           void* stream) {
+// Shared checks of the step entry points; fills the step-mode plan.
+ring_status step_plan(const void* q_shard, const void* kchunk, const void* vchunk, const ring_chunk_ids* ids, int B,
+                      int Hq, int Hkv, int D, float scale, int dtype, Plan* out) {
   if (!ids) return RING_EINVAL;
-  if (!aligned16(q_shard) || !aligned16(kchunk) || !aligned16(vchunk) || !aligned16(m) || !aligned16(l) ||
-      !aligned16(O))
-    return RING_EINVAL;
+  if (!aligned16(q_shard) || !aligned16(kchunk) || !aligned16(vchunk)) return RING_EINVAL;
   if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv) return RING_EINVAL;
   if (ids->n_q < 1 || ids->n_q > RING_MAX_CHUNKS_PER_RANK || ids->n_kv < 1 ||
       ids->n_kv > RING_MAX_CHUNKS_PER_RANK || ids->chunk_len < 1 || ids->stripes < 0)
@@ -294,6 +253,108 @@ ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* 
     }
   p.Sq = p.nqc * p.C;
   p.Skv = p.nkc * p.C;
+  *out = p;
+  return RING_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ring_status ring_attn_fwd_counted(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                                  int Hkv, int S, int D, int P, int causal, int layout, float scale, int dtype,
+                                  unsigned long long* counters, void* stream) {
+  Plan p;
+  ring_status rs = ring_plan(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, &p);
+  if (rs != RING_OK) return rs;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == RING_FP32)
+    return from_cuda(launch_attn_simt(p, false, q, k, v, out, lse, nullptr, nullptr, nullptr, scale, st));
+  TcArgs a{q, k, v, out, lse, nullptr, nullptr, nullptr, counters, scale, error_word()};
+  return from_cuda(launch_attn_tc(p, a, st));
+}
+
+ring_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                          int S, int D, int P, int causal, int layout, float scale, int dtype, void* stream) {
+  return ring_attn_fwd_counted(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, nullptr,
+                               stream);
+}
+
+ring_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                               int Hkv, int S, int D, int P, int causal, int layout, float scale, int dtype,
+                               void* stream) {
+  Plan p;
+  ring_status rs = ring_plan(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, &p);
+  if (rs != RING_OK) return rs;
+  return from_cuda(launch_attn_simt(p, dtype == RING_BF16, q, k, v, out, lse, nullptr, nullptr, nullptr, scale,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t ring_attn_bwd_workspace_bytes(int B, int Hq, int S) {
+  if (B < 1 || Hq < 1 || S < 1) return 0;
+  return ((size_t)B * Hq * S * sizeof(float) + 255) & ~size_t(255);
+}
+
+ring_status ring_attn_bwd_delta(const void* out, const void* dout, float* delta, int B, int Hq, int S, int D,
+                                int dtype, void* stream) {
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(delta)) return RING_EINVAL;
+  if (B < 1 || Hq < 1 || S < 1 || D < 1) return RING_EINVAL;
+  if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
+  return from_cuda(launch_bwd_delta(out, dout, delta, B, Hq, S, D, dtype == RING_BF16,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D, int P,
+                          int causal, int layout, float scale, int dtype, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  Plan p;
+  ring_status rs = ring_plan(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, &p);
+  if (rs != RING_OK) return rs;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return RING_EINVAL;
+  const size_t need = ring_attn_bwd_workspace_bytes(B, Hq, S);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need) return RING_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* delta = static_cast<float*>(workspace);
+  cudaError_t e = launch_bwd_delta(out, dout, delta, B, Hq, S, D, dtype == RING_BF16, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  BwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = lse; a.delta = delta;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.scale = scale;
+  return from_cuda(launch_bwd_simt(p, a, dtype == RING_BF16, st));
+}
+
+ring_status ring_attn_step_bwd(const void* q_shard, const void* kchunk, const void* vchunk, const void* dout_shard,
+                               const float* lse, const float* delta, float* dq_acc, float* dk_acc, float* dv_acc,
+                               const ring_chunk_ids* ids, int B, int Hq, int Hkv, int D, float scale, int dtype,
+                               void* stream) {
+  Plan p;
+  ring_status rs = step_plan(q_shard, kchunk, vchunk, ids, B, Hq, Hkv, D, scale, dtype, &p);
+  if (rs != RING_OK) return rs;
+  if (!aligned16(dout_shard) || !aligned16(lse) || !aligned16(delta) || !aligned16(dq_acc) || !aligned16(dk_acc) ||
+      !aligned16(dv_acc))
+    return RING_EINVAL;
+  BwdArgs a{};
+  a.q = q_shard; a.k = kchunk; a.v = vchunk; a.dout = dout_shard; a.lse = lse; a.delta = delta;
+  a.dq_acc = dq_acc; a.dk_acc = dk_acc; a.dv_acc = dv_acc;
+  a.scale = scale;
+  return from_cuda(launch_bwd_simt(p, a, dtype == RING_BF16, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ring_status ring_attn_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D, void* stream) {
+  if (!aligned16(m) || !aligned16(l) || !aligned16(O)) return RING_EINVAL;
+  if (B < 1 || Hq < 1 || S_loc < 1 || D < 1 || D % 4) return RING_EINVAL;
+  return from_cuda(launch_state_init(m, l, O, B, Hq, S_loc, D, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* vchunk, float* m, float* l, float* O,
+                           const ring_chunk_ids* ids, int B, int Hq, int Hkv, int D, float scale, int dtype,
+                           void* stream) {
+  Plan p;
+  ring_status rs = step_plan(q_shard, kchunk, vchunk, ids, B, Hq, Hkv, D, scale, dtype, &p);
+  if (rs != RING_OK) return rs;
+  if (!aligned16(m) || !aligned16(l) || !aligned16(O)) return RING_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == RING_FP32)
     return from_cuda(launch_attn_simt(p, false, q_shard, kchunk, vchunk, nullptr, nullptr, m, l, O, scale, st));

@@ -31,6 +31,27 @@ struct TcArgs {
 };
 cudaError_t launch_attn_tc(const Plan& p, const TcArgs& a, cudaStream_t st);
 
+// Backward (CUDA cores).  Ring mode writes dq, dk, dv (input dtype); step
+// mode adds into the float32 sums dq_acc, dk_acc, dv_acc instead.
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;     // [B,Sq,Hq,D]
+  const float* lse;     // [B,Hq,Sq] of the forward
+  const float* delta;   // [B,Hq,Sq] = rowsum(dout * out)
+  void* dq;             // [B,Sq,Hq,D]
+  void* dk;             // [B,Skv,Hkv,D]
+  void* dv;
+  float* dq_acc;        // step mode
+  float* dk_acc;
+  float* dv_acc;
+  float scale;
+};
+cudaError_t launch_bwd_delta(const void* out, const void* dout, float* delta, int B, int Hq, int S, int D, bool bf16,
+                             cudaStream_t st);
+cudaError_t launch_bwd_simt(const Plan& p, const BwdArgs& a, bool bf16, cudaStream_t st);
+
 cudaError_t launch_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D, cudaStream_t st);
 cudaError_t launch_state_finalize(const float* m, const float* l, const float* O, void* out, float* lse, int B,
                                   int Hq, int S, int D, bool bf16, cudaStream_t st);

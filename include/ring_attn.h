@@ -179,6 +179,57 @@ ring_status ring_attn_state_finalize(const float* m, const float* l, const float
                                      void* stream);
 
 /*
+ * Backward pass.  The pages use the ring for training but give no backward;
+ * the gradients are the calculus of the forward (L = sum(dout * out)):
+ *   P = exp(scale * Q K^T - lse),  dP = dout V^T,  delta_i = dout_i . out_i,
+ *   dS = P o (dP - delta),  dV = P^T dout,  dK = scale * dS^T Q,
+ *   dQ = scale * dS K   (dK, dV summed over the query heads of a group).
+ * P is recomputed from the forward's lse, tile by tile, in the ring's order:
+ * a K/V block gathers dK, dV from the query chunks it meets as it travels
+ * round the ring ("Lesson 8", section 2); each rank's dQ gathers from the
+ * blocks it meets.  float32 arithmetic on CUDA cores for both dtypes.
+ */
+
+/* Bytes of workspace ring_attn_bwd needs (the delta rows); 0 on bad sizes. */
+size_t ring_attn_bwd_workspace_bytes(int B, int Hq, int S);
+
+/*
+ * ring_attn_bwd_delta -- delta[b,h,i] = sum_d dout[b,i,h,d] * out[b,i,h,d]
+ * for out, dout [B,S,Hq,D] of `dtype`; delta [B,Hq,S] float.
+ */
+ring_status ring_attn_bwd_delta(const void* out, const void* dout, float* delta, int B, int Hq, int S, int D,
+                                int dtype, void* stream);
+
+/*
+ * ring_attn_bwd -- gradients of the whole ring of ring_attn_fwd.
+ * q, out, dout, dq [B,S,Hq,D]; k, v, dk, dv [B,S,Hkv,D], all of `dtype`;
+ * lse [B,Hq,S] float as written by the forward.  Split, causal rule, scale and
+ * errors as ring_attn_fwd; workspace (ring_attn_bwd_workspace_bytes bytes,
+ * 256-byte aligned) receives delta.  dq, dk, dv are overwritten; the results
+ * do not depend on the launch order of tiles (no atomics).
+ */
+ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
+                          int P, int causal, int layout, float scale, int dtype, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
+ * ring_attn_step_bwd -- one hop of the backward ring for one rank: the
+ * gradients of attention of the rank's query shard against the K/V block it
+ * holds.  q_shard, dout_shard [B, n_q*C, Hq, D] and kchunk, vchunk
+ * [B, n_kv*C, Hkv, D] as in ring_attn_step; lse, delta [B, Hq, n_q*C] float of
+ * the WHOLE forward (lse of the full attention, delta from its output).
+ * Adds, in place: dq_acc [B, n_q*C, Hq, D] float (this block's share of the
+ * shard's dQ) and dk_acc, dv_acc [B, n_kv*C, Hkv, D] float (the shard's share
+ * of the block's dK, dV, which travel with the block).  Errors as
+ * ring_attn_step.
+ */
+ring_status ring_attn_step_bwd(const void* q_shard, const void* kchunk, const void* vchunk, const void* dout_shard,
+                               const float* lse, const float* delta, float* dq_acc, float* dk_acc, float* dv_acc,
+                               const ring_chunk_ids* ids, int B, int Hq, int Hkv, int D, float scale, int dtype,
+                               void* stream);
+
+/*
  * ring_attn_decode_partial -- split-KV single-token decode, the KV cache
  * sharded along the sequence into P chunks ("Helix Parallelism", Phase 1).
  *

@@ -1,0 +1,127 @@
+"""Backward of the ring on the GPU against the fp64 oracle (oracle.attention_bwd):
+the fused ring backward for every split, float32 and bf16, and the step API
+driven hop by hop (dK, dV travelling with their block).  The forward's own
+out and lse feed the backward, as in training."""
+import numpy as np
+import pytest
+import torch
+
+import context_exact_attention_ring_b200 as ra
+import oracle
+import workloads as W
+from oracle import schedule as sch
+from tests.helpers import host, need_cuda
+
+pytestmark = pytest.mark.gpu
+
+# max |gpu - oracle| <= TOL * max(1, max |oracle|) per gradient.  float32: sums of at most S
+# float32 products and expf (a few ulp) -- measured 3.5e-6; bf16: the bf16 rounding of each
+# gradient (2^-9 of its size) plus that of the forward output inside delta -- measured 4.0e-3
+TOL_BWD_FP32 = 2e-5
+TOL_BWD_BF16 = 1e-2
+
+
+def _dout(cfg, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    dt = torch.float32 if cfg.dtype == "fp32" else torch.bfloat16
+    return torch.randn((cfg.B, cfg.S, cfg.Hq, cfg.D), generator=g, device="cuda").to(dt)
+
+
+def _check(grads, refs, tol, what):
+    for name, x, r in zip(("dq", "dk", "dv"), grads, refs):
+        err = float(np.max(np.abs(host(x) - r)))
+        bound = tol * max(1.0, float(np.max(np.abs(r))))
+        assert np.all(np.isfinite(host(x))), f"{what} {name}"
+        assert err <= bound, f"{what}: max |{name} - oracle| = {err:.3e} > {bound:.3e}"
+
+
+CASES = [
+    W.Prefill("fp32_noncausal_P1", "fp32", False, "contiguous", 1, 2, 2, 256, 64, 1, 601),
+    W.Prefill("fp32_zigzag_gqa", "fp32", True, "zigzag", 1, 4, 2, 1024, 128, 4, 602),
+    W.Prefill("fp32_striped_ragged", "fp32", True, "striped", 1, 2, 1, 768, 64, 3, 603),
+    W.Prefill("bf16_zigzag_gqa", "bf16", True, "zigzag", 1, 8, 2, 2048, 128, 4, 604),
+    W.Prefill("bf16_ragged_chunks", "bf16", True, "zigzag", 2, 3, 3, 1200, 128, 3, 605),
+    W.Prefill("bf16_zigzag4_d64", "bf16", True, "zigzag4", 1, 4, 1, 2048, 64, 2, 606),
+    W.Prefill("bf16_contiguous_noncausal", "bf16", False, "contiguous", 1, 2, 2, 1024, 128, 4, 607),
+]
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
+def test_ring_backward_against_oracle(cfg):
+    need_cuda()
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    dout = _dout(cfg, cfg.seed + 1)
+    out, lse = ra.ring_attn_fwd(q, k, v, cfg.P, causal=cfg.causal, layout=cfg.layout, scale=cfg.scale)
+    dq, dk, dv = ra.ring_attn_bwd(q, k, v, out, lse, dout, cfg.P, causal=cfg.causal, layout=cfg.layout,
+                                  scale=cfg.scale)
+    torch.cuda.synchronize()
+    refs = oracle.attention_bwd(host(q), host(k), host(v), host(dout), scale=cfg.scale, causal=cfg.causal)
+    _check((dq, dk, dv), refs, TOL_BWD_FP32 if cfg.dtype == "fp32" else TOL_BWD_BF16, cfg.name)
+
+
+def test_backward_same_for_every_split():
+    # exact gradients: the split only changes the order of the sums
+    need_cuda()
+    cfg = W.Prefill("splits", "fp32", True, "zigzag", 1, 2, 2, 768, 64, 2, 608)
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    dout = _dout(cfg, 9)
+    ref = None
+    for layout in ("contiguous", "zigzag", "zigzag3", "striped", "contiguous2"):
+        out, lse = ra.ring_attn_fwd(q, k, v, 2, True, layout, cfg.scale)
+        g = ra.ring_attn_bwd(q, k, v, out, lse, dout, 2, True, layout, cfg.scale)
+        torch.cuda.synchronize()
+        if ref is None:
+            ref = [x.clone() for x in g]
+        else:
+            for x, r in zip(g, ref):
+                assert (x - r).abs().max().item() <= 1e-5, layout
+
+
+def test_backward_delta():
+    need_cuda()
+    g = torch.Generator(device="cuda").manual_seed(5)
+    out = torch.randn((2, 100, 3, 128), generator=g, device="cuda").to(torch.bfloat16)
+    dout = torch.randn((2, 100, 3, 128), generator=g, device="cuda").to(torch.bfloat16)
+    delta = ra.ring_attn_bwd_delta(out, dout)
+    ref = np.einsum("bihd,bihd->bhi", host(out).astype(np.float64), host(dout).astype(np.float64))
+    assert np.max(np.abs(host(delta) - ref)) <= 1e-4
+
+
+@pytest.mark.parametrize("dtype,layout,S,P", [("fp32", "zigzag", 1024, 4), ("bf16", "striped", 1536, 3),
+                                              ("fp32", "contiguous", 512, 4)])
+def test_step_backward_ring(dtype, layout, S, P):
+    # every rank meets every block; dK, dV of a block are summed wherever it is met
+    need_cuda()
+    cfg = W.Prefill("stepbwd", dtype, True, layout, 1, 4, 2, S, 64, P, 609)
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    dout = _dout(cfg, 10)
+    out, lse = ra.ring_attn_fwd(q, k, v, P, True, layout, cfg.scale)
+    delta = ra.ring_attn_bwd_delta(out, dout)
+    own = sch.layout_assignment(P, layout)
+    pos = sch.chunk_positions(S, P, layout)
+    C = sch.chunk_len(S, P, layout)
+    stripes = P if layout == "striped" else 0
+    rows = {r: torch.tensor([t for c in own[r] for t in pos[c]], device="cuda") for r in range(P)}
+    B, Hq, Hkv, D = 1, 4, 2, 64
+    dq = torch.zeros((B, S, Hq, D), device="cuda")
+    dk_acc = {s: torch.zeros((B, len(rows[s]), Hkv, D), device="cuda") for s in range(P)}
+    dv_acc = {s: torch.zeros((B, len(rows[s]), Hkv, D), device="cuda") for s in range(P)}
+    for r in range(P):
+        rr = rows[r]
+        qs, ds = q[:, rr].contiguous(), dout[:, rr].contiguous()
+        ls, dl = lse[:, :, rr].contiguous(), delta[:, :, rr].contiguous()
+        dq_r = torch.zeros((B, len(rr), Hq, D), device="cuda")
+        for src in sch.ring_rotation(P, r):
+            kr = rows[src]
+            ra.ring_attn_step_bwd(qs, k[:, kr].contiguous(), v[:, kr].contiguous(), ds, ls, dl, dq_r, dk_acc[src],
+                                  dv_acc[src], own[r], own[src], C, causal=True, scale=cfg.scale, stripes=stripes)
+        dq[:, rr] = dq_r
+    dk = torch.zeros((B, S, Hkv, D), device="cuda")
+    dv = torch.zeros((B, S, Hkv, D), device="cuda")
+    for s in range(P):
+        dk[:, rows[s]] = dk_acc[s]
+        dv[:, rows[s]] = dv_acc[s]
+    torch.cuda.synchronize()
+    refs = oracle.attention_bwd(host(q), host(k), host(v), host(dout), scale=cfg.scale, causal=True)
+    # float32 accumulators on both sides of the bf16 rounding: the bf16 case keeps the bf16 input error only
+    _check((dq, dk, dv), refs, TOL_BWD_FP32 if dtype == "fp32" else 5e-3, f"steps {dtype} {layout}")
