@@ -1,0 +1,137 @@
+"""Ring attention across GPUs: the send/receive loop of "Lesson 8: Context
+Parallelism", section 2, with one process per GPU (torch.distributed).
+
+Rank r keeps its query shard fixed.  At step t it holds the K/V block that
+started on rank (r - t) mod P and folds it into its (m, l, O) state with
+ring_attn_step, while the same block is already on its way to rank r+1 and
+the next one is arriving from rank r-1 (a double buffer: the transfer of the
+next block overlaps the step).  Blocks land in this GPU's own memory before a
+kernel reads them: every kernel reads local memory only.  The backward runs
+the same loop with ring_attn_step_bwd; the dK, dV sums of a block travel with
+it and take one last hop home.
+
+The chunk ownership follows the splits of ring_attn_fwd (see split_chunks);
+the step functions default to this package's kernels and can be replaced
+(tests drive the loop on CPU ranks with a stand-in step).
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def split_chunks(P: int, layout: str) -> list[list[int]]:
+    """Chunk ids owned by each rank, in shard order.  'contiguous[k]': rank r
+    owns chunks r*k .. r*k+k-1; 'zigzag[k]' (k >= 2, default 2): slot j of rank
+    r is chunk (j//2)*P + r for even j and P*k-1-(j//2)*P-r for odd j;
+    'striped': rank r owns its stripe, numbered r (token t on rank t mod P)."""
+    name = layout.rstrip("0123456789")
+    k = int(layout[len(name):] or (2 if name == "zigzag" else 1))
+    if name == "contiguous":
+        return [[r * k + j for j in range(k)] for r in range(P)]
+    if name == "zigzag":
+        if k < 2:
+            raise ValueError(layout)
+        return [[(j // 2) * P + r if j % 2 == 0 else P * k - 1 - (j // 2) * P - r for j in range(k)]
+                for r in range(P)]
+    if name == "striped" and k == 1:
+        return [[r] for r in range(P)]
+    raise ValueError(layout)
+
+
+def shard_rows(S: int, P: int, layout: str, rank: int) -> torch.Tensor:
+    """Token positions of rank `rank`'s shard, in shard order."""
+    if layout.startswith("striped"):
+        return torch.arange(rank, S, P)
+    own = split_chunks(P, layout)
+    C = S // (P * len(own[0]))
+    return torch.cat([torch.arange(c * C, (c + 1) * C) for c in own[rank]])
+
+
+class Ring:
+    """Neighbour exchange on a process group: rank r sends to r+1, receives from r-1."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+
+    def _global(self, r: int) -> int:
+        return r if self.group is None else dist.get_global_rank(self.group, r)
+
+    def shift(self, send: list, recv: list) -> list:
+        """Post sends of `send` to the next rank and receives into `recv` from
+        the previous one; returns the requests (wait on them before using
+        `recv` or reusing `send`)."""
+        if self.world == 1:
+            return []
+        nxt, prv = self._global((self.rank + 1) % self.world), self._global((self.rank - 1) % self.world)
+        ops = [dist.P2POp(dist.isend, t, nxt, self.group) for t in send]
+        ops += [dist.P2POp(dist.irecv, t, prv, self.group) for t in recv]
+        return dist.batch_isend_irecv(ops)
+
+
+def _wait(reqs):
+    for r in reqs:
+        r.wait()
+
+
+def ring_forward(q_shard, k_block, v_block, layout="zigzag", causal=True, scale=None, ring=None, step=None,
+                 new_state=None, finalize=None):
+    """Attention of this rank's query shard against every rank's K/V block.
+
+    q_shard [B, S_loc, Hq, D], k_block, v_block [B, S_loc, Hkv, D]: this rank's
+    shard (its chunks stacked in split_chunks order, or its stripe).  Returns
+    (out [B, S_loc, Hq, D], lse [B, Hq, S_loc]) for the shard."""
+    from . import new_state as _new_state, ring_attn_state_finalize, ring_attn_step
+    ring = ring or Ring()
+    step = step or ring_attn_step
+    P, r = ring.world, ring.rank
+    own = split_chunks(P, layout)
+    C = q_shard.shape[1] // len(own[r])
+    stripes = P if layout.startswith("striped") else 0
+    B, S_loc, Hq, D = q_shard.shape
+    m, l, O = (new_state or _new_state)(B, Hq, S_loc, D, device=q_shard.device)
+    cur = [k_block.contiguous(), v_block.contiguous()]
+    nxt = [torch.empty_like(x) for x in cur]
+    for t in range(P):
+        src = (r - t) % P
+        reqs = ring.shift(cur, nxt) if t < P - 1 else []
+        step(q_shard, cur[0], cur[1], m, l, O, own[r], own[src], C, causal=causal, scale=scale, stripes=stripes)
+        _wait(reqs)
+        if t < P - 1:
+            cur, nxt = nxt, cur
+    return (finalize or ring_attn_state_finalize)(m, l, O, dtype=q_shard.dtype)
+
+
+def ring_backward(q_shard, k_block, v_block, out_shard, lse_shard, dout_shard, layout="zigzag", causal=True,
+                  scale=None, ring=None, step=None, delta_fn=None):
+    """Gradients (dq, dk, dv) of this rank's shard.  dK, dV of a block are
+    summed by every rank it visits, then sent home.  float32 sums; the results
+    take the dtype of q."""
+    from . import ring_attn_bwd_delta, ring_attn_step_bwd
+    ring = ring or Ring()
+    step = step or ring_attn_step_bwd
+    P, r = ring.world, ring.rank
+    own = split_chunks(P, layout)
+    C = q_shard.shape[1] // len(own[r])
+    stripes = P if layout.startswith("striped") else 0
+    delta = (delta_fn or ring_attn_bwd_delta)(out_shard, dout_shard)
+    f32 = dict(device=q_shard.device, dtype=torch.float32)
+    dq = torch.zeros(q_shard.shape, **f32)
+    kv = [k_block.contiguous(), v_block.contiguous()]
+    kv_nxt = [torch.empty_like(x) for x in kv]
+    gr = [torch.zeros(k_block.shape, **f32), torch.zeros(v_block.shape, **f32)]
+    gr_nxt = [torch.empty_like(x) for x in gr]
+    for t in range(P):
+        src = (r - t) % P
+        reqs = ring.shift(kv, kv_nxt) if t < P - 1 else []   # the next block arrives during the step
+        step(q_shard, kv[0], kv[1], dout_shard, lse_shard, delta, dq, gr[0], gr[1], own[r], own[src], C,
+             causal=causal, scale=scale, stripes=stripes)
+        reqs += ring.shift(gr, gr_nxt)                        # this block's sums follow it (home after step P-1)
+        _wait(reqs)
+        if P > 1:
+            gr, gr_nxt = gr_nxt, gr
+            if t < P - 1:
+                kv, kv_nxt = kv_nxt, kv
+    return dq.to(q_shard.dtype), gr[0].to(k_block.dtype), gr[1].to(v_block.dtype)

@@ -1,0 +1,203 @@
+"""The cross-GPU ring loop (context_exact_attention_ring_b200/ring.py) on
+CPU ranks: world sizes 2 to 4 as gloo processes, every split, forward and
+backward.  The kernels need a GPU, so the ranks use a stand-in step written
+here in numpy (the online-softmax update and the blockwise gradient with the
+global lse); what is tested is the loop itself -- which block a rank holds at
+each step, the double-buffered exchange, the dK/dV sums travelling with their
+block and the last hop home -- against the fp64 oracle of the whole problem.
+A one-rank run on the GPU drives the real kernels through the same loop."""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from context_exact_attention_ring_b200 import ring as R
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _positions(ids, C, stripes):
+    if stripes:
+        (c,) = ids
+        return np.arange(C) * stripes + c
+    return np.concatenate([np.arange(c * C, (c + 1) * C) for c in ids])
+
+
+def _scores(q, k, qpos, kpos, scale, causal, G):
+    # q [B,Sq,Hq,D], k [B,Sk,Hkv,D] -> [B,Hq,Sq,Sk] with the causal mask on positions
+    kh = np.repeat(k, G, axis=2)
+    s = np.einsum("bihd,bjhd->bhij", q, kh) * scale
+    if causal:
+        s = np.where(kpos[None, :] <= qpos[:, None], s, -np.inf)
+    return s
+
+
+def fake_new_state(B, Hq, S_loc, D, device="cpu"):
+    return (torch.full((B, Hq, S_loc), -np.inf, dtype=torch.float64), torch.zeros((B, Hq, S_loc), dtype=torch.float64),
+            torch.zeros((B, S_loc, Hq, D), dtype=torch.float64))
+
+
+def fake_step(q, k, v, m, l, O, q_ids, kv_ids, C, causal=True, scale=None, stripes=0):
+    """Section-3 update of the state with one block (numpy, float64)."""
+    qn, kn, vn = (x.double().numpy() for x in (q, k, v))
+    G = qn.shape[2] // kn.shape[2]
+    s = _scores(qn, kn, _positions(q_ids, C, stripes), _positions(kv_ids, C, stripes), scale, causal, G)
+    mm, ll, oo = m.numpy(), l.numpy(), O.numpy()
+    blk = s.max(axis=-1)
+    mt = np.maximum(mm, blk)
+    live = np.isfinite(mt)
+    ms = np.where(live, mt, 0.0)
+    alpha = np.where(np.isfinite(mm), np.exp(mm - ms), 0.0)
+    p = np.exp(s - ms[..., None])
+    lnew = ll * alpha + p.sum(-1)
+    ldiv = np.where(lnew > 0, lnew, 1.0)
+    vh = np.repeat(vn, G, axis=2)
+    pv = np.einsum("bhij,bjhd->bihd", p, vh)
+    onew = oo * np.transpose(alpha * ll / ldiv, (0, 2, 1))[..., None] + pv / np.transpose(ldiv, (0, 2, 1))[..., None]
+    m.copy_(torch.from_numpy(np.where(live, mt, mm)))
+    l.copy_(torch.from_numpy(np.where(live, lnew, ll)))
+    O.copy_(torch.from_numpy(np.where(np.transpose(live, (0, 2, 1))[..., None], onew, oo)))
+
+
+def fake_finalize(m, l, O, dtype=None):
+    return O.clone(), m + torch.log(l)
+
+
+def fake_delta(out, dout):
+    return torch.einsum("bihd,bihd->bhi", out.double(), dout.double())
+
+
+def fake_step_bwd(q, k, v, dout, lse, delta, dq, dk, dv, q_ids, kv_ids, C, causal=True, scale=None, stripes=0):
+    """One block's share of the gradients with the global lse (numpy, float64)."""
+    qn, kn, vn, on = (x.double().numpy() for x in (q, k, v, dout))
+    G = qn.shape[2] // kn.shape[2]
+    s = _scores(qn, kn, _positions(q_ids, C, stripes), _positions(kv_ids, C, stripes), scale, causal, G)
+    p = np.exp(s - lse.double().numpy()[..., None])                   # [B,Hq,Sq,Sk]
+    vh, kh = np.repeat(vn, G, axis=2), np.repeat(kn, G, axis=2)
+    dp = np.einsum("bihd,bjhd->bhij", on, vh)
+    ds = p * (dp - delta.double().numpy()[..., None])
+    B, Sk, Hkv, D = kn.shape
+    dq += torch.from_numpy(scale * np.einsum("bhij,bjhd->bihd", ds, kh)).to(dq.dtype)
+    dkh = scale * np.einsum("bhij,bihd->bjhd", ds, qn)
+    dvh = np.einsum("bhij,bihd->bjhd", p, on)
+    dk += torch.from_numpy(dkh.reshape(B, Sk, Hkv, G, D).sum(3)).to(dk.dtype)
+    dv += torch.from_numpy(dvh.reshape(B, Sk, Hkv, G, D).sum(3)).to(dv.dtype)
+
+
+def _inputs(B, S, Hq, Hkv, D, seed):
+    rng = np.random.default_rng(seed)
+    f = lambda *s: rng.standard_normal(s).astype(np.float32)
+    return f(B, S, Hq, D), f(B, S, Hkv, D), f(B, S, Hkv, D), f(B, S, Hq, D)
+
+
+def _rank(rank, world, port, layout, q_out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        B, S, Hq, Hkv, D = 1, 48 * world, 4, 2, 8
+        scale = 0.4
+        q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 21)
+        rows = R.shard_rows(S, world, layout, rank).numpy()
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows]))
+        out, lse = R.ring_forward(t(q), t(k), t(v), layout=layout, causal=True, scale=scale, step=fake_step,
+                                  new_state=fake_new_state, finalize=fake_finalize)
+        dq, dk, dv = R.ring_backward(t(q).double(), t(k).double(), t(v).double(), out, lse, t(dout).double(),
+                                     layout=layout, causal=True, scale=scale, step=fake_step_bwd,
+                                     delta_fn=fake_delta)
+        q_out.put((rank, rows, out.numpy(), lse.numpy(), dq.numpy(), dk.numpy(), dv.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,layout", [(2, "zigzag"), (3, "contiguous"), (2, "striped"), (3, "zigzag3"),
+                                          (4, "zigzag"), (4, "striped")])
+def test_ring_loop_on_cpu_ranks(world, layout):
+    import oracle
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, layout, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [qq.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    B, S, Hq, Hkv, D = 1, 48 * world, 4, 2, 8
+    q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 21)
+    rows_all = oracle.all_rows(B, Hq, S)
+    ro, rl = oracle.attention_rows(q, k, v, rows_all, scale=0.4, causal=True)
+    ro = ro.reshape(B, Hq, S, D).transpose(0, 2, 1, 3)
+    rl = rl.reshape(B, Hq, S)
+    dq_ref, dk_ref, dv_ref = oracle.attention_bwd(q, k, v, dout, scale=0.4, causal=True)
+    for rank, rows, out, lse, dq, dk, dv in res:
+        np.testing.assert_allclose(out, ro[:, rows], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(lse, rl[:, :, rows], atol=1e-12, rtol=0)
+        # the loop keeps its dQ, dK, dV sums in float32 (as on the GPU): float32 rounding only
+        np.testing.assert_allclose(dq, dq_ref[:, rows], atol=2e-6, rtol=0)
+        np.testing.assert_allclose(dk, dk_ref[:, rows], atol=2e-6, rtol=0)
+        np.testing.assert_allclose(dv, dv_ref[:, rows], atol=2e-6, rtol=0)
+
+
+def test_split_chunks_match_the_schedule_enumerator():
+    from oracle import schedule as sch
+    for P in (1, 2, 3, 4, 8):
+        for layout in ("contiguous", "zigzag", "zigzag3", "zigzag4", "contiguous2", "striped"):
+            assert R.split_chunks(P, layout) == [sch.layout_assignment(P, layout)[r] for r in range(P)]
+    for S, P, layout in ((96, 4, "zigzag"), (60, 3, "striped"), (64, 2, "zigzag4")):
+        pos = sch.chunk_positions(S, P, layout)
+        own = sch.layout_assignment(P, layout)
+        for r in range(P):
+            assert R.shard_rows(S, P, layout, r).tolist() == [t for c in own[r] for t in pos[c]]
+
+
+def _gpu_rank(port, q_out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        import context_exact_attention_ring_b200 as ra
+        import workloads as W
+        cfg = W.Prefill("ring1", "bf16", True, "zigzag", 1, 4, 2, 2048, 128, 1, 33)
+        q, k, v = W.prefill_inputs(cfg, "cuda")
+        g = torch.Generator(device="cuda").manual_seed(3)
+        dout = torch.randn(q.shape, generator=g, device="cuda").to(q.dtype)
+        out, lse = R.ring_forward(q, k, v, layout="zigzag", scale=cfg.scale)
+        ref_o, ref_l = ra.ring_attn_fwd(q, k, v, 1, True, "zigzag", cfg.scale)
+        dq, dk, dv = R.ring_backward(q, k, v, out, lse, dout, layout="zigzag", scale=cfg.scale)
+        rq, rk, rv = ra.ring_attn_bwd(q, k, v, ref_o, ref_l, dout, 1, True, "zigzag", cfg.scale)
+        torch.cuda.synchronize()
+        errs = [(out.float() - ref_o.float()).abs().max().item(), (lse - ref_l).abs().max().item()]
+        errs += [(a.float() - b.float()).abs().max().item() for a, b in ((dq, rq), (dk, rk), (dv, rv))]
+        q_out.put(errs)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_ring_loop_one_gpu_rank_runs_the_kernels():
+    from tests.helpers import need_cuda
+    need_cuda()
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    p = ctx.Process(target=_gpu_rank, args=(_free_port(), qq))
+    p.start()
+    errs = qq.get(timeout=300)
+    p.join(60)
+    assert p.exitcode == 0
+    # one rank: the loop is one step of the tensor-core step kernel against the fused ring kernel
+    assert errs[0] <= 2e-2 and errs[1] <= 1e-3
+    assert max(errs[2:]) <= 3e-2
