@@ -42,7 +42,7 @@ EXPORTED = (
     "ring_attn_merge", "ring_attn_sched_stats", "ring_attn_device_error", "ring_attn_strerror",
     "ring_attn_version", "ring_attn_built_arch", "ring_attn_selftest_wait", "ring_attn_decode_partial_noalloc",
     "ring_attn_decode_fused", "ring_attn_kv_append", "ring_attn_bwd", "ring_attn_bwd_delta",
-    "ring_attn_bwd_workspace_bytes", "ring_attn_step_bwd",
+    "ring_attn_bwd_workspace_bytes", "ring_attn_step_bwd", "ring_attn_bwd_simt",
 )
 
 
@@ -85,6 +85,7 @@ def lib():
                                    vp],
         "ring_attn_kv_append": [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp],
         "ring_attn_bwd": [vp] * 9 + [i32] * 8 + [f32, i32, vp, sz, vp],
+        "ring_attn_bwd_simt": [vp] * 9 + [i32] * 8 + [f32, i32, vp, sz, vp],
         "ring_attn_bwd_delta": [vp, vp, vp, i32, i32, i32, i32, i32, vp],
         "ring_attn_step_bwd": [vp] * 9 + [ctypes.POINTER(ChunkIds), i32, i32, i32, i32, f32, i32, vp],
         "ring_attn_merge": [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp],
@@ -206,7 +207,7 @@ def ring_attn_bwd_delta(out, dout, delta=None):
 
 
 def ring_attn_bwd(q, k, v, out, lse, dout, P, causal=True, layout="zigzag", scale=None, dq=None, dk=None, dv=None,
-                  workspace=None):
+                  workspace=None, _name="ring_attn_bwd"):
     """Gradients (dq, dk, dv) of the whole ring for the output gradient dout."""
     _cuda(q, k, v, out, lse, dout, dq, dk, dv, workspace)
     B, S, Hq, D = q.shape
@@ -220,11 +221,18 @@ def ring_attn_bwd(q, k, v, out, lse, dout, P, causal=True, layout="zigzag", scal
     if workspace is None:
         workspace = torch.empty(int(lib().ring_attn_bwd_workspace_bytes(B, Hq, S)), device=q.device,
                                 dtype=torch.uint8)
-    st = lib().ring_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
-                             _ptr(dv), B, Hq, Hkv, S, D, int(P), int(bool(causal)), _layout(layout), scale,
-                             _dtype_code(q), _ptr(workspace), workspace.numel(), _stream())
-    _check(st, "ring_attn_bwd")
+    st = getattr(lib(), _name)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                               _ptr(dv), B, Hq, Hkv, S, D, int(P), int(bool(causal)), _layout(layout), scale,
+                               _dtype_code(q), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, _name)
     return dq, dk, dv
+
+
+def ring_attn_bwd_simt(q, k, v, out, lse, dout, P, causal=True, layout="zigzag", scale=None, dq=None, dk=None,
+                       dv=None, workspace=None):
+    """The CUDA-core cross-check path of ring_attn_bwd."""
+    return ring_attn_bwd(q, k, v, out, lse, dout, P, causal, layout, scale, dq, dk, dv, workspace,
+                         _name="ring_attn_bwd_simt")
 
 
 def ring_attn_step_bwd(q_shard, kchunk, vchunk, dout_shard, lse, delta, dq_acc, dk_acc, dv_acc, q_ids, kv_ids,

@@ -304,10 +304,10 @@ ring_status ring_attn_bwd_delta(const void* out, const void* dout, float* delta,
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
-ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                          const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D, int P,
-                          int causal, int layout, float scale, int dtype, void* workspace, size_t workspace_bytes,
-                          void* stream) {
+static ring_status bwd_impl(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
+                            int P, int causal, int layout, float scale, int dtype, void* workspace,
+                            size_t workspace_bytes, void* stream, bool simt) {
   Plan p;
   ring_status rs = ring_plan(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, &p);
   if (rs != RING_OK) return rs;
@@ -322,7 +322,24 @@ ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const voi
   a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = lse; a.delta = delta;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.scale = scale;
+  if (dtype == RING_BF16 && !simt) return from_cuda(launch_bwd_tc(p, a, error_word(), st));
   return from_cuda(launch_bwd_simt(p, a, dtype == RING_BF16, st));
+}
+
+ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D, int P,
+                          int causal, int layout, float scale, int dtype, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, workspace,
+                  workspace_bytes, stream, false);
+}
+
+ring_status ring_attn_bwd_simt(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
+                               int P, int causal, int layout, float scale, int dtype, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, workspace,
+                  workspace_bytes, stream, true);
 }
 
 ring_status ring_attn_step_bwd(const void* q_shard, const void* kchunk, const void* vchunk, const void* dout_shard,
@@ -339,7 +356,9 @@ ring_status ring_attn_step_bwd(const void* q_shard, const void* kchunk, const vo
   a.q = q_shard; a.k = kchunk; a.v = vchunk; a.dout = dout_shard; a.lse = lse; a.delta = delta;
   a.dq_acc = dq_acc; a.dk_acc = dk_acc; a.dv_acc = dv_acc;
   a.scale = scale;
-  return from_cuda(launch_bwd_simt(p, a, dtype == RING_BF16, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == RING_BF16) return from_cuda(launch_bwd_tc(p, a, error_word(), st));
+  return from_cuda(launch_bwd_simt(p, a, false, st));
 }
 
 ring_status ring_attn_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D, void* stream) {

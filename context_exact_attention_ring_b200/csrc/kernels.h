@@ -51,6 +51,9 @@ struct BwdArgs {
 cudaError_t launch_bwd_delta(const void* out, const void* dout, float* delta, int B, int Hq, int S, int D, bool bf16,
                              cudaStream_t st);
 cudaError_t launch_bwd_simt(const Plan& p, const BwdArgs& a, bool bf16, cudaStream_t st);
+// Backward on the tensor cores (bf16): a K/V-major launch (dK, dV) then a
+// Q-major launch (dQ).
+cudaError_t launch_bwd_tc(const Plan& p, const BwdArgs& a, unsigned int* err, cudaStream_t st);
 
 cudaError_t launch_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D, cudaStream_t st);
 cudaError_t launch_state_finalize(const float* m, const float* l, const float* O, void* out, float* lse, int B,

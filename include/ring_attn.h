@@ -187,7 +187,8 @@ ring_status ring_attn_state_finalize(const float* m, const float* l, const float
  * P is recomputed from the forward's lse, tile by tile, in the ring's order:
  * a K/V block gathers dK, dV from the query chunks it meets as it travels
  * round the ring ("Lesson 8", section 2); each rank's dQ gathers from the
- * blocks it meets.  float32 arithmetic on CUDA cores for both dtypes.
+ * blocks it meets.  bf16: tensor cores (bf16 products, fp32 accumulation);
+ * float32: CUDA cores.
  */
 
 /* Bytes of workspace ring_attn_bwd needs (the delta rows); 0 on bad sizes. */
@@ -212,6 +213,17 @@ ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const voi
                           const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
                           int P, int causal, int layout, float scale, int dtype, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/*
+ * ring_attn_bwd_simt -- ring_attn_bwd on CUDA cores with float32 FMA for both
+ * dtypes (the bf16 ring_attn_bwd runs on the tensor cores: tcgen05 products
+ * of 128 x 128 tiles, fp32 accumulation in tensor memory).  Slow; it exists
+ * to cross-check the tensor-core path.  Arguments and errors as ring_attn_bwd.
+ */
+ring_status ring_attn_bwd_simt(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
+                               int P, int causal, int layout, float scale, int dtype, void* workspace,
+                               size_t workspace_bytes, void* stream);
 
 /*
  * ring_attn_step_bwd -- one hop of the backward ring for one rank: the

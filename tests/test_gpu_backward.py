@@ -125,3 +125,21 @@ def test_step_backward_ring(dtype, layout, S, P):
     refs = oracle.attention_bwd(host(q), host(k), host(v), host(dout), scale=cfg.scale, causal=True)
     # float32 accumulators on both sides of the bf16 rounding: the bf16 case keeps the bf16 input error only
     _check((dq, dk, dv), refs, TOL_BWD_FP32 if dtype == "fp32" else 5e-3, f"steps {dtype} {layout}")
+
+
+@pytest.mark.parametrize("layout,S,P,Hq,Hkv,D", [("zigzag", 4096, 4, 8, 2, 128), ("striped", 3072, 3, 4, 4, 128),
+                                                 ("contiguous", 2048, 2, 4, 1, 64), ("zigzag4", 4096, 2, 6, 2, 128)])
+def test_tensor_core_backward_matches_cuda_cores(layout, S, P, Hq, Hkv, D):
+    # two independent implementations on the same bf16 inputs and forward results
+    need_cuda()
+    cfg = W.Prefill("tcsimt", "bf16", True, layout, 1, Hq, Hkv, S, D, P, 610)
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    dout = _dout(cfg, 11)
+    out, lse = ra.ring_attn_fwd(q, k, v, P, True, layout, cfg.scale)
+    g1 = ra.ring_attn_bwd(q, k, v, out, lse, dout, P, True, layout, cfg.scale)
+    g2 = ra.ring_attn_bwd_simt(q, k, v, out, lse, dout, P, True, layout, cfg.scale)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    for name, a, b in zip(("dq", "dk", "dv"), g1, g2):
+        scale_ = max(1.0, b.float().abs().max().item())
+        assert (a.float() - b.float()).abs().max().item() <= TOL_BWD_BF16 * scale_, name
