@@ -402,6 +402,10 @@ PROFILE_CASES = {
                                            name="ring_bf16_causal_zigzag4_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
     "tc_full_striped": dataclasses.replace(W.CFG4, layout="striped",
                                            name="ring_bf16_causal_striped_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
+    # backward of the S=128k GQA workload (tensor cores: K/V-major then Q-major launch)
+    "bwd_full": W.CFG4,
+    # backward of the causal zig-zag MHA workload with 1% of keys x8 (a small case for ncu)
+    "bwd": W.CFG3,
     # split-KV decode on 4 x 65536-token sequences (K+V 1.07 GB > L2, lengths U[32k, 64k])
     "decode": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),
     "decode_fused": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),
@@ -419,7 +423,19 @@ def run_profile(args):
     name = args.profile
     cfg = PROFILE_CASES[name]
     dev = torch.device("cuda", 0)
-    if isinstance(cfg, W.Prefill):
+    if isinstance(cfg, W.Prefill) and name.startswith("bwd"):
+        q, k, v = W.prefill_inputs(cfg, dev)
+        g = torch.Generator(device=dev).manual_seed(cfg.seed + 7)
+        dout = torch.randn(q.shape, generator=g, device=dev).to(q.dtype)
+        out, lse = ra.ring_attn_fwd(q, k, v, cfg.P, causal=cfg.causal, layout=cfg.layout, scale=cfg.scale)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(int(ra.lib().ring_attn_bwd_workspace_bytes(cfg.B, cfg.Hq, cfg.S)), device=dev,
+                         dtype=torch.uint8)
+        fn = lambda: ra.ring_attn_bwd(q, k, v, out, lse, dout, cfg.P, causal=cfg.causal, layout=cfg.layout,
+                                      scale=cfg.scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+        # the usual backward convention: 2.5x the forward's FLOPs (the two launches compute 3.5x)
+        work, unit = 2.5 * cfg.flops() / 1e12, "TFLOP/s"
+    elif isinstance(cfg, W.Prefill):
         q, k, v = W.prefill_inputs(cfg, dev)
         out = torch.empty_like(q)
         lse = torch.empty((cfg.B, cfg.Hq, cfg.S), device=dev, dtype=torch.float32)

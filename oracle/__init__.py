@@ -9,7 +9,8 @@ Contents
   attn_fp64.c   the definition of (causal / GQA / variable-length) attention
                 in fp64, threaded over query rows          -> ``attention_rows``;
                 and its gradients (the calculus of that
-                definition; the pages give no backward)    -> ``attention_bwd``
+                definition; the pages give no backward)    -> ``attention_bwd``,
+                ``attention_bwd_dq_rows`` (sampled rows)
   brute.py      a second, independent numpy fp64 oracle that materialises the
                 whole score matrix (tiny shapes only)     -> ``brute``
   schedule.py   the chunk assignment / ring rotation / causal workload
@@ -69,6 +70,11 @@ def _load():
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_double,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_attn_bwd_dq_rows.restype = ctypes.c_int
+        lib.oracle_attn_bwd_dq_rows.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -150,6 +156,23 @@ def attention_bwd(q, k, v, dout, *, scale: float, causal: bool, qpos=None, kpos=
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd failed with code {rc}")
     return dq, dk, dv
+
+
+def attention_bwd_dq_rows(q, k, v, dout, rows, *, scale: float, causal: bool, threads: int = 0):
+    """fp64 dq of the requested query rows (b, h, i) only: each row needs just
+    its own scores, so large problems can be sampled.  Returns [n, D] float64."""
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, S, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    assert Sk == S and v.shape == k.shape and dout.shape == q.shape and Hq % Hkv == 0
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    dq = np.zeros((rows.shape[0], D), dtype=np.float64)
+    rc = _load().oracle_attn_bwd_dq_rows(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, B, S, Hq,
+                                         Hkv, D, int(bool(causal)), float(scale), rows.ctypes.data, rows.shape[0],
+                                         dq.ctypes.data, int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd_dq_rows failed with code {rc}")
+    return dq
 
 
 def all_rows(B: int, H: int, S: int) -> np.ndarray:

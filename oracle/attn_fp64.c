@@ -274,3 +274,92 @@ int oracle_attn_bwd(const float *q, const float *k, const float *v, const float 
   free(jobs); free(th);
   return err;
 }
+
+/*
+ * dq of selected query rows only (the same calculus as oracle_attn_bwd, for
+ * one row at a time: its scores, lse, dp_j, delta and ds_j need only that
+ * row), so large problems can be checked on sampled rows.
+ * rows [nrows][3] = (b, h, i); dq [nrows][D] double.
+ */
+typedef struct {
+  const float *q, *k, *v, *dout;
+  int B, S, Hq, Hkv, D, causal;
+  double scale;
+  const int32_t *rows;
+  int64_t r0, r1;
+  double *dq;
+  int err;
+} qjob_t;
+
+static void *dq_rows_worker(void *arg) {
+  qjob_t *J = (qjob_t *)arg;
+  const int G = J->Hq / J->Hkv, D = J->D;
+  double *s = (double *)malloc(sizeof(double) * (size_t)J->S);
+  double *dp = (double *)malloc(sizeof(double) * (size_t)J->S);
+  if (!s || !dp) { free(s); free(dp); J->err = 1; return NULL; }
+  for (int64_t r = J->r0; r < J->r1; ++r) {
+    const int b = J->rows[3 * r], h = J->rows[3 * r + 1], i = J->rows[3 * r + 2], g = h / G;
+    const float *qi = J->q + (((int64_t)b * J->S + i) * J->Hq + h) * D;
+    const float *oi = J->dout + (((int64_t)b * J->S + i) * J->Hq + h) * D;
+    double *dqi = J->dq + r * D;
+    for (int d = 0; d < D; ++d) dqi[d] = 0.0;
+    const int nj = J->causal ? i + 1 : J->S;
+    double m = -INFINITY;
+    for (int j = 0; j < nj; ++j) {
+      const float *kj = J->k + (((int64_t)b * J->S + j) * J->Hkv + g) * D;
+      const float *vj = J->v + (((int64_t)b * J->S + j) * J->Hkv + g) * D;
+      double a = 0.0, c = 0.0;
+      for (int d = 0; d < D; ++d) {
+        a += (double)qi[d] * (double)kj[d];
+        c += (double)oi[d] * (double)vj[d];
+      }
+      s[j] = J->scale * a;
+      dp[j] = c;
+      if (s[j] > m) m = s[j];
+    }
+    if (nj == 0) continue;
+    double Z = 0.0;
+    for (int j = 0; j < nj; ++j) Z += exp(s[j] - m);
+    const double lse = m + log(Z);
+    double delta = 0.0;
+    for (int j = 0; j < nj; ++j) delta += exp(s[j] - lse) * dp[j];
+    for (int j = 0; j < nj; ++j) {
+      const double ds = exp(s[j] - lse) * (dp[j] - delta);
+      const float *kj = J->k + (((int64_t)b * J->S + j) * J->Hkv + g) * D;
+      for (int d = 0; d < D; ++d) dqi[d] += J->scale * ds * (double)kj[d];
+    }
+  }
+  free(s);
+  free(dp);
+  return NULL;
+}
+
+int oracle_attn_bwd_dq_rows(const float *q, const float *k, const float *v, const float *dout,
+                            int B, int S, int Hq, int Hkv, int D, int causal, double scale,
+                            const int32_t *rows, int64_t nrows, double *dq, int nthreads) {
+  if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return 1;
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0 || i >= S) return 1;
+  }
+  if (nthreads <= 0) nthreads = oracle_cores();
+  if (nthreads > nrows) nthreads = nrows > 0 ? (int)nrows : 1;
+  if (nthreads < 1) nthreads = 1;
+  qjob_t *jobs = (qjob_t *)calloc((size_t)nthreads, sizeof(qjob_t));
+  pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+  if (!jobs || !th) { free(jobs); free(th); return 2; }
+  int err = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    qjob_t *J = &jobs[t];
+    J->q = q; J->k = k; J->v = v; J->dout = dout;
+    J->B = B; J->S = S; J->Hq = Hq; J->Hkv = Hkv; J->D = D; J->causal = causal; J->scale = scale;
+    J->rows = rows; J->r0 = nrows * t / nthreads; J->r1 = nrows * (t + 1) / nthreads; J->dq = dq;
+    if (pthread_create(&th[t], NULL, dq_rows_worker, J) != 0) { err = 3; th[t] = 0; }
+  }
+  for (int t = 0; t < nthreads; ++t) {
+    if (th[t]) pthread_join(th[t], NULL);
+    if (jobs[t].err) err = 2;
+  }
+  free(jobs); free(th);
+  return err;
+}

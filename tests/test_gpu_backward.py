@@ -143,3 +143,34 @@ def test_tensor_core_backward_matches_cuda_cores(layout, S, P, Hq, Hkv, D):
     for name, a, b in zip(("dq", "dk", "dv"), g1, g2):
         scale_ = max(1.0, b.float().abs().max().item())
         assert (a.float() - b.float()).abs().max().item() <= TOL_BWD_BF16 * scale_, name
+
+
+def test_full_size_backward_sampled_rows_and_invariants():
+    # causal zig-zag GQA, B1 Hq32 Hkv8 S131072 D128 P16 (the timed forward workload): dq on
+    # sampled rows of four heads against the row-at-a-time fp64 oracle; dk and dv through
+    # properties that hold at any size: shifting every key by one vector leaves the output
+    # unchanged (sum_j dk_j = 0 per kv head) and the weights of a row sum to one
+    # (sum_j dv_j = sum over the group's rows of dout)
+    need_cuda()
+    cfg = W.CFG4
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    dout = _dout(cfg, 12)
+    out, lse = ra.ring_attn_fwd(q, k, v, cfg.P, True, cfg.layout, cfg.scale)
+    dq, dk, dv = ra.ring_attn_bwd(q, k, v, out, lse, dout, cfg.P, True, cfg.layout, cfg.scale)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    rows = np.array([r for r in W.sample_rows(cfg, 24) if r[1] in (0, 9, 22, 31)], dtype=np.int32)
+    ref = oracle.attention_bwd_dq_rows(host(q), host(k), host(v), host(dout), rows, scale=cfg.scale, causal=True)
+    got = host(dq)[rows[:, 0], rows[:, 2], rows[:, 1]]
+    assert np.max(np.abs(got - ref)) <= TOL_BWD_BF16 * max(1.0, float(np.max(np.abs(ref))))
+    G = cfg.Hq // cfg.Hkv
+    dk64 = dk.double().sum(dim=1).cpu().numpy()                                  # [B, Hkv, D]
+    dv64 = dv.double().sum(dim=1).cpu().numpy()
+    do64 = dout.double().sum(dim=1).reshape(cfg.B, cfg.Hkv, G, cfg.D).sum(2).cpu().numpy()
+    # Two roundings break the identities by random walks: each summed bf16 element (2^-9 of its
+    # size, over S rows), and the bf16 P and dS inside the products -- a query row's bf16 weights
+    # sum to 1 only within about 2^-9, which walks over the S*G rows of dout (or q) of the group
+    walk = lambda x: 8.0 * np.sqrt(cfg.S) * 2.0 ** -9 * float(x.float().pow(2).mean().sqrt().item())
+    rows_walk = lambda y: 4.0 * np.sqrt(cfg.S * G) * 2.0 ** -9 * float(y.float().pow(2).mean().sqrt().item())
+    assert np.max(np.abs(dk64)) <= walk(dk) + cfg.scale * rows_walk(q) * 8.0
+    assert np.max(np.abs(dv64 - do64)) <= walk(dv) + rows_walk(dout)

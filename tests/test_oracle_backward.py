@@ -132,3 +132,14 @@ def test_positions_select_the_same_keys_as_the_causal_rule():
     dq_part, _, _ = oracle.attention_bwd(q[:, 8:], k, v, dout[:, 8:], scale=0.5, causal=True,
                                          qpos=np.arange(8, 16))
     np.testing.assert_allclose(dq_part, a[0][:, 8:], atol=1e-13, rtol=0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_dq_rows_equal_the_full_backward(causal):
+    # the row-at-a-time dq (for large problems) against the full backward pinned above
+    q, k, v, dout = _inputs(2, 50, 4, 2, 16, 17)
+    dq, _, _ = oracle.attention_bwd(q, k, v, dout, scale=0.3, causal=causal)
+    rows = oracle.all_rows(2, 4, 50)
+    got = oracle.attention_bwd_dq_rows(q, k, v, dout, rows, scale=0.3, causal=causal)
+    ref = dq.transpose(0, 2, 1, 3).reshape(-1, 16)
+    np.testing.assert_allclose(got, ref, atol=1e-12, rtol=0)
