@@ -20,13 +20,21 @@
 // shared-memory tiles are the forward's 128-row, 128-byte-swizzled boxes,
 // read K-major by the SS products and MN-major by the TS products.
 //
+// Each step covers 64 query rows (K/V-major) or 64 keys (Q-major), so tensor
+// memory holds two T1/T2 pairs beside the accumulators and the two
+// elementwise groups ping-pong: while one turns its pair into P / dS, the
+// tensor cores accumulate the other's and compute the next pair
+// (issue order T(0) T(1) | TS(0) T(2) | TS(1) T(3) | ...), as the forward
+// kernel does with its two query tiles.
+//
 // Warp roles (12 warps): warp 0 TMA producer (the whole warp also stages the
 // step's lse and delta in the K/V-major kernel), warp 1 MMA issuer and
-// tensor-memory owner, warps 4-7 and 8-11 the two elementwise groups: thread
-// t owns row t of T1/T2, group w the columns [64w, 64w + 64).  Tensor memory
-// (512 columns): T1 [0,128), T2 [128,256), accumulators [256, 256 + 2D);
-// the bf16 P / dS of group w overwrite columns [64w, 64w + 32) of T1 / T2
-// once read.  Every wait is bounded (as in the forward kernel).
+// tensor-memory owner, warps 4-7 and 8-11 the two elementwise groups (group
+// g takes the steps i with i % 2 == g of every item; thread t owns row t of
+// its T1/T2 pair).  Tensor memory (512 columns): T1 pair [0,64) [64,128),
+// T2 pair [128,192) [192,256), accumulators [256, 256 + 2D); the bf16 P / dS
+// of a step overwrite the first 32 columns of its T1 / T2 once read.  Every
+// wait is bounded (as in the forward kernel).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -38,8 +46,8 @@
 namespace ra {
 
 namespace tb {
-constexpr int BR = 128;                 // rows of every tile
-constexpr int NST = 2;                  // step stages
+constexpr int BR = 128;                 // rows of an item tile (and of T1/T2)
+constexpr int BS = 64;                  // rows of a K/V-major step (query rows)
 constexpr int THREADS = 384;
 constexpr int SLAB = 128 * 64 * 2;      // one 128-row x 64-column bf16 box
 constexpr uint32_t TMEM_COLS = 512;
@@ -47,16 +55,17 @@ constexpr int REG_LOW = 96, REG_HIGH = 184;
 constexpr int REG_NEED = (128 * REG_LOW + 256 * REG_HIGH + THREADS - 1) / THREADS;
 }  // namespace tb
 
-template <int D>
+template <int D, int SR>
 struct BwdSmem {
+  static constexpr int NST = SR == 64 ? 4 : 2;          // step stages
   alignas(1024) uint8_t x[2][tb::BR * D * 2];           // item tiles (K, V) or (Q, dO)
-  alignas(1024) uint8_t y[tb::NST][2][tb::BR * D * 2];  // step tiles (Q, dO) or (K, V)
-  float ylse[tb::NST][tb::BR];                          // K/V-major: lse * log2(e) of the step's queries
-  float ydl[tb::NST][tb::BR];                           //            and their delta
+  alignas(1024) uint8_t y[NST][2][SR * D * 2];          // step tiles (Q, dO) or (K, V)
+  float ylse[NST][SR];                                  // K/V-major: lse * log2(e) of the step's queries
+  float ydl[NST][SR];                                   //            and their delta
   alignas(8) uint64_t x_full, x_empty, teardown;
-  alignas(8) uint64_t y_full[tb::NST];
-  alignas(8) uint64_t y_empty[tb::NST];
-  alignas(8) uint64_t s_full;
+  alignas(8) uint64_t y_full[NST];
+  alignas(8) uint64_t y_empty[NST];
+  alignas(8) uint64_t s_full[2];
   alignas(8) uint64_t p_full[2];
   alignas(8) uint64_t acc_full, acc_empty;
   uint32_t tmem_base;
@@ -90,7 +99,7 @@ __device__ __forceinline__ KvItem kv_item(const Plan& p, int L) {
   return it;
 }
 
-// One step of a K/V-major item: a 128-row query tile of head h in chunk qs.
+// One step of a K/V-major item: a 64-row query tile of head h in chunk qs.
 struct QStep {
   int h, qs, q_off, nq, q0, k0;
 };
@@ -98,7 +107,7 @@ struct QStepIter {
   int h, n, qt;
 };
 __device__ __forceinline__ bool qstep_next(const Plan& p, const KvItem& it, QStepIter& s, QStep& out) {
-  const int G = p.Hq / p.Hkv, tpq = cdiv(p.C, tb::BR);
+  const int G = p.Hq / p.Hkv, tpq = cdiv(p.C, tb::BS);
   while (s.h < G) {
     if (s.n >= p.nqc) {
       s.n = 0;
@@ -112,10 +121,19 @@ __device__ __forceinline__ bool qstep_next(const Plan& p, const KvItem& it, QSte
     }
     // the block of rank srank meets ranks srank, srank+1, ... (ring mode); buffer order (step mode)
     const int qs = p.mode == kModeRing ? rank_chunk(p, (it.srank + s.n / p.cpr) % p.P, s.n % p.cpr) : s.n;
-    const int q_off = s.qt * tb::BR;
-    const int nq = imin(tb::BR, p.C - q_off);
-    const int q0 = q_pos_base(p, qs) + q_off;
+    const int qb = q_pos_base(p, qs);
     const int k0 = kv_pos_base(p, q_gid(p, qs), it.ks) + it.k_off;
+    if (s.qt == 0 && p.causal) {
+      // tiles whose last query precedes the first key are never met: start at the first one that is
+      if (qb + p.C - 1 < k0) {
+        s.qt = tpq;
+        continue;
+      }
+      s.qt = imax(0, (k0 - qb + 1 + tb::BS - 1) / tb::BS - 1);
+    }
+    const int q_off = s.qt * tb::BS;
+    const int nq = imin(tb::BS, p.C - q_off);
+    const int q0 = qb + q_off;
     ++s.qt;
     if (p.causal && k0 > q0 + nq - 1) continue;   // every key after every query of the tile
     out.h = it.g * G + s.h;
@@ -127,6 +145,24 @@ __device__ __forceinline__ bool qstep_next(const Plan& p, const KvItem& it, QSte
     return true;
   }
   return false;
+}
+
+__device__ __forceinline__ int qstep_count(const Plan& p, const KvItem& it) {
+  const int G = p.Hq / p.Hkv, tpq = cdiv(p.C, tb::BS);
+  int n = 0;
+  for (int c = 0; c < p.nqc; ++c) {
+    const int qs = p.mode == kModeRing ? rank_chunk(p, (it.srank + c / p.cpr) % p.P, c % p.cpr) : c;
+    const int qb = q_pos_base(p, qs);
+    const int k0 = kv_pos_base(p, q_gid(p, qs), it.ks) + it.k_off;
+    if (!p.causal) {
+      n += tpq;
+    } else if (qb + p.C - 1 >= k0) {
+      int t = imax(0, (k0 - qb + 1 + tb::BS - 1) / tb::BS - 1);
+      if (qb + imin((t + 1) * tb::BS, p.C) - 1 < k0) ++t;   // (defensive: the formula already lands here)
+      n += tpq - t;
+    }
+  }
+  return n * G;
 }
 
 // Q-major item: one 128-row query tile of head h (longest work first).
@@ -149,32 +185,40 @@ __device__ __forceinline__ QItem q_item(const Plan& p, int L) {
   return it;
 }
 
-// TMA load of one 128-row tile (D/64 boxes) at row x of chunk slot `slot`
-template <int D>
+// TMA load of one ROWS-row tile (D/64 boxes of ROWS x 64, slab after slab) at
+// row x of chunk slot `slot`
+template <int D, int ROWS>
 __device__ __forceinline__ void load_tile(const Plan& p, uint32_t dst, const CUtensorMap* tm, uint32_t bar, int head,
                                           int slot, int x, int b, uint64_t pol) {
 #pragma unroll
   for (int sl = 0; sl < D / 64; ++sl) {
     if (p.strided)
-      tma_load_5d(dst + sl * tb::SLAB, tm, bar, sl * 64, head, slot, x, b, pol);
+      tma_load_5d(dst + sl * ROWS * 128, tm, bar, sl * 64, head, slot, x, b, pol);
     else
-      tma_load_4d(dst + sl * tb::SLAB, tm, bar, sl * 64, head, buf_row(p, slot, x), b, pol);
+      tma_load_4d(dst + sl * ROWS * 128, tm, bar, sl * 64, head, buf_row(p, slot, x), b, pol);
   }
 }
 
 template <int D, bool kKvMajor>
 __global__ void __launch_bounds__(tb::THREADS, 1)
-    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmX1, const __grid_constant__ CUtensorMap tmX2,
+                       const __grid_constant__ CUtensorMap tmY1, const __grid_constant__ CUtensorMap tmY2,
                        const BwdTcParams prm) {
   using namespace tb;
+  // K/V-major: 64-row steps, the two groups ping-pong between two T1/T2 pairs; Q-major:
+  // 128-key steps (tensor memory holds one pair beside dQ), both groups on every step,
+  // group g on the columns [64g, 64g + 64)
+  constexpr int SR = kKvMajor ? BS : BR;
+  constexpr bool PP = kKvMajor;
+  using Smem = BwdSmem<D, SR>;
+  constexpr int NST = Smem::NST;
   extern __shared__ uint8_t smem_raw[];
-  BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Plan& p = prm.p;
   unsigned int* err = prm.err;
   volatile int* abort_flag = &sm.abort_flag;
-  constexpr uint32_t TILE = BR * D * 2;
+  constexpr uint32_t XTILE = BR * D * 2, YTILE = SR * D * 2;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sm.x_full), 1);
@@ -184,7 +228,8 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
       mbar_init(smem_u32(&sm.y_full[s]), 1);
       mbar_init(smem_u32(&sm.y_empty[s]), 1);
     }
-    mbar_init(smem_u32(&sm.s_full), 1);
+    mbar_init(smem_u32(&sm.s_full[0]), 1);
+    mbar_init(smem_u32(&sm.s_full[1]), 1);
     mbar_init(smem_u32(&sm.p_full[0]), 128);
     mbar_init(smem_u32(&sm.p_full[1]), 128);
     mbar_init(smem_u32(&sm.acc_full), 1);
@@ -208,10 +253,10 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
       // ============================================================ producer (whole warp)
       const uint64_t pol_x = l2_policy_evict_first();
       const uint64_t pol_y = l2_policy_evict_last();
-      const CUtensorMap* x1 = kKvMajor ? &tmK : &tmQ;
-      const CUtensorMap* x2 = kKvMajor ? &tmV : &tmO;
-      const CUtensorMap* y1 = kKvMajor ? &tmQ : &tmK;
-      const CUtensorMap* y2 = kKvMajor ? &tmO : &tmV;
+      const CUtensorMap* x1 = &tmX1;
+      const CUtensorMap* x2 = &tmX2;
+      const CUtensorMap* y1 = &tmY1;
+      const CUtensorMap* y2 = &tmY2;
       if (lane == 0) {
         tma_prefetch_desc(x1);
         tma_prefetch_desc(x2);
@@ -233,36 +278,42 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
           const KvItem it = kv_item(p, L);
           if (lane == 0) {
             const uint32_t xb = smem_u32(&sm.x_full);
-            mbar_arrive_expect_tx(xb, 2 * TILE);
-            load_tile<D>(p, smem_u32(sm.x[0]), x1, xb, it.g, it.ks, it.k_off, it.b, pol_x);
-            load_tile<D>(p, smem_u32(sm.x[1]), x2, xb, it.g, it.ks, it.k_off, it.b, pol_x);
+            mbar_arrive_expect_tx(xb, 2 * XTILE);
+            load_tile<D, BR>(p, smem_u32(sm.x[0]), x1, xb, it.g, it.ks, it.k_off, it.b, pol_x);
+            load_tile<D, BR>(p, smem_u32(sm.x[1]), x2, xb, it.g, it.ks, it.k_off, it.b, pol_x);
           }
           __syncwarp();
           QStepIter si{0, 0, 0};
           QStep st;
           while (qstep_next(p, it, si, st)) {
-            if (!stage_wait(ycnt)) { ok = false; break; }
-            const int s = ycnt % NST;
-            // the step's lse (log2 units) and delta; columns past the tile get +inf / 0, i.e. P = 0
+            // the step's lse (log2 units) and delta, loaded before waiting for a free stage so
+            // that their latency hides behind the wait; columns past the tile get +inf / 0 (P = 0)
             const size_t base = ((size_t)it.b * p.Hq + st.h) * p.Sq;
+            float l2[BS / 32], dl[BS / 32];
 #pragma unroll
-            for (int i = 0; i < BR / 32; ++i) {
+            for (int i = 0; i < BS / 32; ++i) {
               const int c = lane + 32 * i;
-              float l2 = CUDART_INF_F, dl = 0.f;
+              l2[i] = CUDART_INF_F;
+              dl[i] = 0.f;
               if (c < st.nq) {
                 const size_t li = base + buf_row(p, st.qs, st.q_off + c);
-                l2 = prm.a.lse[li] * 1.4426950408889634f;
-                dl = prm.a.delta[li];
+                l2[i] = __ldg(prm.a.lse + li);
+                dl[i] = __ldg(prm.a.delta + li);
               }
-              sm.ylse[s][c] = l2;
-              sm.ydl[s][c] = dl;
+            }
+            if (!stage_wait(ycnt)) { ok = false; break; }
+            const int s = ycnt % NST;
+#pragma unroll
+            for (int i = 0; i < BS / 32; ++i) {
+              sm.ylse[s][lane + 32 * i] = l2[i] * 1.4426950408889634f;
+              sm.ydl[s][lane + 32 * i] = dl[i];
             }
             __syncwarp();
             if (lane == 0) {
               const uint32_t fb = smem_u32(&sm.y_full[s]);
-              mbar_arrive_expect_tx(fb, 2 * TILE);   // the arrive also publishes ylse / ydl
-              load_tile<D>(p, smem_u32(sm.y[s][0]), y1, fb, st.h, st.qs, st.q_off, it.b, pol_y);
-              load_tile<D>(p, smem_u32(sm.y[s][1]), y2, fb, st.h, st.qs, st.q_off, it.b, pol_y);
+              mbar_arrive_expect_tx(fb, 2 * YTILE);   // the arrive also publishes ylse / ydl
+              load_tile<D, BS>(p, smem_u32(sm.y[s][0]), y1, fb, st.h, st.qs, st.q_off, it.b, pol_y);
+              load_tile<D, BS>(p, smem_u32(sm.y[s][1]), y2, fb, st.h, st.qs, st.q_off, it.b, pol_y);
             }
             __syncwarp();
             ++ycnt;
@@ -271,22 +322,22 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
           const QItem it = q_item(p, L);
           if (lane == 0) {
             const uint32_t xb = smem_u32(&sm.x_full);
-            mbar_arrive_expect_tx(xb, 2 * TILE);
-            load_tile<D>(p, smem_u32(sm.x[0]), x1, xb, it.h, it.qs, it.q_off, it.b, pol_x);
-            load_tile<D>(p, smem_u32(sm.x[1]), x2, xb, it.h, it.qs, it.q_off, it.b, pol_x);
+            mbar_arrive_expect_tx(xb, 2 * XTILE);
+            load_tile<D, BR>(p, smem_u32(sm.x[0]), x1, xb, it.h, it.qs, it.q_off, it.b, pol_x);
+            load_tile<D, BR>(p, smem_u32(sm.x[1]), x2, xb, it.h, it.qs, it.q_off, it.b, pol_x);
           }
           __syncwarp();
           KvIter ki;
           kv_begin(p, it.qs, ki);
           KvTile t;
-          while (kv_next(p, it.q0 + it.nq - 1, BR, cdiv(p.C, BR), ki, t)) {
+          while (kv_next(p, it.q0 + it.nq - 1, SR, cdiv(p.C, SR), ki, t)) {
             if (!stage_wait(ycnt)) { ok = false; break; }
             const int s = ycnt % NST;
             if (lane == 0) {
               const uint32_t fb = smem_u32(&sm.y_full[s]);
-              mbar_arrive_expect_tx(fb, 2 * TILE);
-              load_tile<D>(p, smem_u32(sm.y[s][0]), y1, fb, it.g, t.slot, t.k0, it.b, pol_y);
-              load_tile<D>(p, smem_u32(sm.y[s][1]), y2, fb, it.g, t.slot, t.k0, it.b, pol_y);
+              mbar_arrive_expect_tx(fb, 2 * YTILE);
+              load_tile<D, SR>(p, smem_u32(sm.y[s][0]), y1, fb, it.g, t.slot, t.k0, it.b, pol_y);
+              load_tile<D, SR>(p, smem_u32(sm.y[s][1]), y2, fb, it.g, t.slot, t.k0, it.b, pol_y);
             }
             __syncwarp();
             ++ycnt;
@@ -302,88 +353,110 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
     } else if (warp == 1) {
       // ============================================================ MMA issuer
       if (lane == 0) {
-        const uint32_t idesc_ss = idesc_bf16_f32(BR, BR, false);
-        const uint32_t idesc_ts = idesc_bf16_f32(BR, D, true);
+        const uint32_t idesc_ss = idesc_bf16_f32(BR, SR, false);   // T = X (128 rows) x Y^T (SR rows)
+        const uint32_t idesc_ts = idesc_bf16_f32(BR, D, true);     // acc += T (bf16) x Y (MN-major)
         const uint32_t hi = (uint32_t)(sw128_desc(0, 16, 1024) >> 32);
-        const uint32_t T1 = tmem, T2 = tmem + 128, A0 = tmem + 256, A1 = tmem + 256 + D;
-        const uint32_t lx[2] = {(uint32_t)sw128_desc(smem_u32(sm.x[0]), 16, 1024),
-                                (uint32_t)sw128_desc(smem_u32(sm.x[1]), 16, 1024)};
-        uint32_t ly_k[NST][2], ly_mn[NST][2];   // step tiles read K-major (SS) and MN-major (TS)
-#pragma unroll
-        for (int s = 0; s < NST; ++s)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            ly_k[s][j] = (uint32_t)sw128_desc(smem_u32(sm.y[s][j]), 16, 1024);
-            ly_mn[s][j] = (uint32_t)sw128_desc(smem_u32(sm.y[s][j]), SLAB, 1024);
-          }
-        uint32_t ycnt = 0, steps = 0, n_items = 0;
+        const uint32_t T1[2] = {tmem, tmem + 64}, T2[2] = {tmem + 128, tmem + 192};
+        const uint32_t A0 = tmem + 256, A1 = tmem + 256 + D;
+        constexpr uint32_t YSLAB = SR * 128;                         // one SR-row x 64-column box
+        constexpr uint32_t YSTAGE16 = (2 * YTILE) >> 4, YTILE16 = YTILE >> 4;
+        const uint32_t lx0 = (uint32_t)sw128_desc(smem_u32(sm.x[0]), 16, 1024);
+        const uint32_t lx1 = (uint32_t)sw128_desc(smem_u32(sm.x[1]), 16, 1024);
+        const uint32_t ly_k = (uint32_t)sw128_desc(smem_u32(sm.y[0][0]), 16, 1024);     // K-major (SS)
+        const uint32_t ly_mn = (uint32_t)sw128_desc(smem_u32(sm.y[0][0]), YSLAB, 1024); // MN-major (TS)
+        uint32_t ycnt = 0, n_items = 0, pb[2] = {0u, 0u};
         bool ok = true;
-        auto issue_ss = [&](uint32_t d, uint32_t a, uint32_t b) {
-          mma_ss_lo_first(d, a, b, hi, idesc_ss);
-#pragma unroll
-          for (int k = 1; k < D / 16; ++k) {
-            const uint32_t off = ((k / 4) * SLAB + (k % 4) * 32) >> 4;
-            mma_ss_lo(d, a + off, b + off, hi, idesc_ss);
-          }
+        auto wait_y = [&](uint32_t c) -> bool {
+          if (!mbar_wait(smem_u32(&sm.y_full[c % NST]), (c / NST) & 1u, abort_flag, kWaitKvFull, err)) return false;
+          tc_fence_after();
+          return true;
         };
-        // acc += T[:, half w] (bf16, tmem) x Y[rows of half w] (MN-major); `first` clears acc
-        auto issue_ts_half = [&](uint32_t acc, uint32_t tsrc, uint32_t b, int w, bool first) {
+        // T1[b] = X1 Y1^T, T2[b] = X2 Y2^T for the step in stage c
+        auto issue_T = [&](int b, uint32_t c) {
+          const uint32_t y1 = ly_k + (c % NST) * YSTAGE16, y2 = y1 + YTILE16;
+          mma_ss_lo_first(T1[b], lx0, y1, hi, idesc_ss);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int k = 4 * w + kk;
-            const uint32_t a = tsrc + 64 * w + kk * 8;
-            const uint32_t bk = b + k * ((16 * 128) >> 4);
-            if (first && kk == 0)
-              mma_ts_lo_pred(acc, a, bk, hi, idesc_ts, 0u);
+          for (int k = 1; k < D / 16; ++k)
+            mma_ss_lo(T1[b], lx0 + (((k / 4) * SLAB + (k % 4) * 32) >> 4), y1 + (((k / 4) * YSLAB + (k % 4) * 32) >> 4),
+                      hi, idesc_ss);
+          mma_ss_lo_first(T2[b], lx1, y2, hi, idesc_ss);
+#pragma unroll
+          for (int k = 1; k < D / 16; ++k)
+            mma_ss_lo(T2[b], lx1 + (((k / 4) * SLAB + (k % 4) * 32) >> 4), y2 + (((k / 4) * YSLAB + (k % 4) * 32) >> 4),
+                      hi, idesc_ss);
+          mma_commit(smem_u32(&sm.s_full[b]));
+        };
+        // acc += T (bf16 pairs) x Y (MN-major) over the 64 rows k0 .. k0 + 63 of the step tile: the
+        // pairs of those rows start at column tsrc; `first` clears acc
+        auto issue_ts = [&](uint32_t acc, uint32_t tsrc, uint32_t ymn, int k0, bool first) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t bk = ymn + (k0 / 16 + k) * ((16 * 128) >> 4);
+            if (first && k == 0)
+              mma_ts_lo_pred(acc, tsrc, bk, hi, idesc_ts, 0u);
             else
-              mma_ts_lo(acc, a, bk, hi, idesc_ts);
+              mma_ts_lo(acc, tsrc + k * 8, bk, hi, idesc_ts);
           }
         };
         for (int L = blockIdx.x; L < prm.items && ok; L += gridDim.x, ++n_items) {
           if (!mbar_wait(smem_u32(&sm.x_full), n_items & 1u, abort_flag, kWaitQFull, err)) { ok = false; break; }
           tc_fence_after();
-          bool first = true;
-          auto run_step = [&]() -> bool {
-            const int s = ycnt % NST;
-            if (!mbar_wait(smem_u32(&sm.y_full[s]), (ycnt / NST) & 1u, abort_flag, kWaitKvFull, err)) return false;
-            tc_fence_after();
-            issue_ss(T1, lx[0], ly_k[s][0]);
-            issue_ss(T2, lx[1], ly_k[s][1]);
-            mma_commit(smem_u32(&sm.s_full));
-            if (first && n_items > 0) {
-              // the accumulators are read by the previous item's epilogue until acc_empty
-              if (!mbar_wait(smem_u32(&sm.acc_empty), (n_items - 1) & 1u, abort_flag, kWaitOFinal, err))
-                return false;
-              tc_fence_after();
-            }
-            for (int w = 0; w < 2; ++w) {
-              if (!mbar_wait(smem_u32(&sm.p_full[w]), steps & 1u, abort_flag, kWaitPFull, err)) return false;
-              tc_fence_after();
-              issue_ts_half(A0, T2, ly_mn[s][0], w, first && w == 0);        // dK or dQ += dS x Y1
-              if constexpr (kKvMajor) issue_ts_half(A1, T1, ly_mn[s][1], w, first && w == 0);   // dV += P x Y2
-            }
-            mma_commit(smem_u32(&sm.y_empty[s]));
-            first = false;
-            ++ycnt;
-            ++steps;
-            return true;
-          };
+          int n;
           if constexpr (kKvMajor) {
-            const KvItem it = kv_item(p, L);
-            QStepIter si{0, 0, 0};
-            QStep st;
-            while (qstep_next(p, it, si, st))
-              if (!(ok = run_step())) break;
+            n = qstep_count(p, kv_item(p, L));
           } else {
             const QItem it = q_item(p, L);
-            KvIter ki;
-            kv_begin(p, it.qs, ki);
-            KvTile t;
-            while (kv_next(p, it.q0 + it.nq - 1, BR, cdiv(p.C, BR), ki, t))
-              if (!(ok = run_step())) break;
+            n = kv_count(p, it.qs, it.q0 + it.nq - 1, SR, cdiv(p.C, SR));
+          }
+          if constexpr (!PP) {
+            // one pair: T | TS over the columns of group 0 | TS over those of group 1
+            for (int i = 0; i < n && ok; ++i) {
+              const uint32_t c = ycnt + i;
+              if (!(ok = wait_y(c))) break;
+              issue_T(0, c);
+              if (i == 0 && n_items > 0) {
+                if (!(ok = mbar_wait(smem_u32(&sm.acc_empty), (n_items - 1) & 1u, abort_flag, kWaitOFinal, err)))
+                  break;
+                tc_fence_after();
+              }
+              const uint32_t ymn = ly_mn + (c % NST) * YSTAGE16;
+              for (int w = 0; w < 2 && ok; ++w) {
+                if (!(ok = mbar_wait(smem_u32(&sm.p_full[w]), pb[0] & 1u, abort_flag, kWaitPFull, err))) break;
+                tc_fence_after();
+                issue_ts(A0, T2[0] + 64 * w, ymn, 64 * w, i == 0 && w == 0);
+              }
+              ++pb[0];
+              mma_commit(smem_u32(&sm.y_empty[c % NST]));
+            }
+          }
+          // T(0), T(1) | TS(0) T(2) | TS(1) T(3) | ...
+          for (int i = 0; PP && i < 2 && i < n && ok; ++i) {
+            if (!(ok = wait_y(ycnt + i))) break;
+            issue_T(i, ycnt + i);
+          }
+          if (PP && n > 0 && ok && n_items > 0) {
+            // the accumulators are read by the previous item's epilogue until acc_empty
+            ok = mbar_wait(smem_u32(&sm.acc_empty), (n_items - 1) & 1u, abort_flag, kWaitOFinal, err);
+            tc_fence_after();
+          }
+          for (int i = 0; PP && i < n && ok; ++i) {
+            const int b = i & 1;
+            const uint32_t c = ycnt + i;
+            if (!(ok = mbar_wait(smem_u32(&sm.p_full[b]), pb[b] & 1u, abort_flag, kWaitPFull, err))) break;
+            ++pb[b];
+            tc_fence_after();
+            const uint32_t ymn = ly_mn + (c % NST) * YSTAGE16;
+            issue_ts(A0, T2[b], ymn, 0, i == 0);                                  // dK += dS^T x Q
+            issue_ts(A1, T1[b], ymn + YTILE16, 0, i == 0);                          // dV += P^T x dO
+            mma_commit(smem_u32(&sm.y_empty[c % NST]));
+            if (i + 2 < n) {
+              if (!(ok = wait_y(c + 2))) break;
+              issue_T(b, c + 2);
+            }
           }
           if (!ok) break;
-          if (first && n_items > 0) {
+          ycnt += n;
+          if (n == 0 && n_items > 0) {
             // an item without steps still hands the accumulators over in order
             if (!mbar_wait(smem_u32(&sm.acc_empty), (n_items - 1) & 1u, abort_flag, kWaitOFinal, err)) {
               ok = false;
@@ -401,50 +474,58 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
   } else {
     setmaxnreg_inc<REG_HIGH>();
     // ============================================================ elementwise groups
-    const int w = (warp - 4) >> 2;            // column half of this group
+    const int g = (warp - 4) >> 2;            // group: steps i with i % 2 == g of every item
     const int wi = warp & 3;                  // tensor-memory lane quarter
     const int row = wi * 32 + lane;           // row of T1/T2 owned by this thread
     const uint32_t lane_off = (uint32_t)(wi * 32) << 16;
-    const uint32_t T1 = tmem + lane_off, T2 = tmem + lane_off + 128;
+    // ping-pong: this group's own pair, all its 64 columns; otherwise the one pair, columns [64g, 64g + 64)
+    const uint32_t T1 = tmem + lane_off + (PP ? 64 * g : 0), T2 = tmem + lane_off + 128 + (PP ? 64 * g : 0);
+    constexpr int CB = 0;
+    const int cb = PP ? CB : 64 * g;            // first column of this group in its pair
     const uint32_t A0 = tmem + lane_off + 256, A1 = tmem + lane_off + 256 + D;
     const float sl2 = prm.sl2;
-    uint32_t ycnt = 0, steps = 0, n_items = 0;
+    uint32_t ycnt = 0, ns = 0, n_items = 0;
     bool ok = true;
 
-    // Q-major step: dS of this thread's query row over the group's 64 key columns.  Column j
-    // is masked when j > lim (causal) or j >= ncols (past the tile); rows past the tile carry
-    // lse = +inf, i.e. P = 0.
-    auto elementwise_q = [&](float l2_row, float dl_row, int lim, int ncols, bool need_mask) -> bool {
-      const bool got = mbar_wait(smem_u32(&sm.s_full), steps & 1u, abort_flag, kWaitSFull, err);
+    // One step of this group: read the pair, write bf16 P (K/V-major only) and dS over its
+    // first 32 columns, hand it to the MMA issuer.  `mask(j)` tells whether column j is cut.
+    auto step = [&](auto lse2_of, auto delta_of, auto masked) -> bool {
+      const bool got = mbar_wait(smem_u32(&sm.s_full[PP ? g : 0]), ns & 1u, abort_flag, kWaitSFull, err);
       if (!__all_sync(0xffffffffu, got)) return false;
+      ++ns;
+      if constexpr (kKvMajor) {
+        // the producer's ylse / ydl stores are published by this stage's full barrier
+        const bool f = mbar_wait(smem_u32(&sm.y_full[ycnt % NST]), (ycnt / NST) & 1u, abort_flag, kWaitKvFull, err);
+        if (!__all_sync(0xffffffffu, f)) return false;
+      }
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const int col = 64 * w + 32 * c;
         uint32_t r1[32], r2[32];
-        tmem_ld32(T1 + col, r1);
-        tmem_ld32(T2 + col, r2);
+        tmem_ld32(T1 + cb + 32 * c, r1);
+        tmem_ld32(T2 + cb + 32 * c, r2);
         tmem_wait_ld();
-        uint32_t dk[16];
+        uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float ds[2];
+          float pe[2], ds[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int j = col + 2 * e + u;
-            float x = ex2(fmaf(__uint_as_float(r1[2 * e + u]), sl2, -l2_row));
-            if (need_mask && (j > lim || j >= ncols)) x = 0.f;
-            ds[u] = x * (__uint_as_float(r2[2 * e + u]) - dl_row);
+            const int j = cb + 32 * c + 2 * e + u;   // column of the step tile
+            float x = ex2(fmaf(__uint_as_float(r1[2 * e + u]), sl2, -lse2_of(j)));
+            if (masked(j)) x = 0.f;
+            pe[u] = x;
+            ds[u] = x * (__uint_as_float(r2[2 * e + u]) - delta_of(j));
           }
+          pk[e] = pack_bf16x2(pe[0], pe[1]);
           dk[e] = pack_bf16x2(ds[0], ds[1]);
         }
-        tmem_st16(T2 + 64 * w + 16 * c, dk);
+        if constexpr (kKvMajor) tmem_st16(T1 + cb + 16 * c, pk);
+        tmem_st16(T2 + cb + 16 * c, dk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.p_full[w]));
-      ++ycnt;
-      ++steps;
+      mbar_arrive(smem_u32(&sm.p_full[g]));
       return true;
     };
 
@@ -454,54 +535,23 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
         const KvItem it = kv_item(p, L);
         QStepIter si{0, 0, 0};
         QStep st;
+        const bool row_live = row < it.nk;
         while (qstep_next(p, it, si, st)) {
-          // key row `row` (position k0 + row) sees query column j iff k0 + row <= q0 + j, so
-          // columns j < lim_causal are masked; rows past the tile see nothing; columns past
-          // the tile carry lse = +inf (P = 0)
-          const int lim_causal = p.causal ? (st.k0 + row) - st.q0 : -BR;
-          const bool full = !p.causal || st.k0 + BR - 1 <= st.q0;
-          const bool need = !full || it.nk < BR;
-          const int s = ycnt % NST;
-          const bool got = mbar_wait(smem_u32(&sm.s_full), steps & 1u, abort_flag, kWaitSFull, err);
-          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-          const bool f = mbar_wait(smem_u32(&sm.y_full[s]), (ycnt / NST) & 1u, abort_flag, kWaitKvFull, err);
-          if (!__all_sync(0xffffffffu, f)) { ok = false; break; }
-          tc_fence_after();
-          const bool row_live = row < it.nk;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int col = 64 * w + 32 * c;
-            uint32_t r1[32], r2[32];
-            tmem_ld32(T1 + col, r1);
-            tmem_ld32(T2 + col, r2);
-            tmem_wait_ld();
-            uint32_t pk[16], dk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float pe[2], ds[2];
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int j = col + 2 * e + u;
-                float x = ex2(fmaf(__uint_as_float(r1[2 * e + u]), sl2, -sm.ylse[s][j]));
-                if (need && (!row_live || j < lim_causal)) x = 0.f;   // columns >= nq carry lse = +inf
-                pe[u] = x;
-                ds[u] = x * (__uint_as_float(r2[2 * e + u]) - sm.ydl[s][j]);
-              }
-              pk[e] = pack_bf16x2(pe[0], pe[1]);
-              dk[e] = pack_bf16x2(ds[0], ds[1]);
-            }
-            tmem_st16(T1 + 64 * w + 16 * c, pk);
-            tmem_st16(T2 + 64 * w + 16 * c, dk);
+          if ((nsteps & 1) == g) {
+            // key row (position k0 + row) sees query column j iff k0 + row <= q0 + j; columns
+            // past the tile carry lse = +inf (P = 0); rows past the tile see nothing
+            const int lim = p.causal ? (st.k0 + row) - st.q0 : -BS;
+            const bool need = (p.causal && st.k0 + BR - 1 > st.q0) || !row_live;
+            const int sidx = ycnt % NST;
+            if (!(ok = step([&](int j) { return sm.ylse[sidx][j]; }, [&](int j) { return sm.ydl[sidx][j]; },
+                            [&](int j) { return need && (!row_live || j < lim); })))
+              break;
           }
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(smem_u32(&sm.p_full[w]));
           ++ycnt;
-          ++steps;
           ++nsteps;
         }
         if (!ok) break;
-        // ---- epilogue: dK (scaled) and dV rows of this item; group w writes columns [D/2 w, D/2 (w+1))
+        // ---- epilogue: dK (scaled) and dV rows of this item; group g writes columns [D/2 g, D/2 (g+1))
         const bool fin = mbar_wait(smem_u32(&sm.acc_full), n_items & 1u, abort_flag, kWaitOFinal, err);
         if (!__all_sync(0xffffffffu, fin)) { ok = false; break; }
         tc_fence_after();
@@ -509,7 +559,7 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
         const size_t orow = ((size_t)it.b * p.Skv + buf_row(p, it.ks, it.k_off + (live ? row : 0))) * p.Hkv + it.g;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          const int col = (D / 2) * w + 32 * c;
+          const int col = (D / 2) * g + 32 * c;
           uint32_t rk[32], rv[32];
           tmem_ld32(A0 + col, rk);
           tmem_ld32(A1 + col, rv);
@@ -557,11 +607,17 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
         KvIter ki;
         kv_begin(p, it.qs, ki);
         KvTile t;
-        while (kv_next(p, it.q0 + it.nq - 1, BR, cdiv(p.C, BR), ki, t)) {
-          // query row (position q0 + row) sees key column j iff pos0 + j <= q0 + row
-          const int lim = p.causal ? qpos - t.pos0 : BR;
-          const bool need = (p.causal && t.pos0 + BR - 1 > it.q0) || t.nvalid < BR;
-          if (!(ok = elementwise_q(l2_row, dl_row, lim, t.nvalid, need))) break;
+        while (kv_next(p, it.q0 + it.nq - 1, SR, cdiv(p.C, SR), ki, t)) {
+          {
+            // query row (position q0 + row) sees key column j iff pos0 + j <= q0 + row
+            const int lim = p.causal ? qpos - t.pos0 : SR;
+            const int nv = t.nvalid;
+            const bool need = (p.causal && t.pos0 + SR - 1 > it.q0) || nv < SR;
+            if (!(ok = step([&](int) { return l2_row; }, [&](int) { return dl_row; },
+                            [&](int j) { return need && (j > lim || j >= nv); })))
+              break;
+          }
+          ++ycnt;
           ++nsteps;
         }
         if (!ok) break;
@@ -571,7 +627,7 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
         const size_t orow = ((size_t)it.b * p.Sq + buf_row(p, it.qs, it.q_off + (live ? row : 0))) * p.Hq + it.h;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          const int col = (D / 2) * w + 32 * c;
+          const int col = (D / 2) * g + 32 * c;
           uint32_t rq[32];
           tmem_ld32(A0 + col, rq);
           tmem_wait_ld();
@@ -612,20 +668,20 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
 
 template <int D, bool kKvMajor>
 static cudaError_t launch_bwd_tc_d(const Plan& p, const BwdArgs& a, unsigned int* err, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, to;
-  const void* qp = a.q;
-  if (p.strided) {
-    if (!make_tmap_striped(&tq, qp, p.B, p.Sq, p.P, p.Hq, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_striped(&to, a.dout, p.B, p.Sq, p.P, p.Hq, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_striped(&tk, a.k, p.B, p.Skv, p.P, p.Hkv, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_striped(&tv, a.v, p.B, p.Skv, p.P, p.Hkv, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  } else if (!make_tmap_bhsd(&tq, qp, p.B, p.Sq, p.Hq, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B) ||
-             !make_tmap_bhsd(&to, a.dout, p.B, p.Sq, p.Hq, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B) ||
-             !make_tmap_bhsd(&tk, a.k, p.B, p.Skv, p.Hkv, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B) ||
-             !make_tmap_bhsd(&tv, a.v, p.B, p.Skv, p.Hkv, D, 64, tb::BR, CU_TENSOR_MAP_SWIZZLE_128B)) {
-    return cudaErrorInvalidValue;
-  }
+  // item tiles: 128-row boxes; step tiles: 64-row boxes
+  auto map = [&](CUtensorMap* m, const void* base, int rows, int heads, int box_rows) {
+    return p.strided ? make_tmap_striped(m, base, p.B, rows, p.P, heads, D, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B)
+                     : make_tmap_bhsd(m, base, p.B, rows, heads, D, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+  };
+  CUtensorMap x1, x2, y1, y2;
+  bool ok;
+  if (kKvMajor)
+    ok = map(&x1, a.k, p.Skv, p.Hkv, tb::BR) && map(&x2, a.v, p.Skv, p.Hkv, tb::BR) &&
+         map(&y1, a.q, p.Sq, p.Hq, tb::BS) && map(&y2, a.dout, p.Sq, p.Hq, tb::BS);
+  else
+    ok = map(&x1, a.q, p.Sq, p.Hq, tb::BR) && map(&x2, a.dout, p.Sq, p.Hq, tb::BR) &&
+         map(&y1, a.k, p.Skv, p.Hkv, tb::BR) && map(&y2, a.v, p.Skv, p.Hkv, tb::BR);
+  if (!ok) return cudaErrorInvalidValue;
   BwdTcParams prm;
   prm.p = p;
   prm.a = a;
@@ -636,7 +692,7 @@ static cudaError_t launch_bwd_tc_d(const Plan& p, const BwdArgs& a, unsigned int
   if (items <= 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
   prm.items = (int)items;
-  const size_t smem = sizeof(BwdSmem<D>) + 1024;
+  const size_t smem = sizeof(BwdSmem<D, kKvMajor ? tb::BS : tb::BR>) + 1024;
   auto kern = attn_bwd_tc_kernel<D, kKvMajor>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -645,7 +701,7 @@ static cudaError_t launch_bwd_tc_d(const Plan& p, const BwdArgs& a, unsigned int
   if (e != cudaSuccess) return e;
   if (fa.numRegs < tb::REG_NEED) return cudaErrorNotSupported;
   const int grid = prm.items < num_sms() ? prm.items : num_sms();
-  kern<<<grid, tb::THREADS, smem, st>>>(tq, tk, tv, to, prm);
+  kern<<<grid, tb::THREADS, smem, st>>>(x1, x2, y1, y2, prm);
   return cudaGetLastError();
 }
 
