@@ -60,8 +60,8 @@ struct BwdSmem {
   static constexpr int NST = SR == 64 ? 4 : 2;          // step stages
   alignas(1024) uint8_t x[2][tb::BR * D * 2];           // item tiles (K, V) or (Q, dO)
   alignas(1024) uint8_t y[NST][2][SR * D * 2];          // step tiles (Q, dO) or (K, V)
-  float ylse[NST][SR];                                  // K/V-major: lse * log2(e) of the step's queries
-  float ydl[NST][SR];                                   //            and their delta
+  alignas(16) float ylse[NST][SR];                      // K/V-major: -lse * log2(e) of the step's queries
+  alignas(16) float ydl[NST][SR];                       //            and -delta
   alignas(8) uint64_t x_full, x_empty, teardown;
   alignas(8) uint64_t y_full[NST];
   alignas(8) uint64_t y_empty[NST];
@@ -304,9 +304,9 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
             if (!stage_wait(ycnt)) { ok = false; break; }
             const int s = ycnt % NST;
 #pragma unroll
-            for (int i = 0; i < BS / 32; ++i) {
-              sm.ylse[s][lane + 32 * i] = l2[i] * 1.4426950408889634f;
-              sm.ydl[s][lane + 32 * i] = dl[i];
+            for (int i = 0; i < BS / 32; ++i) {   // stored negated: the elementwise pass adds them
+              sm.ylse[s][lane + 32 * i] = -(l2[i] * 1.4426950408889634f);
+              sm.ydl[s][lane + 32 * i] = -dl[i];
             }
             __syncwarp();
             if (lane == 0) {
@@ -488,8 +488,10 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
     bool ok = true;
 
     // One step of this group: read the pair, write bf16 P (K/V-major only) and dS over its
-    // first 32 columns, hand it to the MMA issuer.  `mask(j)` tells whether column j is cut.
-    auto step = [&](auto lse2_of, auto delta_of, auto masked) -> bool {
+    // first 32 columns, hand it to the MMA issuer.  nl_of(j) / nd_of(j) give -lse*log2(e) and
+    // -delta of columns j, j+1 as a packed pair; masked(j) tells whether column j is cut.
+    const uint64_t sl2x2 = pack2(sl2, sl2);
+    auto step = [&](auto nl_of, auto nd_of, auto masked, bool need) -> bool {
       const bool got = mbar_wait(smem_u32(&sm.s_full[PP ? g : 0]), ns & 1u, abort_flag, kWaitSFull, err);
       if (!__all_sync(0xffffffffu, got)) return false;
       ++ns;
@@ -508,17 +510,20 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float pe[2], ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int j = cb + 32 * c + 2 * e + u;   // column of the step tile
-            float x = ex2(fmaf(__uint_as_float(r1[2 * e + u]), sl2, -lse2_of(j)));
-            if (masked(j)) x = 0.f;
-            pe[u] = x;
-            ds[u] = x * (__uint_as_float(r2[2 * e + u]) - delta_of(j));
+          const int j = cb + 32 * c + 2 * e;   // column of the step tile (pair j, j+1)
+          float x0, x1;
+          unpack2(ffma2(pack2(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1])), sl2x2, nl_of(j)), x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          if (need) {
+            if (masked(j)) p0 = 0.f;
+            if (masked(j + 1)) p1 = 0.f;
           }
-          pk[e] = pack_bf16x2(pe[0], pe[1]);
-          dk[e] = pack_bf16x2(ds[0], ds[1]);
+          const uint64_t pp = pack2(p0, p1);
+          float d0, d1;
+          unpack2(fmul2(pp, fadd2(pack2(__uint_as_float(r2[2 * e]), __uint_as_float(r2[2 * e + 1])), nd_of(j))), d0,
+                  d1);
+          pk[e] = pack_bf16x2(p0, p1);
+          dk[e] = pack_bf16x2(d0, d1);
         }
         if constexpr (kKvMajor) tmem_st16(T1 + cb + 16 * c, pk);
         tmem_st16(T2 + cb + 16 * c, dk);
@@ -543,8 +548,11 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
             const int lim = p.causal ? (st.k0 + row) - st.q0 : -BS;
             const bool need = (p.causal && st.k0 + BR - 1 > st.q0) || !row_live;
             const int sidx = ycnt % NST;
-            if (!(ok = step([&](int j) { return sm.ylse[sidx][j]; }, [&](int j) { return sm.ydl[sidx][j]; },
-                            [&](int j) { return need && (!row_live || j < lim); })))
+            const float2* nl = reinterpret_cast<const float2*>(sm.ylse[sidx]);
+            const float2* nd = reinterpret_cast<const float2*>(sm.ydl[sidx]);
+            if (!(ok = step([&](int j) { const float2 v = nl[j >> 1]; return pack2(v.x, v.y); },
+                            [&](int j) { const float2 v = nd[j >> 1]; return pack2(v.x, v.y); },
+                            [&](int j) { return !row_live || j < lim; }, need)))
               break;
           }
           ++ycnt;
@@ -613,8 +621,9 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
             const int lim = p.causal ? qpos - t.pos0 : SR;
             const int nv = t.nvalid;
             const bool need = (p.causal && t.pos0 + SR - 1 > it.q0) || nv < SR;
-            if (!(ok = step([&](int) { return l2_row; }, [&](int) { return dl_row; },
-                            [&](int j) { return need && (j > lim || j >= nv); })))
+            const uint64_t nl2 = pack2(-l2_row, -l2_row), nd2 = pack2(-dl_row, -dl_row);
+            if (!(ok = step([&](int) { return nl2; }, [&](int) { return nd2; },
+                            [&](int j) { return j > lim || j >= nv; }, need)))
               break;
           }
           ++ycnt;
