@@ -371,6 +371,16 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
           tc_fence_after();
           return true;
         };
+        // dst = X Y^T for tile j (0: X1 Y1^T, 1: X2 Y2^T) of the step in stage c (no commit)
+        auto issue_prod = [&](uint32_t dst, int j, uint32_t c) {
+          const uint32_t xa = j ? lx1 : lx0;
+          const uint32_t yb = ly_k + (c % NST) * YSTAGE16 + (j ? YTILE16 : 0u);
+          mma_ss_lo_first(dst, xa, yb, hi, idesc_ss);
+#pragma unroll
+          for (int k = 1; k < D / 16; ++k)
+            mma_ss_lo(dst, xa + (((k / 4) * SLAB + (k % 4) * 32) >> 4), yb + (((k / 4) * YSLAB + (k % 4) * 32) >> 4),
+                      hi, idesc_ss);
+        };
         // T1[b] = X1 Y1^T, T2[b] = X2 Y2^T for the step in stage c
         auto issue_T = [&](int b, uint32_t c) {
           const uint32_t y1 = ly_k + (c % NST) * YSTAGE16, y2 = y1 + YTILE16;
@@ -409,24 +419,43 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
             n = kv_count(p, it.qs, it.q0 + it.nq - 1, SR, cdiv(p.C, SR));
           }
           if constexpr (!PP) {
-            // one pair: T | TS over the columns of group 0 | TS over those of group 1
+            // Three 128-column regions rotate between S and dP: step i puts S in region
+            // (2i) % 3 and dP in (2i + 1) % 3.  S(i) is free once the groups have read it, so
+            // dP(i+1) reuses it and S(i+2) takes the third region: while the groups work on
+            // step i the tensor cores compute S(i+1); after them, dQ += dS(i) K(i), dP(i+1), S(i+2).
+            auto region = [&](int r) -> uint32_t { return tmem + (r == 2 ? 384u : 128u * r); };
+            if (n > 0 && ok) {
+              if ((ok = wait_y(ycnt))) {
+                issue_prod(region(0), 0, ycnt);
+                issue_prod(region(1), 1, ycnt);
+                mma_commit(smem_u32(&sm.s_full[0]));
+                if (n > 1 && (ok = wait_y(ycnt + 1))) issue_prod(region(2), 0, ycnt + 1);
+              }
+            }
+            if (ok && n > 0 && n_items > 0) {
+              ok = mbar_wait(smem_u32(&sm.acc_empty), (n_items - 1) & 1u, abort_flag, kWaitOFinal, err);
+              tc_fence_after();
+            }
             for (int i = 0; i < n && ok; ++i) {
               const uint32_t c = ycnt + i;
-              if (!(ok = wait_y(c))) break;
-              issue_T(0, c);
-              if (i == 0 && n_items > 0) {
-                if (!(ok = mbar_wait(smem_u32(&sm.acc_empty), (n_items - 1) & 1u, abort_flag, kWaitOFinal, err)))
-                  break;
-                tc_fence_after();
-              }
+              const uint32_t rd = region((2 * i + 1) % 3);
               const uint32_t ymn = ly_mn + (c % NST) * YSTAGE16;
               for (int w = 0; w < 2 && ok; ++w) {
                 if (!(ok = mbar_wait(smem_u32(&sm.p_full[w]), pb[0] & 1u, abort_flag, kWaitPFull, err))) break;
                 tc_fence_after();
-                issue_ts(A0, T2[0] + 64 * w, ymn, 64 * w, i == 0 && w == 0);
+                issue_ts(A0, rd + 64 * w, ymn, 64 * w, i == 0 && w == 0);   // dQ += dS(i) K(i)
               }
+              if (!ok) break;
               ++pb[0];
               mma_commit(smem_u32(&sm.y_empty[c % NST]));
+              if (i + 1 < n) {
+                issue_prod(region((2 * (i + 1) + 1) % 3), 1, c + 1);        // dP(i+1) over S(i)
+                mma_commit(smem_u32(&sm.s_full[0]));                        // S(i+1) and dP(i+1)
+              }
+              if (i + 2 < n) {
+                if (!(ok = wait_y(c + 2))) break;
+                issue_prod(region((2 * (i + 2)) % 3), 0, c + 2);             // S(i+2) over dS(i)
+              }
             }
           }
           // T(0), T(1) | TS(0) T(2) | TS(1) T(3) | ...
@@ -478,10 +507,11 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
     const int wi = warp & 3;                  // tensor-memory lane quarter
     const int row = wi * 32 + lane;           // row of T1/T2 owned by this thread
     const uint32_t lane_off = (uint32_t)(wi * 32) << 16;
-    // ping-pong: this group's own pair, all its 64 columns; otherwise the one pair, columns [64g, 64g + 64)
-    const uint32_t T1 = tmem + lane_off + (PP ? 64 * g : 0), T2 = tmem + lane_off + 128 + (PP ? 64 * g : 0);
-    constexpr int CB = 0;
-    const int cb = PP ? CB : 64 * g;            // first column of this group in its pair
+    // ping-pong: this group's own pair, all its 64 columns; otherwise the step's pair of rotating
+    // regions (see the MMA issuer), columns [64g, 64g + 64)
+    uint32_t T1 = tmem + lane_off + (PP ? 64 * g : 0), T2 = tmem + lane_off + 128 + (PP ? 64 * g : 0);
+    const int cb = PP ? 0 : 64 * g;             // first column of this group in its pair
+    auto region = [&](int r) -> uint32_t { return tmem + lane_off + (r == 2 ? 384u : 128u * r); };
     const uint32_t A0 = tmem + lane_off + 256, A1 = tmem + lane_off + 256 + D;
     const float sl2 = prm.sl2;
     uint32_t ycnt = 0, ns = 0, n_items = 0;
@@ -622,6 +652,8 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
             const int nv = t.nvalid;
             const bool need = (p.causal && t.pos0 + SR - 1 > it.q0) || nv < SR;
             const uint64_t nl2 = pack2(-l2_row, -l2_row), nd2 = pack2(-dl_row, -dl_row);
+            T1 = region((2 * nsteps) % 3);
+            T2 = region((2 * nsteps + 1) % 3);
             if (!(ok = step([&](int) { return nl2; }, [&](int) { return nd2; },
                             [&](int j) { return j > lim || j >= nv; }, need)))
               break;
