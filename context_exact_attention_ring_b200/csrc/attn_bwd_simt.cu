@@ -146,10 +146,9 @@ __global__ void __launch_bounds__(256) attn_bwd_kv_kernel(Plan p, BwdArgs a) {
   for (int t = 0; t < D / 4; ++t) dk[t] = dv[t] = 0.f;
 
   // query chunks in the order the block travels: ranks s, s+1, ... (ring mode); buffer order (step mode)
-  const int nq_chunks = p.mode == kModeRing ? p.nqc : p.nqc;
   const int s_rank = p.mode == kModeRing ? chunk_owner(p, ks) : 0;
   for (int h = g * G; h < (g + 1) * G; ++h) {
-    for (int n = 0; n < nq_chunks; ++n) {
+    for (int n = 0; n < p.nqc; ++n) {
       int qs;
       if (p.mode == kModeRing) {
         const int r = (s_rank + n / p.cpr) % p.P;

@@ -43,6 +43,8 @@ CASES = [
     W.Prefill("bf16_ragged_chunks", "bf16", True, "zigzag", 2, 3, 3, 1200, 128, 3, 605),
     W.Prefill("bf16_zigzag4_d64", "bf16", True, "zigzag4", 1, 4, 1, 2048, 64, 2, 606),
     W.Prefill("bf16_contiguous_noncausal", "bf16", False, "contiguous", 1, 2, 2, 1024, 128, 4, 607),
+    W.Prefill("bf16_odd_group_zigzag3", "bf16", True, "zigzag3", 1, 6, 2, 1536, 128, 2, 611),
+    W.Prefill("bf16_striped_ragged_gqa", "bf16", True, "striped", 1, 8, 2, 2700, 64, 3, 612),
 ]
 
 
