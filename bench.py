@@ -219,39 +219,71 @@ def run_ours(args):
     dvalue = replica_throughput(dbytes, args.steps, world, dec_sum) / 1e9    # GB/s, all ranks
 
     # ---------------------------------------------------------------- end to end (host buffers)
+    # Every step copies its inputs from pinned host memory, runs ring_attn_fwd and copies out and
+    # lse back to pinned host memory.  Steps are pipelined the way a serving loop uses the
+    # asynchronous API: two device slots and three streams, so the host-to-device copy of step
+    # i+1 and the device-to-host copy of step i-1 run while step i computes.
     e2e = None
     if not args.no_e2e:
         hq = q.cpu().pin_memory()
         hk = k.cpu().pin_memory()
         hv = v.cpu().pin_memory()
-        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        e2e_steps = max(1, min(args.steps, 3))
+        hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        hlse = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+        slots = [dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v), o=torch.empty_like(out),
+                      l=torch.empty_like(lse)) for _ in range(2)]
+        s_in, s_c, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        inputs_free = [torch.cuda.Event() for _ in range(2)]    # compute of the slot's last step is done
+        inputs_ready = [torch.cuda.Event() for _ in range(2)]
+        outputs_free = [torch.cuda.Event() for _ in range(2)]   # the slot's last outputs are on the host
+        computed = [torch.cuda.Event() for _ in range(2)]
+        e2e_steps = max(2, args.steps)
 
-        def e2e_step():
-            q2 = hq.to(dev, non_blocking=True)
-            k2 = hk.to(dev, non_blocking=True)
-            v2 = hv.to(dev, non_blocking=True)
-            o2, l2 = ra.ring_attn_fwd(q2, k2, v2, cfg.P, causal=True, layout=cfg.layout, scale=cfg.scale)
-            hout.copy_(o2, non_blocking=True)
-            hlse.copy_(l2, non_blocking=True)
+        def e2e_step(i):
+            sl, s_ = slots[i % 2], i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(inputs_free[s_])
+                sl["q"].copy_(hq, non_blocking=True)
+                sl["k"].copy_(hk, non_blocking=True)
+                sl["v"].copy_(hv, non_blocking=True)
+                inputs_ready[s_].record(s_in)
+            with torch.cuda.stream(s_c):
+                s_c.wait_event(inputs_ready[s_])
+                if i >= 2:
+                    s_c.wait_event(outputs_free[s_])
+                ra.ring_attn_fwd(sl["q"], sl["k"], sl["v"], cfg.P, causal=True, layout=cfg.layout, scale=cfg.scale,
+                                 out=sl["o"], lse=sl["l"])
+                computed[s_].record(s_c)
+                inputs_free[s_].record(s_c)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[s_])
+                hout[s_].copy_(sl["o"], non_blocking=True)
+                hlse[s_].copy_(sl["l"], non_blocking=True)
+                outputs_free[s_].record(s_out)
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         barrier(dist)
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(st)
-        for _ in range(e2e_steps):
-            e2e_step()
-        a1.record(st)
+        a0.record(s_in)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        s_in.wait_stream(s_out)
+        a1.record(s_in)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(dist, a0.elapsed_time(a1))
+        # the result really came back: the last step's output on the host equals the device result
+        assert torch.equal(hout[(e2e_steps - 1) % 2][0, :4].to(dev), out[0, :4])
         h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
-        d2h = hout.numel() * 2 + hlse.numel() * 4
+        d2h = hout[0].numel() * 2 + hlse[0].numel() * 4
         e2e = {"value": round(flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(e2e_ms / e2e_steps, 3), "path": "pinned host -> ring_attn_fwd -> pinned host"}
+               "ms_per_step": round(e2e_ms / e2e_steps, 3), "steps": e2e_steps,
+               "path": "pinned host -> ring_attn_fwd -> pinned host; 2 device slots, copy-in / compute / copy-out "
+                       "streams overlapping consecutive steps"}
 
     # ---------------------------------------------------------------- roofline of the dominant kernel
     pre_avg = statistics.mean(pre_ms)
