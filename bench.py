@@ -285,6 +285,34 @@ def run_ours(args):
                "path": "pinned host -> ring_attn_fwd -> pinned host; 2 device slots, copy-in / compute / copy-out "
                        "streams overlapping consecutive steps"}
 
+    # ---------------------------------------------------------------- backward of the same ring
+    # Timed after the main region on the same inputs (the forward's out and lse), outside the
+    # step; the usual convention counts 2.5x the forward's FLOPs for dQ, dK, dV.
+    bwd = None
+    if not args.no_bwd:
+        g = torch.Generator(device=dev).manual_seed(cfg.seed + 7)
+        gout = torch.randn(q.shape, generator=g, device=dev).to(q.dtype)
+        gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(int(ra.lib().ring_attn_bwd_workspace_bytes(cfg.B, cfg.Hq, cfg.S)), device=dev,
+                         dtype=torch.uint8)
+        bfn = lambda: ra.ring_attn_bwd(q, k, v, out, lse, gout, cfg.P, causal=True, layout=cfg.layout,
+                                       scale=cfg.scale, dq=gq, dk=gk, dv=gv, workspace=ws)
+        bfn()
+        torch.cuda.synchronize()
+        barrier(dist)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(st)
+        for _ in range(2):
+            bfn()
+        b1.record(st)
+        torch.cuda.synchronize()
+        bwd_ms = max_over_ranks(dist, b0.elapsed_time(b1)) / 2
+        bwd_tf = 2.5 * flops * world / (bwd_ms / 1e3) / 1e12
+        bwd = {"metric": "causal-adjusted backward TFLOP/s (2.5x the forward FLOPs)", "value": round(bwd_tf, 1),
+               "unit": "TFLOP/s", "ms_per_call": round(bwd_ms, 3), "launches_per_call": 3,
+               "kernels": "bwd_delta_kernel + attn_bwd_tc_kernel<128,true> (dK, dV) + <128,false> (dQ)"}
+        del gout, gq, gk, gv, ws
+
     # ---------------------------------------------------------------- roofline of the dominant kernel
     pre_avg = statistics.mean(pre_ms)
     achieved_tf = flops / (pre_avg / 1e3) / 1e12
@@ -321,6 +349,7 @@ def run_ours(args):
                                 "peak_kind": f"{pk_kind} HBM copy"}},
         "prefill_ms_per_step": round(pre_avg, 3),
         "e2e": e2e,
+        "backward": bwd,
         "gpu_launches": args.steps * 3,
         "clocks": clk,
     }
@@ -515,6 +544,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward timing after the main region")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)
