@@ -148,6 +148,38 @@ def decode_bytes(cfg, lens: np.ndarray) -> float:
     return kv + q + parts + out
 
 
+def step_ring(ra, cfg, q, k, v, dev):
+    """The whole ring of `cfg` through the step API: for each rank r, a fresh
+    state, then P calls of ring_attn_step (hop t folds the block that started
+    on rank (r - t) mod P), then the finalisation of the state.  The state
+    (m, l, O fp32) is read and written in HBM by every call.  Returns the
+    closure, the number of library launches per ring, and rank P-1's output
+    with its token positions (for a check against the fused ring)."""
+    from context_exact_attention_ring_b200 import ring
+    P = cfg.P
+    own = ring.split_chunks(P, cfg.layout)
+    C = cfg.S // (P * len(own[0]))
+    rows = [ring.shard_rows(cfg.S, P, cfg.layout, r).to(dev) for r in range(P)]
+    qs = [q[:, rr].contiguous() for rr in rows]
+    ks = [k[:, rr].contiguous() for rr in rows]
+    vs = [v[:, rr].contiguous() for rr in rows]
+    S_loc = int(rows[0].numel())
+    m, l, O = ra.new_state(cfg.B, cfg.Hq, S_loc, cfg.D, dev)
+    o_r = torch.empty((cfg.B, S_loc, cfg.Hq, cfg.D), device=dev, dtype=q.dtype)
+    lse_r = torch.empty((cfg.B, cfg.Hq, S_loc), device=dev, dtype=torch.float32)
+
+    def run():
+        for r in range(P):
+            ra.ring_attn_state_init(m, l, O)
+            for t in range(P):
+                src = (r - t) % P
+                ra.ring_attn_step(qs[r], ks[src], vs[src], m, l, O, own[r], own[src], C, causal=cfg.causal,
+                                  scale=cfg.scale)
+            ra.ring_attn_state_finalize(m, l, O, dtype=q.dtype, out=o_r, lse=lse_r)
+
+    return run, P * (P + 2), o_r, rows[P - 1]
+
+
 def run_ours(args):
     import context_exact_attention_ring_b200 as ra
 
@@ -313,6 +345,36 @@ def run_ours(args):
                "kernels": "bwd_delta_kernel + attn_bwd_tc_kernel<128,true> (dK, dV) + <128,false> (dQ)"}
         del gout, gq, gk, gv, ws
 
+    # ---------------------------------------------------------------- the same ring through the step API
+    # P ranks x P hops of ring_attn_step with the state in HBM (what a multi-GPU ring runs per rank),
+    # timed after the main region; its output is checked against the fused ring's.
+    step_api = None
+    if not args.no_step:
+        srun, slaunch, so, srows = step_ring(ra, cfg, q, k, v, dev)
+        srun()
+        torch.cuda.synchronize()
+        diff = float((so.float() - out[:, srows].float()).abs().max())
+        if not diff <= 2e-2:
+            raise RuntimeError(f"step API result differs from the fused ring by {diff}")
+        barrier(dist)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(st)
+        for _ in range(2):
+            srun()
+        c1.record(st)
+        torch.cuda.synchronize()
+        if ra.ring_attn_device_error()[0] != ra.RING_OK:
+            raise RuntimeError("device error in the step API timing")
+        step_ms = max_over_ranks(dist, c0.elapsed_time(c1)) / 2
+        step_tf = flops * world / (step_ms / 1e3) / 1e12
+        peak_s = pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]
+        step_api = {"metric": "causal-adjusted TFLOP/s of the same ring through ring_attn_step "
+                              "(P ranks x P hops, state read and written in HBM by every call)",
+                    "value": round(step_tf, 1), "unit": "TFLOP/s", "ms_per_ring": round(step_ms, 3),
+                    "calls_per_ring": cfg.P * cfg.P, "launches_per_ring": slaunch,
+                    "frac": round(step_tf / world / peak_s, 4), "max_abs_diff_vs_fused_out": round(diff, 5)}
+        del srun, so
+
     # ---------------------------------------------------------------- roofline of the dominant kernel
     pre_avg = statistics.mean(pre_ms)
     achieved_tf = flops / (pre_avg / 1e3) / 1e12
@@ -350,6 +412,7 @@ def run_ours(args):
         "prefill_ms_per_step": round(pre_avg, 3),
         "e2e": e2e,
         "backward": bwd,
+        "step_api": step_api,
         "gpu_launches": args.steps * 3,
         "clocks": clk,
     }
@@ -463,6 +526,8 @@ PROFILE_CASES = {
                                            name="ring_bf16_causal_zigzag4_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
     "tc_full_striped": dataclasses.replace(W.CFG4, layout="striped",
                                            name="ring_bf16_causal_striped_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),
+    # the S=128k GQA workload as P x P calls of ring_attn_step (state in HBM)
+    "step_full": W.CFG4,
     # backward of the S=128k GQA workload (tensor cores: K/V-major then Q-major launch)
     "bwd_full": W.CFG4,
     # backward of the causal zig-zag MHA workload with 1% of keys x8 (a small case for ncu)
@@ -496,6 +561,10 @@ def run_profile(args):
                                       scale=cfg.scale, dq=dq, dk=dk, dv=dv, workspace=ws)
         # the usual backward convention: 2.5x the forward's FLOPs (the two launches compute 3.5x)
         work, unit = 2.5 * cfg.flops() / 1e12, "TFLOP/s"
+    elif isinstance(cfg, W.Prefill) and name.startswith("step"):
+        q, k, v = W.prefill_inputs(cfg, dev)
+        fn, _, _, _ = step_ring(ra, cfg, q, k, v, dev)
+        work, unit = cfg.flops() / 1e12, "TFLOP/s"
     elif isinstance(cfg, W.Prefill):
         q, k, v = W.prefill_inputs(cfg, dev)
         out = torch.empty_like(q)
@@ -545,6 +614,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward timing after the main region")
+    ap.add_argument("--no-step", action="store_true", help="skip the step-API timing after the main region")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)
