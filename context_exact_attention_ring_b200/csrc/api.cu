@@ -184,7 +184,7 @@ ring_status decode_args(const void* q, const void* k, const void* v, const int32
   if ((long long)B * Smax * Hkv * D >= (1LL << 42)) return RING_EINVAL;
   if (dtype != RING_BF16 || D != 128) return RING_EUNSUPPORTED;
   const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4) return RING_EUNSUPPORTED;
+  if (!decode_group_supported(G)) return RING_EUNSUPPORTED;
   const size_t need = decode_workspace_bytes(B, Hq, Hkv, Smax, D, P);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need) return RING_EINVAL;
   DecodeArgs a{};

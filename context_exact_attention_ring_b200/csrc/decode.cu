@@ -1,26 +1,34 @@
-// Split-KV single-token decode ("NVIDIA unveils Helix Parallelism", Phase 1:
-// the KV cache sharded along the sequence; each shard yields a partial result
-// that is merged afterwards).
+// Split-KV single-token decode on the tensor cores ("NVIDIA unveils Helix
+// Parallelism", Phase 1: the KV cache sharded along the sequence; each shard
+// yields a partial result that is merged afterwards).
 //
 // Work unit = (chunk p, batch b, kv head g, sub-split s): RPS consecutive rows
 // of one chunk.  A persistent grid (one CTA per SM) walks the units in chunk
 // order, so the always-full early chunks come first and the ragged tails of
-// the sequences last.  Per CTA:
-//   warp 0       TMA producer: 96-row K and V boxes into a 4-stage ring of
-//                shared memory (bounded waits on the stage barriers);
-//   warps 1..12  consumers: a half warp owns one K/V row per pass; a lane
-//                holds 8 of the 128 dims of every query head of the kv head
-//                (scaled by scale*log2 e), so each K/V element is widened to
-//                fp32 once; partial dot products (packed f32x2 FMA) are
-//                reduced by a transposing half-warp butterfly that leaves each
-//                lane the score of one head; that head's lanes fold the row
-//                into the running (m, l) -- the online-softmax update of
-//                "Lesson 8: Context Parallelism", section 3 -- keeping a stale
-//                max until a score exceeds it by 2^8 (exact: the same base
-//                scales l and O), and broadcast the weight to the other lanes
-//                for the PV update.
-// At the end of a unit the 32 group states are folded (shuffles, then shared
-// memory).  A chunk covered by one sub-split writes its partial directly;
+// the sequences last.  The G query heads of a kv head share every K/V row, so
+// a 128-row K/V tile is one pair of small tcgen05 products (the heads padded
+// to the smallest N of the instruction, 16):
+//   S^T = K Q^T      M = 128 keys,  N = 16 heads, K = 128 dims  (K, Q K-major)
+//   O^T += V^T P^T   M = 128 dims,  N = 16 heads, K = 128 keys  (V MN-major)
+// with S^T and O^T in tensor memory.  Warp roles:
+//   warps 0-3  softmax group: thread t owns tensor-memory lane t, i.e. key
+//              row t of S^T and dimension t of O^T; it turns its G scores
+//              into weights against a per-head base shared by the whole CTA
+//              and writes them (bf16) as P^T, the B operand of O^T, in
+//              shared memory;
+//   warp 4     TMA producer: the unit's query rows (128-byte swizzle, padded
+//              rows stay zero), then K and V tiles into a 3-stage ring;
+//   warp 5     MMA issuer and tensor-memory owner: S(j+1) is issued before
+//              the O^T update of tile j, so the softmax of tile j+1 overlaps it.
+// The online softmax of "Lesson 8: Context Parallelism", section 3, with a
+// lazy base: a head's base moves only when one of its scores exceeds it by
+// more than 2^8 (a block-wide OR decides, and only then are the tile maxima
+// reduced and O^T rescaled), which is exact because l and O share the base.
+// Two sums are kept, as in the prefill kernel: the fp32 sum of the weights
+// (gives lse) and the sum of their bf16 values (normalises O, so that the
+// weights applied to V sum to one).
+// At the end of a unit the thread of dimension d holds O[h][d] for the G
+// heads.  A chunk covered by one sub-split writes its partial directly;
 // otherwise every sub-split writes to the workspace and the last CTA to
 // arrive (atomic counter, reset by that CTA) folds them into the chunk's
 // partial.  With an output buffer the merge runs in the same launch: the CTA
@@ -30,6 +38,7 @@
 // positions [p*C, (p+1)*C)) or, for a cache filled by the round-robin append
 // of "NVIDIA unveils Helix Parallelism" (KV cache growth), from the chunk's
 // own fill count.  The kernel is HBM-bound: each valid K/V byte is read once.
+// Every wait is bounded; the softmax warps leave together (block-wide ORs).
 #include <cuda_bf16.h>
 #include <type_traits>
 #include <cuda_runtime.h>
@@ -42,16 +51,19 @@ namespace ra {
 
 namespace dec {
 constexpr int D = 128;
-constexpr int ROWS = 96;                    // rows per stage
-constexpr int NST = 4;                      // stages
-constexpr int RPS = 4032;                   // rows per sub-split (a multiple of ROWS)
-constexpr int STAGE_BYTES = 2 * ROWS * D * 2;
-constexpr int NCW = 12;                     // consumer warps
-constexpr int UPI = 4;                      // rows per half warp handled together
-constexpr int THREADS = 32 * (1 + NCW);
-static_assert(ROWS % (2 * UPI * NCW) == 0, "a stage is covered by whole iterations of all consumer warps");
-static_assert(RPS % ROWS == 0, "stages never straddle two sub-splits");
+constexpr int BN = 128;                     // K/V rows per tile (the M of S^T)
+constexpr int NQ = 16;                      // query heads padded to the smallest N of the product
+constexpr int NST = 3;                      // K/V stages
+constexpr int RPS = 4096;                   // rows per sub-split (a multiple of BN)
+constexpr int SLAB = BN * 64 * 2;           // one 128-row x 64-column bf16 box (16 KB)
+constexpr int TILE_BYTES = BN * D * 2;      // one K or V tile (32 KB)
+constexpr int QSLAB = NQ * 128;             // 16 rows x 64 columns of bf16 (2 KB)
+constexpr int NSW = 4;                      // softmax warps
+constexpr int CT = 32 * NSW;                // softmax threads
+constexpr int THREADS = CT + 64;            // + producer warp + MMA warp
+constexpr uint32_t TMEM_COLS = 64;          // S^T (2 x 16 columns), O^T (16 columns)
 constexpr float LAZY = 8.f;                 // log2 of the largest tolerated growth before rescaling
+static_assert(RPS % BN == 0, "tiles never straddle two sub-splits");
 }  // namespace dec
 
 struct DecGeom {
@@ -76,87 +88,6 @@ __device__ __forceinline__ int chunk_end(const DecodeArgs& a, const DecodeExtra&
   const int len = min(max(a.seqlens[b], 0), a.Smax);
   return min(len, (p + 1) * Cd);
 }
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float* f) {
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(u[i] << 16);
-    f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
-  }
-}
-
-// 8 bf16 -> 4 packed pairs of float (exact widening)
-__device__ __forceinline__ void bf16x8_to_f32x2(const uint4 w, uint64_t* f2) {
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) f2[i] = pack2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
-}
-
-// Each lane keeps its G heads in a lane-dependent order (slot i holds head
-// head_of_slot(lane, i)) chosen so that the transposing half-warp sum below
-// needs no selects: at each of the first log2(G) butterfly levels a lane keeps
-// the first half of its remaining slots and sends the second half, which its
-// partner holds, in the same head order, in its own second half.
-template <int G>
-__device__ __forceinline__ int head_of_slot(int lane, int i) {
-  const int hi = (lane >> 3) & 1, odd = (lane >> 2) & 1;
-  if constexpr (G == 4) {
-    const int pair = (i >> 1) ? 1 - hi : hi;
-    const int mem = (i & 1) ? 1 - odd : odd;
-    return 2 * pair + mem;
-  } else if constexpr (G == 2) {
-    return i ? 1 - hi : hi;
-  } else {
-    return 0;
-  }
-}
-
-// Sum over the 16 lanes of a half warp of the G per-head partial sums (slot
-// order), leaving in every lane the full sum of head own_head(lane) = the head
-// of its slot 0.  G = 4 takes 5 shuffles instead of 16.
-template <int G>
-__device__ __forceinline__ float half_warp_transpose_sum(const float (&v)[G]) {
-  if constexpr (G == 4) {
-    const float k0 = v[0] + __shfl_xor_sync(0xffffffffu, v[2], 8);
-    const float k1 = v[1] + __shfl_xor_sync(0xffffffffu, v[3], 8);
-    float x = k0 + __shfl_xor_sync(0xffffffffu, k1, 4);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    return x;
-  } else if constexpr (G == 2) {
-    float x = v[0] + __shfl_xor_sync(0xffffffffu, v[1], 8);
-    x += __shfl_xor_sync(0xffffffffu, x, 4);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    return x;
-  } else {
-    float x = v[0];
-#pragma unroll
-    for (int off = 8; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-    return x;
-  }
-}
-
-// Lane (xor distance) in the same half warp whose slot 0 holds the head of
-// this lane's slot i: the reduced score of a head is replicated in every lane
-// whose slot 0 is that head, so a butterfly shuffle reaches it.
-template <int G>
-__device__ __forceinline__ constexpr int slot_xor(int i) {
-  return G == 4 ? (i << 2) : G == 2 ? (i << 3) : 0;
-}
-
-template <int G>
-struct DecSmem {
-  alignas(1024) uint8_t stage[dec::NST][dec::STAGE_BYTES];
-  float wpart[dec::NCW][G][dec::D];
-  float wm[dec::NCW][G];
-  float wl[dec::NCW][G];
-  alignas(8) uint64_t full[dec::NST];
-  alignas(8) uint64_t empty[dec::NST];
-  int is_last;      // set by one thread between two consumer barriers, read by all after the second
-  int abort_flag;
-};
 
 // Counts one finished chunk of (b, kv head g) with an acquire-release atomic
 // (after a barrier that follows the CTA's writes of that chunk's partial, so
@@ -241,9 +172,9 @@ __device__ __noinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x,
     for (int k = 0; k < D / 32; ++k) out[(bh0 + h) * D + lane + 32 * k] = __float2bfloat16_rn(acc[h][k]);
 }
 
-// Called by consumer warp 0 (all lanes) after the CTA's writes of a chunk's
-// final partial and a consumer barrier: one lane counts the chunk; the warp
-// that completes the count of (b, g) merges it.  The other consumer warps do
+// Called by softmax warp 0 (all lanes) after the CTA's writes of a chunk's
+// final partial and a softmax-group barrier: one lane counts the chunk; the warp
+// that completes the count of (b, g) merges it.  The other softmax warps do
 // not wait.
 template <int G>
 __device__ __forceinline__ void chunk_final_count(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
@@ -255,306 +186,488 @@ __device__ __forceinline__ void chunk_final_count(const DecodeArgs& a, const Dec
   }
 }
 
+template <int G>
+struct DecSmem {
+  alignas(1024) uint8_t kv[dec::NST][2][dec::TILE_BYTES];   // K, V tiles: 2 slabs of 128 rows x 128 B each
+  alignas(1024) uint8_t q[2][2 * dec::QSLAB];                 // padded query rows, by unit parity
+  alignas(1024) uint8_t pt[2][2 * dec::QSLAB];                // P^T (16 head rows x 128 keys), by tile parity
+  float red[2][dec::NSW][G];                                  // cross-warp reductions
+  alignas(8) uint64_t kv_full[dec::NST], kv_empty[dec::NST];
+  alignas(8) uint64_t q_full[2], q_empty[2];
+  alignas(8) uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  alignas(8) uint64_t o_full, o_free, teardown;
+  uint32_t tmem_base;
+  int is_last;      // set by one thread between two softmax-group barriers, read by all after the second
+  int abort_flag;
+};
+
+// Instruction descriptor of kind::f16 (bf16 A and B, f32 accumulation) with
+// the major-ness of both operands (bit 15: A, bit 16: B; 1 = MN-major).
+__host__ __device__ constexpr uint32_t idesc_f16_ab(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// G consecutive 32-bit columns of this warp's 32 lanes (G = 1, 2, 4, 8, 16)
+template <int G>
+__device__ __forceinline__ void tmem_ld_g(uint32_t taddr, float (&v)[G]) {
+  uint32_t r[G];
+  if constexpr (G == 1) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+  } else if constexpr (G == 2) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+  } else if constexpr (G == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(taddr));
+  } else if constexpr (G == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  } else {
+    static_assert(G == 16, "G");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  }
+#pragma unroll
+  for (int i = 0; i < G; ++i) v[i] = __uint_as_float(r[i]);
+}
+template <int G>
+__device__ __forceinline__ void tmem_st_g(uint32_t taddr, const float (&v)[G]) {
+  uint32_t r[G];
+#pragma unroll
+  for (int i = 0; i < G; ++i) r[i] = __float_as_uint(v[i]);
+  if constexpr (G == 1) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r[0]) : "memory");
+  } else if constexpr (G == 2) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(r[0]), "r"(r[1])
+                 : "memory");
+  } else if constexpr (G == 4) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
+  } else if constexpr (G == 8) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+  } else {
+    static_assert(G == 16, "G");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Unit u -> (b, kv head g, chunk p, sub-split) and its rows [r0, r1) (r0 >= r1: nothing to read).
+struct DecUnit {
+  int b, g, p, sub, r0, r1, ntiles;
+};
+template <bool kShard>
+__device__ __forceinline__ DecUnit dec_unit(const DecodeArgs& a, const DecodeExtra& x, const DecGeom& geo, int u) {
+  DecUnit U;
+  int t = u;
+  U.sub = t % geo.nsub; t /= geo.nsub;
+  U.g = t % a.Hkv; t /= a.Hkv;
+  U.b = t % a.B;
+  U.p = t / a.B;
+  U.r0 = U.p * geo.Cd + U.sub * dec::RPS;
+  U.r1 = min(U.r0 + dec::RPS, chunk_end<kShard>(a, x, geo.Cd, U.b, U.p));
+  U.ntiles = U.r0 < U.r1 ? (U.r1 - U.r0 + dec::BN - 1) / dec::BN : 0;
+  return U;
+}
+
 // kMerge: the launch also merges the partials (a.out != null); kShard: valid
 // rows come from per-chunk fill counts (a.shard_lens != null).  Separate
 // instantiations, so that the plain partial kernel carries none of their code.
 template <int G, bool kMerge, bool kShard>
 __global__ void __launch_bounds__(dec::THREADS, 1)
-    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DecodeArgs a,
-                  DecGeom geo, DecodeExtra x) {
+    decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, DecodeArgs a, DecGeom geo, DecodeExtra x) {
   using namespace dec;
   extern __shared__ uint8_t smem_raw[];
   DecSmem<G>& sm = *reinterpret_cast<DecSmem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sm.abort_flag;
+  unsigned int* err = a.err;
 
+  // the padded query rows and the padded P^T rows stay zero (never written again)
+  {
+    uint4* z = reinterpret_cast<uint4*>(&sm.q[0][0]);
+    constexpr int n16 = (int)((sizeof(sm.q) + sizeof(sm.pt)) / 16);
+    for (int i = threadIdx.x; i < n16; i += THREADS) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(smem_u32(&sm.full[s]), 1);
-      mbar_init(smem_u32(&sm.empty[s]), NCW);
+      mbar_init(smem_u32(&sm.kv_full[s]), 1);
+      mbar_init(smem_u32(&sm.kv_empty[s]), 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.q_full[i]), 1);
+      mbar_init(smem_u32(&sm.q_empty[i]), 1);
+      mbar_init(smem_u32(&sm.s_full[i]), 1);
+      mbar_init(smem_u32(&sm.s_free[i]), CT);
+      mbar_init(smem_u32(&sm.p_full[i]), CT);
+      mbar_init(smem_u32(&sm.o_done[i]), 1);
+    }
+    mbar_init(smem_u32(&sm.o_full), 1);
+    mbar_init(smem_u32(&sm.o_free), CT);
+    mbar_init(smem_u32(&sm.teardown), 1);
     sm.abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
   }
+  if (warp == NSW + 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
+  if (warp == NSW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const uint64_t pol = l2_policy_evict_first();
-      uint32_t cnt = 0;
+      const uint64_t pol_kv = l2_policy_evict_first();
+      const uint64_t pol_q = l2_policy_evict_last();
+      uint32_t cnt = 0, nq = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < geo.units && ok; u += gridDim.x) {
-        int t = u;
-        const int sub = t % geo.nsub; t /= geo.nsub;
-        const int g = t % a.Hkv; t /= a.Hkv;
-        const int b = t % a.B;
-        const int p = t / a.B;
-        const int r0 = p * geo.Cd + sub * RPS;
-        const int r1 = min(r0 + RPS, chunk_end<kShard>(a, x, geo.Cd, b, p));
-        for (int row = r0; row < r1; row += ROWS) {
+        const DecUnit U = dec_unit<kShard>(a, x, geo, u);
+        if (U.ntiles == 0) continue;
+        const int qb = nq & 1;
+        if (nq >= 2 && !mbar_wait(smem_u32(&sm.q_empty[qb]), ((nq >> 1) - 1) & 1u, abort_flag, kWaitQEmpty, err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t qf = smem_u32(&sm.q_full[qb]);
+        mbar_arrive_expect_tx(qf, G * D * 2);
+        for (int sl = 0; sl < 2; ++sl)
+          tma_load_4d(smem_u32(sm.q[qb]) + sl * QSLAB, &tmQ, qf, sl * 64, 0, U.b * a.Hq + U.g * G, 0, pol_q);
+        ++nq;
+        for (int j = 0; j < U.ntiles; ++j) {
           const int s = cnt % NST;
-          const uint32_t ph = (cnt / NST) & 1u;
-          if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag, kWaitDecodeEmpty, a.err)) { ok = false; break; }
-          const uint32_t fb = smem_u32(&sm.full[s]);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          const uint32_t dst = smem_u32(sm.stage[s]);
-          tma_load_4d(dst, &tmK, fb, 0, g, row, b, pol);
-          tma_load_4d(dst + ROWS * D * 2, &tmV, fb, 0, g, row, b, pol);
+          if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((cnt / NST) & 1u) ^ 1u, abort_flag, kWaitDecodeEmpty, err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&sm.kv_full[s]);
+          mbar_arrive_expect_tx(fb, 2 * TILE_BYTES);
+          const int row = U.r0 + j * BN;
+          for (int sl = 0; sl < 2; ++sl) {
+            tma_load_4d(smem_u32(sm.kv[s][0]) + sl * SLAB, &tmK, fb, sl * 64, U.g, row, U.b, pol_kv);
+            tma_load_4d(smem_u32(sm.kv[s][1]) + sl * SLAB, &tmV, fb, sl * 64, U.g, row, U.b, pol_kv);
+          }
           ++cnt;
         }
       }
       // do not leave while copies are still landing in shared memory
-      for (uint32_t c = (cnt > (uint32_t)NST ? cnt - NST : 0); c < cnt; ++c) {
-        const int s = c % NST;
-        mbar_wait(smem_u32(&sm.full[s]), (c / NST) & 1u, nullptr, kWaitTeardown, a.err);
-      }
+      for (uint32_t c = (cnt > (uint32_t)NST ? cnt - NST : 0); c < cnt; ++c)
+        mbar_wait(smem_u32(&sm.kv_full[c % NST]), (c / NST) & 1u, nullptr, kWaitTeardown, err);
+      for (uint32_t c = (nq > 2u ? nq - 2u : 0u); c < nq; ++c)
+        mbar_wait(smem_u32(&sm.q_full[c & 1]), (c >> 1) & 1u, nullptr, kWaitTeardown, err);
     }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
-  // Lane layout: each half warp (16 lanes) owns one K/V row per pass; lane
-  // (dh, j) holds dims [dh*64 + 8j, dh*64 + 8j + 8) of every one of the G
-  // query heads and of their output rows (the 16 lanes read the row's 256
-  // contiguous bytes).  Per row: partial dot products, a transposing
-  // half-warp reduction that leaves each lane the full score of one head,
-  // the online-softmax update done by that head's lanes, and a broadcast of
-  // the G weights p_h for the PV update.  Each K/V element is widened once.
-  const int cw = warp - 1;                 // consumer warp 0..NCW-1
-  const int ctid = threadIdx.x - 32;       // 0..32*NCW-1
-  const int half = lane >> 4;
-  const int dcol = ((lane >> 3) & 1) * 64 + (lane & 7) * 8;   // first dim of this lane
-  const int oh = head_of_slot<G>(lane, 0);   // the head whose running (m, l) this lane keeps
-  const float qscale = a.scale * 1.4426950408889634f;
-  uint32_t cnt = 0;
-  const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(a.q);
-  constexpr int CT = 32 * NCW;
-
-  for (int u = blockIdx.x; u < geo.units; u += gridDim.x) {
-    int t = u;
-    const int sub = t % geo.nsub; t /= geo.nsub;
-    const int g = t % a.Hkv; t /= a.Hkv;
-    const int b = t % a.B;
-    const int p = t / a.B;
-    const int c0 = p * geo.Cd;
-    const int nvalid_chunk = chunk_rows<kShard>(a, x, geo.Cd, b, p);
-    const int n_live = (nvalid_chunk + RPS - 1) / RPS;
-    const int r0 = c0 + sub * RPS;
-    const int r1 = min(r0 + RPS, c0 + nvalid_chunk);
-
-    if (nvalid_chunk == 0) {
-      if (sub == 0) {
-        for (int e = ctid; e < G * D; e += CT) {
-          const int h = e / D, d = e - h * D;
-          a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = 0.f;
+  } else if (warp == NSW + 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t tS[2] = {tmem, tmem + 16}, tO = tmem + 32;
+      constexpr uint32_t idS = idesc_f16_ab(BN, NQ, false, false);   // S^T = K Q^T
+      constexpr uint32_t idPV = idesc_f16_ab(D, NQ, true, false);    // O^T += V^T P^T
+      uint32_t cnt = 0, nq = 0, tj = 0, nu = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < geo.units && ok; u += gridDim.x) {
+        const DecUnit U = dec_unit<kShard>(a, x, geo, u);
+        if (U.ntiles == 0) continue;
+        const int qb = nq & 1;
+        if (!mbar_wait(smem_u32(&sm.q_full[qb]), (nq >> 1) & 1u, abort_flag, kWaitQFull, err)) { ok = false; break; }
+        tc_fence_after();
+        ++nq;
+        const uint64_t qdesc = sw128_desc(smem_u32(sm.q[qb]), 16, 1024);
+        for (int j = 0; j <= U.ntiles && ok; ++j) {
+          if (j < U.ntiles) {
+            // S^T(j) into buffer t & 1, once the softmax has read S^T(t - 2) from it
+            const uint32_t c = cnt + j, s = c % NST, t = tj + j, sb = t & 1u;
+            if (!mbar_wait(smem_u32(&sm.kv_full[s]), (c / NST) & 1u, abort_flag, kWaitDecodeFull, err)) {
+              ok = false;
+              break;
+            }
+            if (t >= 2 && !mbar_wait(smem_u32(&sm.s_free[sb]), ((t >> 1) - 1) & 1u, abort_flag, kWaitSFull, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t kdesc = sw128_desc(smem_u32(sm.kv[s][0]), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+              mma_ss(tS[sb], kdesc + ((((k >> 2) * SLAB) + (k & 3) * 32) >> 4),
+                     qdesc + ((((k >> 2) * QSLAB) + (k & 3) * 32) >> 4), idS, k > 0 ? 1u : 0u);
+            mma_commit(smem_u32(&sm.s_full[sb]));
+            if (j == U.ntiles - 1) mma_commit(smem_u32(&sm.q_empty[qb]));
+          }
+          if (j > 0) {
+            // O^T += V^T(j-1) P^T(j-1)
+            const uint32_t c = cnt + j - 1, s = c % NST, t = tj + j - 1, pb = t & 1u;
+            if (!mbar_wait(smem_u32(&sm.p_full[pb]), (t >> 1) & 1u, abort_flag, kWaitPFull, err)) {
+              ok = false;
+              break;
+            }
+            if (j == 1 && nu > 0 &&
+                !mbar_wait(smem_u32(&sm.o_free), (nu - 1) & 1u, abort_flag, kWaitOFinal, err)) {   // O^T was read
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t vdesc = sw128_desc(smem_u32(sm.kv[s][1]), SLAB, 1024);
+            const uint64_t pdesc = sw128_desc(smem_u32(sm.pt[pb]), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < BN / 16; ++k)
+              mma_ss(tO, vdesc + ((k * 16 * 128) >> 4), pdesc + ((((k >> 2) * QSLAB) + (k & 3) * 32) >> 4), idPV,
+                     (j > 1 || k > 0) ? 1u : 0u);
+            mma_commit(smem_u32(&sm.o_done[pb]));
+            mma_commit(smem_u32(&sm.kv_empty[s]));
+          }
         }
-        if (ctid < G) a.part_lse[(size_t)(b * a.Hq + g * G + ctid) * a.P + p] = -CUDART_INF_F;
-        if constexpr (kMerge) {
-          named_bar_sync(1, CT);   // the chunk's partial is written before it is counted
-          if (cw == 0) chunk_final_count<G>(a, x, b, g, lane);
-        }
+        if (!ok) break;
+        mma_commit(smem_u32(&sm.o_full));
+        cnt += U.ntiles;
+        tj += U.ntiles;
+        ++nu;
       }
-      continue;
+      // every MMA issued so far must be complete before tensor memory is freed
+      mma_commit(smem_u32(&sm.teardown));
+      mbar_wait(smem_u32(&sm.teardown), 0, nullptr, kWaitTeardown, err);
     }
-    if (r0 >= r1) continue;
-
-    // this lane's 8 dims of the G query heads, scaled by scale * log2(e)
-    uint64_t q2[G][4];   // slot order (see head_of_slot)
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float f[8];
-      const int head = head_of_slot<G>(lane, h);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + ((size_t)b * a.Hq + g * G + head) * D + dcol), f);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) q2[h][i] = pack2(f[2 * i] * qscale, f[2 * i + 1] * qscale);
-    }
-    // running state: m, l of head oh (this lane's owned head); O rows of all heads
-    float m = -CUDART_INF_F, l = 0.f;
-    uint64_t o2[G][4];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o2[h][i] = 0ull;
-
+  } else {
+    // ------------------------------------------------------------ softmax group
+    const int row = threadIdx.x;                             // key row of S^T, dimension of O^T
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tO = tmem + lane_off + 32;
+    const float sl2 = a.scale * 1.4426950408889634f;
+    // this thread's P^T entries: row h, key `row` (128-byte swizzle: 16-byte chunk XOR row)
+    const uint32_t pt_base = (uint32_t)((row >> 6) * QSLAB + (row & 7) * 2);
+    const int kc = (row & 63) >> 3;
+    uint32_t tj = 0, nu = 0;
     bool ok = true;
-    for (int row = r0; row < r1 && ok; row += ROWS) {
-      const int s = cnt % NST;
-      const uint32_t ph = (cnt / NST) & 1u;
-      if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, kWaitDecodeFull, a.err)) { ok = false; break; }
-      const uint8_t* Ks = sm.stage[s];
-      const uint8_t* Vs = Ks + ROWS * D * 2;
-      // UPI passes per iteration: their reductions and broadcasts interleave
-#pragma unroll
-      for (int pass = 0; pass < ROWS / (2 * NCW); pass += UPI) {
-        int rr[UPI];
-        bool valid[UPI];
-        uint64_t x2[UPI][4];
-        float part[UPI][G];
-#pragma unroll
-        for (int u = 0; u < UPI; ++u) {
-          rr[u] = (pass + u) * 2 * NCW + cw * 2 + half;
-          valid[u] = row + rr[u] < r1;
-          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Ks + rr[u] * 256 + dcol * 2), x2[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < UPI; ++u)
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const uint64_t acc = ffma2(q2[h][1], x2[u][1], ffma2(q2[h][0], x2[u][0], 0ull));
-            part[u][h] = hsum2(ffma2(q2[h][3], x2[u][3], ffma2(q2[h][2], x2[u][2], acc)));
+    for (int u = blockIdx.x; u < geo.units; u += gridDim.x) {
+      const DecUnit U = dec_unit<kShard>(a, x, geo, u);
+      const int nvalid_chunk = chunk_rows<kShard>(a, x, geo.Cd, U.b, U.p);
+      const int n_live = (nvalid_chunk + RPS - 1) / RPS;
+      if (nvalid_chunk == 0) {
+        if (U.sub == 0) {
+          for (int e = row; e < G * D; e += CT) {
+            const int h = e / D, d = e - h * D;
+            a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * D + d] = 0.f;
           }
-#pragma unroll
-        for (int u = 0; u < UPI; ++u)
-          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(Vs + rr[u] * 256 + dcol * 2), x2[u]);
-        float sc[UPI];
-#pragma unroll
-        for (int u = 0; u < UPI; ++u) {
-          sc[u] = half_warp_transpose_sum<G>(part[u]);
-          if (!valid[u]) sc[u] = -CUDART_INF_F;
-        }
-        // online update with the UPI rows (the base moves at most once per iteration)
-        float smax = sc[0];
-#pragma unroll
-        for (int u = 1; u < UPI; ++u) smax = fmaxf(smax, sc[u]);
-        const bool moved = smax > m + LAZY;
-        if (__any_sync(0xffffffffu, moved)) {
-          float f = 1.f;
-          if (moved) {
-            f = (m == -CUDART_INF_F) ? 0.f : ex2(m - smax);
-            m = smax;
-            l *= f;
-          }
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float fh = __shfl_xor_sync(0xffffffffu, f, slot_xor<G>(h));
-            const uint64_t f2 = pack2(fh, fh);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) o2[h][i] = fmul2(o2[h][i], f2);
+          if (row < G) a.part_lse[(size_t)(U.b * a.Hq + U.g * G + row) * a.P + U.p] = -CUDART_INF_F;
+          if constexpr (kMerge) {
+            named_bar_sync(1, CT);   // the chunk's partial is written before it is counted
+            if (warp == 0) chunk_final_count<G>(a, x, U.b, U.g, lane);
           }
         }
-        const bool live = m != -CUDART_INF_F;
-        float pw[UPI];
+        continue;
+      }
+      if (U.ntiles == 0) continue;
+
+      // per head: base m (the same in every thread), fp32 sum l and bf16-value sum lt of this thread's rows
+      float m[G], l[G], lt[G];
 #pragma unroll
-        for (int u = 0; u < UPI; ++u) {
-          pw[u] = (valid[u] && live) ? ex2(sc[u] - m) : 0.f;
-          l += pw[u];
+      for (int h = 0; h < G; ++h) {
+        m[h] = -CUDART_INF_F;
+        l[h] = 0.f;
+        lt[h] = 0.f;
+      }
+      for (int j = 0; j < U.ntiles; ++j) {
+        const uint32_t t = tj + j, sb = t & 1u;
+        bool good = mbar_wait(smem_u32(&sm.s_full[sb]), (t >> 1) & 1u, abort_flag, kWaitSFull, err);
+        // P^T buffer sb is free once O^T has taken P^T(t - 2)
+        if (good && t >= 2) good = mbar_wait(smem_u32(&sm.o_done[sb]), ((t >> 1) - 1) & 1u, abort_flag, kWaitPFull, err);
+        if (named_bar_any(1, CT, !good || !ok)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        float xs[G];
+        tmem_ld_g<G>(tmem + lane_off + 16 * sb, xs);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sm.s_free[sb]));
+        const bool valid = U.r0 + j * BN + row < U.r1;
+        if (!valid) {
+          // a row past the valid ones (a cache's unwritten rows may hold any bits): its weight is 0,
+          // and its V row is zeroed so that the product never meets 0 x NaN
+          uint4* vr = reinterpret_cast<uint4*>(sm.kv[t % NST][1] + row * 128);
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) vr[sl * (SLAB / 16) + c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        bool exceed = false;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
+          xs[h] = valid ? xs[h] * sl2 : -CUDART_INF_F;
+          exceed |= xs[h] > m[h] + LAZY;
+        }
+        if (named_bar_any(1, CT, exceed)) {
+          // move the base of the heads whose tile maximum exceeds it (always on a unit's first tile)
+          const int rb = j & 1;   // reduction buffer: the next use is two barriers away
 #pragma unroll
-          for (int u = 0; u < UPI; ++u) {
-            const float pu = __shfl_xor_sync(0xffffffffu, pw[u], slot_xor<G>(h));
-            const uint64_t p2 = pack2(pu, pu);
+          for (int h = 0; h < G; ++h) {
+            const float mw = warp_max(xs[h]);
+            if (lane == 0) sm.red[rb][warp][h] = mw;
+          }
+          named_bar_sync(1, CT);
+          float alpha[G];
+          bool moved = false;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) o2[h][i] = ffma2(p2, x2[u][i], o2[h][i]);
+          for (int h = 0; h < G; ++h) {
+            float mt = sm.red[rb][0][h];
+#pragma unroll
+            for (int w = 1; w < NSW; ++w) mt = fmaxf(mt, sm.red[rb][w][h]);
+            alpha[h] = 1.f;
+            if (mt > m[h] + LAZY) {
+              alpha[h] = m[h] == -CUDART_INF_F ? 0.f : ex2(m[h] - mt);
+              m[h] = mt;
+              moved = true;
+            }
+            l[h] *= alpha[h];
+            lt[h] *= alpha[h];
+          }
+          if (j > 0 && moved) {   // the same decision in every thread (from the shared maxima)
+            // O^T holds this unit's earlier tiles: rescale its columns once O^T(t - 1) is complete
+            const uint32_t tp = t - 1;
+            if (!mbar_wait(smem_u32(&sm.o_done[tp & 1u]), (tp >> 1) & 1u, abort_flag, kWaitPFull, err)) ok = false;
+            __syncwarp();
+            tc_fence_after();
+            float o[G];
+            tmem_ld_g<G>(tO, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < G; ++h) o[h] *= alpha[h];
+            tmem_st_g<G>(tO, o);
+            tmem_wait_st();
+          }
+        }
+        // weights against the base; P^T(t) in shared memory for the tensor cores
+        uint8_t* ptb = sm.pt[sb];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float pw = m[h] == -CUDART_INF_F ? 0.f : ex2(xs[h] - m[h]);
+          const uint32_t bits = pack_bf16x2(pw, 0.f) & 0xffffu;
+          l[h] += pw;
+          lt[h] += __uint_as_float(bits << 16);
+          *reinterpret_cast<uint16_t*>(ptb + pt_base + (h >> 3) * 1024 + (h & 7) * 128 + ((kc ^ (h & 7)) << 4)) =
+              (uint16_t)bits;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sm.p_full[sb]));
+      }
+      if (!ok) break;
+      tj += U.ntiles;
+
+      // ---- the unit's result: O^T after its last product, sums reduced over the 128 threads
+      const bool fin = mbar_wait(smem_u32(&sm.o_full), nu & 1u, abort_flag, kWaitOFinal, err);
+      if (named_bar_any(1, CT, !fin)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float o[G];
+      tmem_ld_g<G>(tO, o);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.o_free));
+      ++nu;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float ls = warp_sum(l[h]), lts = warp_sum(lt[h]);
+        if (lane == 0) {
+          sm.red[0][warp][h] = ls;
+          sm.red[1][warp][h] = lts;
+        }
+      }
+      named_bar_sync(1, CT);
+      float* ws_unit = a.ws_part + ((((size_t)(U.b * a.Hkv + U.g) * a.P + U.p) * geo.nsub + U.sub) * G) * (D + 1);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float L = 0.f, LT = 0.f;
+#pragma unroll
+        for (int w = 0; w < NSW; ++w) {
+          L += sm.red[0][w][h];
+          LT += sm.red[1][w][h];
+        }
+        const float od = o[h] / LT;
+        const float lse = (m[h] + log2f(L)) * 0.6931471805599453f;
+        if (n_live == 1) {
+          a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * D + row] = od;
+          if (row == 0) a.part_lse[(size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p] = lse;
+        } else {
+          ws_unit[h * (D + 1) + row] = od;
+          if (row == 0) ws_unit[h * (D + 1) + D] = lse;
+        }
+      }
+      named_bar_sync(1, CT);   // sm.red is free again
+      if (n_live > 1) {
+        if (row == 0) {
+          unsigned int* ctr = a.ws_count + (size_t)(U.b * a.Hkv + U.g) * a.P + U.p;
+          const unsigned int old = atom_add_acq_rel_gpu(ctr, 1u);
+          const int last = (old == (unsigned int)(n_live - 1));
+          if (last) atomicExch(ctr, 0u);       // leave the counter at zero for the next call
+          sm.is_last = last;
+        }
+        named_bar_sync(1, CT);
+        if (sm.is_last) {
+          const float* ws_chunk = a.ws_part + (((size_t)(U.b * a.Hkv + U.g) * a.P + U.p) * geo.nsub) * G * (D + 1);
+          for (int e = row; e < G * D; e += CT) {
+            const int h = e / D, d = e - h * D;
+            float mx = -CUDART_INF_F;
+            for (int s2 = 0; s2 < n_live; ++s2) mx = fmaxf(mx, __ldcg(ws_chunk + (s2 * G + h) * (D + 1) + D));
+            float Lsum = 0.f, acc = 0.f;
+            for (int s2 = 0; s2 < n_live; ++s2) {
+              const float* r = ws_chunk + (s2 * G + h) * (D + 1);
+              const float w = expf(__ldcg(r + D) - mx);
+              Lsum += w;
+              acc = fmaf(w, __ldcg(r + d), acc);
+            }
+            a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * D + d] = acc / Lsum;
+            if (d == 0) a.part_lse[(size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p] = mx + logf(Lsum);
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));   // this warp is done with the stage
-      ++cnt;
+      // this CTA wrote the chunk's final partial: directly, or as the last sub-split to arrive
+      const bool chunk_final = n_live == 1 || sm.is_last;
+      if (named_bar_any(1, CT, !ok || *abort_flag)) break;
+      if constexpr (kMerge)
+        if (chunk_final && warp == 0) chunk_final_count<G>(a, x, U.b, U.g, lane);
     }
-    // (after an expired wait the unit still runs through every named barrier
-    // below, so that all consumer warps leave the loop together)
+  }
 
-    // fold the two half warps (same heads and dims, different rows)
-    {
-      const float mc = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-      const float f = (m == -CUDART_INF_F) ? 0.f : ex2(m - mc);
-      l *= f;
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
-      m = mc;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float fh = __shfl_xor_sync(0xffffffffu, f, slot_xor<G>(h));
-        const uint64_t f2 = pack2(fh, fh);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float x, y;
-          unpack2(fmul2(o2[h][i], f2), x, y);
-          x += __shfl_xor_sync(0xffffffffu, x, 16);
-          y += __shfl_xor_sync(0xffffffffu, y, 16);
-          o2[h][i] = pack2(x, y);
-        }
-      }
-    }
-    if (half == 0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const int head = head_of_slot<G>(lane, h);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          unpack2(o2[h][i], sm.wpart[cw][head][dcol + 2 * i], sm.wpart[cw][head][dcol + 2 * i + 1]);
-      }
-      if ((lane & 3) == 0) {
-        sm.wm[cw][oh] = m;
-        sm.wl[cw][oh] = l;
-      }
-    }
-    named_bar_sync(1, CT);
-
-    // fold the consumer warps: thread -> (head, dim) pairs; natural-log lse at the end
-    float* ws_unit = a.ws_part + ((((size_t)(b * a.Hkv + g) * a.P + p) * geo.nsub + sub) * G) * (D + 1);
-    for (int e = ctid; e < G * D; e += CT) {
-      const int h = e / D, d = e - h * D;
-      float mx = -CUDART_INF_F;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, sm.wm[w][h]);
-      float Lsum = 0.f, acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float f = (sm.wm[w][h] == -CUDART_INF_F) ? 0.f : ex2(sm.wm[w][h] - mx);
-        Lsum = fmaf(sm.wl[w][h], f, Lsum);
-        acc = fmaf(sm.wpart[w][h][d], f, acc);
-      }
-      const float od = acc / Lsum;
-      const float lse = (mx + log2f(Lsum)) * 0.6931471805599453f;
-      if (n_live == 1) {
-        a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = od;
-        if (d == 0) a.part_lse[(size_t)(b * a.Hq + g * G + h) * a.P + p] = lse;
-      } else {
-        ws_unit[h * (D + 1) + d] = od;
-        if (d == 0) ws_unit[h * (D + 1) + D] = lse;
-      }
-    }
-    if (n_live > 1) {
-      named_bar_sync(1, CT);
-      if (ctid == 0) {
-        unsigned int* ctr = a.ws_count + (size_t)(b * a.Hkv + g) * a.P + p;
-        const unsigned int old = atom_add_acq_rel_gpu(ctr, 1u);
-        const int last = (old == (unsigned int)(n_live - 1));
-        if (last) atomicExch(ctr, 0u);       // leave the counter at zero for the next call
-        sm.is_last = last;
-      }
-      named_bar_sync(1, CT);
-      if (sm.is_last) {
-        const float* ws_chunk = a.ws_part + (((size_t)(b * a.Hkv + g) * a.P + p) * geo.nsub) * G * (D + 1);
-        for (int e = ctid; e < G * D; e += CT) {
-          const int h = e / D, d = e - h * D;
-          float mx = -CUDART_INF_F;
-          for (int s2 = 0; s2 < n_live; ++s2) mx = fmaxf(mx, __ldcg(ws_chunk + (s2 * G + h) * (D + 1) + D));
-          float Lsum = 0.f, acc = 0.f;
-          for (int s2 = 0; s2 < n_live; ++s2) {
-            const float* r = ws_chunk + (s2 * G + h) * (D + 1);
-            const float w = expf(__ldcg(r + D) - mx);
-            Lsum += w;
-            acc = fmaf(w, __ldcg(r + d), acc);
-          }
-          a.partials[((size_t)(b * a.Hq + g * G + h) * a.P + p) * D + d] = acc / Lsum;
-          if (d == 0) a.part_lse[(size_t)(b * a.Hq + g * G + h) * a.P + p] = mx + logf(Lsum);
-        }
-      }
-    }
-    // this CTA wrote the chunk's final partial: directly, or as the last sub-split to arrive
-    const bool chunk_final = n_live == 1 || sm.is_last;
-    // shared fold buffers are free again; leave together if any wait expired
-    if (named_bar_any(1, CT, !ok || *abort_flag)) break;
-    if constexpr (kMerge)
-      if (chunk_final && cw == 0) chunk_final_count<G>(a, x, b, g, lane);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == NSW + 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -588,9 +701,11 @@ void decode_workspace_split(void* ws, int B, int Hq, int Hkv, int Smax, int D, i
 
 template <int G, bool kMerge, bool kShard>
 static cudaError_t launch_decode_g(const DecodeArgs& a, const DecodeExtra& x, cudaStream_t st) {
-  CUtensorMap tk, tv;
-  if (!make_tmap_bhsd(&tk, a.k, a.B, a.Smax, a.Hkv, a.D, dec::D, dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tmap_bhsd(&tv, a.v, a.B, a.Smax, a.Hkv, a.D, dec::D, dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+  CUtensorMap tq, tk, tv;
+  // q viewed as B*Hq rows of D; K, V as [B, Smax, Hkv, D]; 64-column boxes, 128-byte swizzle
+  if (!make_tmap_bhsd(&tq, a.q, 1, a.B * a.Hq, 1, a.D, 64, G, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_bhsd(&tk, a.k, a.B, a.Smax, a.Hkv, a.D, 64, dec::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_bhsd(&tv, a.v, a.B, a.Smax, a.Hkv, a.D, 64, dec::BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   DecGeom geo;
   geo.Cd = a.Smax / a.P;
@@ -603,13 +718,13 @@ static cudaError_t launch_decode_g(const DecodeArgs& a, const DecodeExtra& x, cu
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = num_sms();
-  kern<<<grid, dec::THREADS, smem, st>>>(tk, tv, a, geo, x);
+  kern<<<grid, dec::THREADS, smem, st>>>(tq, tk, tv, a, geo, x);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_partial(const DecodeArgs& a, const DecodeExtra& x, cudaStream_t st) {
   const int G = a.Hq / a.Hkv;
-  if (G != 1 && G != 2 && G != 4) return cudaErrorNotSupported;
+  if (!decode_group_supported(G)) return cudaErrorNotSupported;
   const int mode = (x.out != nullptr ? 2 : 0) + (x.shard_lens != nullptr ? 1 : 0);
   auto pick = [&](auto g) -> cudaError_t {
     constexpr int GG = decltype(g)::value;
@@ -620,9 +735,13 @@ cudaError_t launch_decode_partial(const DecodeArgs& a, const DecodeExtra& x, cud
       default: return launch_decode_g<GG, true, true>(a, x, st);
     }
   };
-  if (G == 1) return pick(std::integral_constant<int, 1>{});
-  if (G == 2) return pick(std::integral_constant<int, 2>{});
-  return pick(std::integral_constant<int, 4>{});
+  switch (G) {
+    case 1: return pick(std::integral_constant<int, 1>{});
+    case 2: return pick(std::integral_constant<int, 2>{});
+    case 4: return pick(std::integral_constant<int, 4>{});
+    case 8: return pick(std::integral_constant<int, 8>{});
+    default: return pick(std::integral_constant<int, 16>{});
+  }
 }
 
 }  // namespace ra
@@ -684,7 +803,7 @@ extern "C" ring_status ring_attn_decode_partial_noalloc(const void* q, const voi
   if ((long long)B * Smax * Hkv * D >= (1LL << 42)) return RING_EINVAL;
   if (dtype != RING_BF16 || D != 128) return RING_EUNSUPPORTED;
   const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4) return RING_EUNSUPPORTED;
+  if (!decode_group_supported(G)) return RING_EUNSUPPORTED;
   const size_t need = decode_workspace_bytes(B, Hq, Hkv, Smax, D, P);
   if (need == 0 || need > (size_t)RING_DECODE_NOALLOC_SCRATCH_BYTES) return RING_EINVAL;
   void* ws = nullptr;

@@ -84,6 +84,9 @@ struct DecodeExtra {
   float* out_lse;             // [B,Hq] or null (with out)
   unsigned int* ws_done;      // per-(b, kv head) finished-chunk counters (zero between calls)
 };
+// Query heads per kv head the decode kernel is built for (the heads are the N of
+// its tensor-core products, padded to 16).
+inline bool decode_group_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8 || G == 16; }
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P);
 void decode_workspace_split(void* ws, int B, int Hq, int Hkv, int Smax, int D, int P, float** part,
                             unsigned int** count, unsigned int** done);

@@ -133,7 +133,7 @@ def test_decode_and_merge_argument_checks():
     assert dec(ws=FAKE + 16) == ra.RING_EINVAL          # workspace must be 256-byte aligned
     assert dec(D=64) == ra.RING_EUNSUPPORTED
     assert dec(dtype=1) == ra.RING_EUNSUPPORTED
-    assert dec(Hq=64) == ra.RING_EUNSUPPORTED            # GQA group of 8 is not built
+    assert dec(Hq=24) == ra.RING_EUNSUPPORTED            # GQA group of 3 is not built (1, 2, 4, 8, 16 are)
     assert L.ring_attn_merge(FAKE, FAKE, None, None, 1, 1, 1, 128, 0, None) == ra.RING_EINVAL
     assert L.ring_attn_merge(FAKE, FAKE, FAKE, None, 1, 1, 1, 130, 0, None) == ra.RING_EUNSUPPORTED
     assert L.ring_attn_merge(FAKE, FAKE, FAKE, None, 1, 1, 0, 128, 0, None) == ra.RING_EINVAL

@@ -45,7 +45,7 @@ def make(B, Hq, Hkv, cap, lens, seed):
     return cfg, q, k, v, sl
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 2), (3, 3)])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 2), (3, 3), (16, 2), (32, 2)])   # G = 4, 2, 1, 8, 16
 def test_decode_small(Hq, Hkv):
     need_cuda()
     lens = [0, 1, 5000, 8192, 8193, 32768, 12345, 20000]

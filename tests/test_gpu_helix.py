@@ -111,6 +111,8 @@ def _fused_vs_oracle(q, k, v, sl, P, scale, lens):
     (8, 4, 12000, 3, (12000, 7777, 4032, 4033)),
     (2, 2, 4096, 1, (4096, 100)),
     (16, 4, 16384, 16, (16384, 3, 9000, 16383)),
+    (16, 2, 8192, 2, (8192, 4097, 130)),      # G = 8
+    (16, 1, 4096, 4, (4096, 1025)),           # G = 16
 ])
 def test_fused_decode_against_oracle_and_two_launch_path(Hq, Hkv, cap, P, lens):
     need_cuda()
