@@ -54,7 +54,7 @@ constexpr int D = 128;
 constexpr int BN = 128;                     // K/V rows per tile (the M of S^T)
 constexpr int NQ = 16;                      // query heads padded to the smallest N of the product
 constexpr int NST = 3;                      // K/V stages
-constexpr int RPS = 4096;                   // rows per sub-split (a multiple of BN)
+constexpr int RPS = 8192;                   // rows per sub-split (a multiple of BN)
 constexpr int SLAB = BN * 64 * 2;           // one 128-row x 64-column bf16 box (16 KB)
 constexpr int TILE_BYTES = BN * D * 2;      // one K or V tile (32 KB)
 constexpr int QSLAB = NQ * 128;             // 16 rows x 64 columns of bf16 (2 KB)

@@ -288,7 +288,7 @@ size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D,
  * held until the process exits.  Sizes whose scratch need
  * (ring_attn_decode_workspace_bytes) exceeds that maximum are rejected with
  * RING_EINVAL before anything is launched; the B8 Hq32 Hkv8 D128 2^20-token,
- * 32-chunk decode needs about 34 MB.  The first call on a device looks up the
+ * 32-chunk decode needs about 17 MB.  The first call on a device looks up the
  * array's device address (with that device current); make that first call
  * before any stream capture.  Each call clears the array's arrival counters
  * on `stream`, then launches the same kernel as ring_attn_decode_partial.

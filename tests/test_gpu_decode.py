@@ -82,6 +82,32 @@ def test_decode_small(Hq, Hkv):
     assert torch.equal(out2, out) and torch.equal(lse2, out_lse)
 
 
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_decode_ignores_rows_past_the_length(fused):
+    # A cache's rows past a sequence's length may hold anything (here NaN and Inf): they get
+    # weight 0 and must not reach the result (0 x NaN would).  The oracle reads valid rows only.
+    need_cuda()
+    lens = [1, 300, 4096, 4097, 6000, 8191]
+    cfg, q, k, v, sl = make(len(lens), 8, 2, 8192, lens, 83)
+    P = 2
+    kg, vg = k.clone(), v.clone()
+    for b, L in enumerate(lens):
+        kg[b, L:] = float("nan")
+        vg[b, L:] = float("inf") if b % 2 else float("nan")
+    ws = ra.decode_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.capacity, 128, P)
+    if fused:
+        out, out_lse = ra.ring_attn_decode_fused(q, kg, vg, P, seqlens=sl, scale=cfg.scale, workspace=ws)
+    else:
+        out, out_lse = ra.ring_attn_decode(q, kg, vg, sl, P, cfg.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    assert np.all(np.isfinite(host(out))) and np.all(np.isfinite(host(out_lse)))
+    ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale)
+    for (b, h), ro in ref_o.items():
+        assert abs(host(out_lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
+        assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+
 def test_merge_kernel_against_oracle_formula():
     need_cuda()
     g = torch.Generator(device="cuda").manual_seed(71)
