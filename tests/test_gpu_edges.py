@@ -67,7 +67,7 @@ def test_decode_lengths_out_of_range_are_clamped():
 
 @pytest.mark.parametrize("cap,P,lens", [
     (1000, 4, (1000, 251, 250, 1)),     # chunks of 250 rows: stage boxes straddle chunk ends
-    (8192, 1, (8192, 5000, 4032, 4033)),  # one chunk, split across sub-splits of the kernel
+    (20480, 1, (20480, 8192, 8193, 16385, 5000)),  # one chunk over 1, 2 or 3 of the kernel's 8192-row sub-splits
 ])
 def test_decode_partials_odd_chunks(cap, P, lens):
     need_cuda()

@@ -113,6 +113,7 @@ def _fused_vs_oracle(q, k, v, sl, P, scale, lens):
     (16, 4, 16384, 16, (16384, 3, 9000, 16383)),
     (16, 2, 8192, 2, (8192, 4097, 130)),      # G = 8
     (16, 1, 4096, 4, (4096, 1025)),           # G = 16
+    (8, 2, 24576, 1, (24576, 8193, 17000)),   # chunks over 3, 2, 3 sub-splits, folded before the merge
 ])
 def test_fused_decode_against_oracle_and_two_launch_path(Hq, Hkv, cap, P, lens):
     need_cuda()
