@@ -20,6 +20,9 @@
 //              rows stay zero), then K and V tiles into a 3-stage ring;
 //   warp 5     MMA issuer and tensor-memory owner: S(j+1) is issued before
 //              the O^T update of tile j, so the softmax of tile j+1 overlaps it.
+//   warp 6     merge warp (one-launch decode only): counts each chunk whose
+//              final partial this CTA wrote and merges on the count that
+//              completes the P chunks, off the softmax group's path.
 // The online softmax of "Lesson 8: Context Parallelism", section 3, with a
 // lazy base: a head's base moves only when one of its scores exceeds it by
 // more than 2^8 (a block-wide OR decides, and only then are the tile maxima
@@ -33,7 +36,8 @@
 // arrive (atomic counter, reset by that CTA) folds them into the chunk's
 // partial.  With an output buffer the merge runs in the same launch: the CTA
 // that finishes the last of the P chunks of a (sequence, kv head) -- a second
-// counter, reset the same way -- combines the P partials into out and lse.
+// counter, reset the same way -- combines the P partials into out and lse, in
+// its merge warp.
 // The valid rows of a chunk come from the sequence length (chunk p holds
 // positions [p*C, (p+1)*C)) or, for a cache filled by the round-robin append
 // of "NVIDIA unveils Helix Parallelism" (KV cache growth), from the chunk's
@@ -60,7 +64,7 @@ constexpr int TILE_BYTES = BN * D * 2;      // one K or V tile (32 KB)
 constexpr int QSLAB = NQ * 128;             // 16 rows x 64 columns of bf16 (2 KB)
 constexpr int NSW = 4;                      // softmax warps
 constexpr int CT = 32 * NSW;                // softmax threads
-constexpr int THREADS = CT + 64;            // + producer warp + MMA warp
+constexpr int THREADS = CT + 96;            // + producer warp + MMA warp + merge warp
 constexpr uint32_t TMEM_COLS = 64;          // S^T (2 x 16 columns), O^T (16 columns)
 constexpr float LAZY = 8.f;                 // log2 of the largest tolerated growth before rescaling
 static_assert(RPS % BN == 0, "tiles never straddle two sub-splits");
@@ -172,10 +176,9 @@ __device__ __noinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x,
     for (int k = 0; k < D / 32; ++k) out[(bh0 + h) * D + lane + 32 * k] = __float2bfloat16_rn(acc[h][k]);
 }
 
-// Called by softmax warp 0 (all lanes) after the CTA's writes of a chunk's
-// final partial and a softmax-group barrier: one lane counts the chunk; the warp
-// that completes the count of (b, g) merges it.  The other softmax warps do
-// not wait.
+// Called by the merge warp (all lanes) for a chunk whose final partial this CTA
+// wrote: one lane counts the chunk; the arrival that completes the count of
+// (b, g) merges it in this warp.  The softmax group does not wait.
 template <int G>
 __device__ __forceinline__ void chunk_final_count(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
   int last = 0;
@@ -196,6 +199,9 @@ struct DecSmem {
   alignas(8) uint64_t q_full[2], q_empty[2];
   alignas(8) uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   alignas(8) uint64_t o_full, o_free, teardown;
+  // finished chunks handed from the softmax group to the merge warp (kMerge): a ring of 4 slots
+  int q_b[4], q_g[4];
+  alignas(8) uint64_t q_post[4], q_done[4];
   uint32_t tmem_base;
   int is_last;      // set by one thread between two softmax-group barriers, read by all after the second
   int abort_flag;
@@ -329,6 +335,10 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     mbar_init(smem_u32(&sm.o_full), 1);
     mbar_init(smem_u32(&sm.o_free), CT);
     mbar_init(smem_u32(&sm.teardown), 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&sm.q_post[i]), 1);
+      mbar_init(smem_u32(&sm.q_done[i]), 1);
+    }
     sm.abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -457,7 +467,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       mma_commit(smem_u32(&sm.teardown));
       mbar_wait(smem_u32(&sm.teardown), 0, nullptr, kWaitTeardown, err);
     }
-  } else {
+  } else if (warp < NSW) {
     // ------------------------------------------------------------ softmax group
     const int row = threadIdx.x;                             // key row of S^T, dimension of O^T
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
@@ -468,6 +478,19 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     const int kc = (row & 63) >> 3;
     uint32_t tj = 0, nu = 0;
     bool ok = true;
+    // kMerge: thread 0 hands each chunk whose final partial this CTA wrote (after the barrier
+    // that follows those writes) to the merge warp, which counts it and merges on the count
+    // that completes the P chunks; a sentinel (b = -1) ends the merge warp's loop
+    uint32_t nposted = 0;
+    auto post = [&](int b, int g) {
+      const uint32_t k = nposted & 3u;
+      if (nposted >= 4 && !mbar_wait(smem_u32(&sm.q_done[k]), ((nposted >> 2) - 1) & 1u, abort_flag, kWaitPFull, err))
+        return;
+      sm.q_b[k] = b;
+      sm.q_g[k] = g;
+      mbar_arrive(smem_u32(&sm.q_post[k]));
+      ++nposted;
+    };
     for (int u = blockIdx.x; u < geo.units; u += gridDim.x) {
       const DecUnit U = dec_unit<kShard>(a, x, geo, u);
       const int nvalid_chunk = chunk_rows<kShard>(a, x, geo.Cd, U.b, U.p);
@@ -481,7 +504,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
           if (row < G) a.part_lse[(size_t)(U.b * a.Hq + U.g * G + row) * a.P + U.p] = -CUDART_INF_F;
           if constexpr (kMerge) {
             named_bar_sync(1, CT);   // the chunk's partial is written before it is counted
-            if (warp == 0) chunk_final_count<G>(a, x, U.b, U.g, lane);
+            if (row == 0) post(U.b, U.g);
           }
         }
         continue;
@@ -658,7 +681,23 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       const bool chunk_final = n_live == 1 || sm.is_last;
       if (named_bar_any(1, CT, !ok || *abort_flag)) break;
       if constexpr (kMerge)
-        if (chunk_final && warp == 0) chunk_final_count<G>(a, x, U.b, U.g, lane);
+        if (chunk_final && row == 0) post(U.b, U.g);
+    }
+    if constexpr (kMerge)
+      if (row == 0) post(-1, 0);
+  } else if (warp == NSW + 2) {
+    // ------------------------------------------------------------ merge warp (kMerge)
+    if constexpr (kMerge) {
+      for (uint32_t n = 0;; ++n) {
+        const uint32_t k = n & 3u;
+        const bool got = mbar_wait(smem_u32(&sm.q_post[k]), (n >> 2) & 1u, abort_flag, kWaitPFull, err);
+        if (!__all_sync(0xffffffffu, got)) break;
+        const int b = sm.q_b[k], g = sm.q_g[k];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.q_done[k]));   // the slot is free again
+        if (b < 0) break;
+        chunk_final_count<G>(a, x, b, g, lane);
+      }
     }
   }
 
