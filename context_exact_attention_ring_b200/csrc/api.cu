@@ -182,7 +182,7 @@ ring_status decode_args(const void* q, const void* k, const void* v, const int32
   if (!good_scale(scale)) return RING_EINVAL;
   if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
   if ((long long)B * Smax * Hkv * D >= (1LL << 42)) return RING_EINVAL;
-  if (dtype != RING_BF16 || D != 128) return RING_EUNSUPPORTED;
+  if (dtype != RING_BF16 || (D != 64 && D != 128)) return RING_EUNSUPPORTED;
   const int G = Hq / Hkv;
   if (!decode_group_supported(G)) return RING_EUNSUPPORTED;
   const size_t need = decode_workspace_bytes(B, Hq, Hkv, Smax, D, P);

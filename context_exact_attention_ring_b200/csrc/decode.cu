@@ -54,13 +54,13 @@
 namespace ra {
 
 namespace dec {
-constexpr int D = 128;
+constexpr int DM = 128;                     // head dimensions a tile row holds (D = 64 uses the first half)
 constexpr int BN = 128;                     // K/V rows per tile (the M of S^T)
 constexpr int NQ = 16;                      // query heads padded to the smallest N of the product
 constexpr int NST = 3;                      // K/V stages
 constexpr int RPS = 8192;                   // rows per sub-split (a multiple of BN)
 constexpr int SLAB = BN * 64 * 2;           // one 128-row x 64-column bf16 box (16 KB)
-constexpr int TILE_BYTES = BN * D * 2;      // one K or V tile (32 KB)
+constexpr int TILE_BYTES = BN * DM * 2;     // one K or V tile (32 KB)
 constexpr int QSLAB = NQ * 128;             // 16 rows x 64 columns of bf16 (2 KB)
 constexpr int NSW = 4;                      // softmax warps
 constexpr int CT = 32 * NSW;                // softmax threads
@@ -110,9 +110,9 @@ __device__ __forceinline__ bool count_chunk(const DecodeArgs& a, const DecodeExt
 // visible here).  The update of "Lesson 8: Context Parallelism", section 3,
 // applied to whole partial states:
 //   lse = m* + ln sum_p e^(lse_p - m*),  out = sum_p e^(lse_p - lse) O_p.
-template <int G>
+template <int G, int DH>
 __device__ __noinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
-  constexpr int D = dec::D;
+  constexpr int D = DH;
   __syncwarp();   // lane 0's acquire covers the warp from here on
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(x.out);
   const size_t bh0 = (size_t)b * a.Hq + g * G;
@@ -179,13 +179,13 @@ __device__ __noinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x,
 // Called by the merge warp (all lanes) for a chunk whose final partial this CTA
 // wrote: one lane counts the chunk; the arrival that completes the count of
 // (b, g) merges it in this warp.  The softmax group does not wait.
-template <int G>
+template <int G, int DH>
 __device__ __forceinline__ void chunk_final_count(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
   int last = 0;
   if (lane == 0) last = count_chunk(a, x, b, g);
   if (__shfl_sync(0xffffffffu, last, 0)) {
     __syncwarp();   // lane 0's acquire covers the warp
-    merge_bg<G>(a, x, b, g, lane);
+    merge_bg<G, DH>(a, x, b, g, lane);
   }
 }
 
@@ -301,7 +301,7 @@ __device__ __forceinline__ DecUnit dec_unit(const DecodeArgs& a, const DecodeExt
 // kMerge: the launch also merges the partials (a.out != null); kShard: valid
 // rows come from per-chunk fill counts (a.shard_lens != null).  Separate
 // instantiations, so that the plain partial kernel carries none of their code.
-template <int G, bool kMerge, bool kShard>
+template <int G, int DH, bool kMerge, bool kShard>
 __global__ void __launch_bounds__(dec::THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, DecodeArgs a, DecGeom geo, DecodeExtra x) {
@@ -317,6 +317,14 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     uint4* z = reinterpret_cast<uint4*>(&sm.q[0][0]);
     constexpr int n16 = (int)((sizeof(sm.q) + sizeof(sm.pt)) / 16);
     for (int i = threadIdx.x; i < n16; i += THREADS) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (DH == 64) {
+      // D = 64: the V tiles' second 64-column block is the zero upper half of the M = 128
+      // product O^T += V^T P^T (never written by TMA)
+      for (int st = 0; st < NST; ++st) {
+        uint4* zv = reinterpret_cast<uint4*>(sm.kv[st][1] + SLAB);
+        for (int i = threadIdx.x; i < SLAB / 16; i += THREADS) zv[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
     fence_proxy_async_smem();
   }
   if (threadIdx.x == 0) {
@@ -371,8 +379,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
           break;
         }
         const uint32_t qf = smem_u32(&sm.q_full[qb]);
-        mbar_arrive_expect_tx(qf, G * D * 2);
-        for (int sl = 0; sl < 2; ++sl)
+        mbar_arrive_expect_tx(qf, G * DH * 2);
+        for (int sl = 0; sl < DH / 64; ++sl)
           tma_load_4d(smem_u32(sm.q[qb]) + sl * QSLAB, &tmQ, qf, sl * 64, 0, U.b * a.Hq + U.g * G, 0, pol_q);
         ++nq;
         for (int j = 0; j < U.ntiles; ++j) {
@@ -382,9 +390,9 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             break;
           }
           const uint32_t fb = smem_u32(&sm.kv_full[s]);
-          mbar_arrive_expect_tx(fb, 2 * TILE_BYTES);
+          mbar_arrive_expect_tx(fb, 2 * BN * DH * 2);
           const int row = U.r0 + j * BN;
-          for (int sl = 0; sl < 2; ++sl) {
+          for (int sl = 0; sl < DH / 64; ++sl) {
             tma_load_4d(smem_u32(sm.kv[s][0]) + sl * SLAB, &tmK, fb, sl * 64, U.g, row, U.b, pol_kv);
             tma_load_4d(smem_u32(sm.kv[s][1]) + sl * SLAB, &tmV, fb, sl * 64, U.g, row, U.b, pol_kv);
           }
@@ -402,7 +410,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     if (lane == 0) {
       const uint32_t tS[2] = {tmem, tmem + 16}, tO = tmem + 32;
       constexpr uint32_t idS = idesc_f16_ab(BN, NQ, false, false);   // S^T = K Q^T
-      constexpr uint32_t idPV = idesc_f16_ab(D, NQ, true, false);    // O^T += V^T P^T
+      constexpr uint32_t idPV = idesc_f16_ab(DM, NQ, true, false);   // O^T += V^T P^T (D = 64: upper half zero)
       uint32_t cnt = 0, nq = 0, tj = 0, nu = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < geo.units && ok; u += gridDim.x) {
@@ -428,7 +436,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             tc_fence_after();
             const uint64_t kdesc = sw128_desc(smem_u32(sm.kv[s][0]), 16, 1024);
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k)
+            for (int k = 0; k < DH / 16; ++k)
               mma_ss(tS[sb], kdesc + ((((k >> 2) * SLAB) + (k & 3) * 32) >> 4),
                      qdesc + ((((k >> 2) * QSLAB) + (k & 3) * 32) >> 4), idS, k > 0 ? 1u : 0u);
             mma_commit(smem_u32(&sm.s_full[sb]));
@@ -497,9 +505,9 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
       const int n_live = (nvalid_chunk + RPS - 1) / RPS;
       if (nvalid_chunk == 0) {
         if (U.sub == 0) {
-          for (int e = row; e < G * D; e += CT) {
-            const int h = e / D, d = e - h * D;
-            a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * D + d] = 0.f;
+          for (int e = row; e < G * DH; e += CT) {
+            const int h = e / DH, d = e - h * DH;
+            a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * DH + d] = 0.f;
           }
           if (row < G) a.part_lse[(size_t)(U.b * a.Hq + U.g * G + row) * a.P + U.p] = -CUDART_INF_F;
           if constexpr (kMerge) {
@@ -630,7 +638,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         }
       }
       named_bar_sync(1, CT);
-      float* ws_unit = a.ws_part + ((((size_t)(U.b * a.Hkv + U.g) * a.P + U.p) * geo.nsub + U.sub) * G) * (D + 1);
+      float* ws_unit = a.ws_part + ((((size_t)(U.b * a.Hkv + U.g) * a.P + U.p) * geo.nsub + U.sub) * G) * (DH + 1);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float L = 0.f, LT = 0.f;
@@ -641,12 +649,13 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         }
         const float od = o[h] / LT;
         const float lse = (m[h] + log2f(L)) * 0.6931471805599453f;
+        if (row >= DH) continue;   // D = 64: the upper half of O^T is padding
         if (n_live == 1) {
-          a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * D + row] = od;
+          a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * DH + row] = od;
           if (row == 0) a.part_lse[(size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p] = lse;
         } else {
-          ws_unit[h * (D + 1) + row] = od;
-          if (row == 0) ws_unit[h * (D + 1) + D] = lse;
+          ws_unit[h * (DH + 1) + row] = od;
+          if (row == 0) ws_unit[h * (DH + 1) + DH] = lse;
         }
       }
       named_bar_sync(1, CT);   // sm.red is free again
@@ -660,19 +669,19 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         }
         named_bar_sync(1, CT);
         if (sm.is_last) {
-          const float* ws_chunk = a.ws_part + (((size_t)(U.b * a.Hkv + U.g) * a.P + U.p) * geo.nsub) * G * (D + 1);
-          for (int e = row; e < G * D; e += CT) {
-            const int h = e / D, d = e - h * D;
+          const float* ws_chunk = a.ws_part + (((size_t)(U.b * a.Hkv + U.g) * a.P + U.p) * geo.nsub) * G * (DH + 1);
+          for (int e = row; e < G * DH; e += CT) {
+            const int h = e / DH, d = e - h * DH;
             float mx = -CUDART_INF_F;
-            for (int s2 = 0; s2 < n_live; ++s2) mx = fmaxf(mx, __ldcg(ws_chunk + (s2 * G + h) * (D + 1) + D));
+            for (int s2 = 0; s2 < n_live; ++s2) mx = fmaxf(mx, __ldcg(ws_chunk + (s2 * G + h) * (DH + 1) + DH));
             float Lsum = 0.f, acc = 0.f;
             for (int s2 = 0; s2 < n_live; ++s2) {
-              const float* r = ws_chunk + (s2 * G + h) * (D + 1);
-              const float w = expf(__ldcg(r + D) - mx);
+              const float* r = ws_chunk + (s2 * G + h) * (DH + 1);
+              const float w = expf(__ldcg(r + DH) - mx);
               Lsum += w;
               acc = fmaf(w, __ldcg(r + d), acc);
             }
-            a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * D + d] = acc / Lsum;
+            a.partials[((size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p) * DH + d] = acc / Lsum;
             if (d == 0) a.part_lse[(size_t)(U.b * a.Hq + U.g * G + h) * a.P + U.p] = mx + logf(Lsum);
           }
         }
@@ -696,7 +705,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.q_done[k]));   // the slot is free again
         if (b < 0) break;
-        chunk_final_count<G>(a, x, b, g, lane);
+        chunk_final_count<G, DH>(a, x, b, g, lane);
       }
     }
   }
@@ -738,7 +747,7 @@ void decode_workspace_split(void* ws, int B, int Hq, int Hkv, int Smax, int D, i
   *done = reinterpret_cast<unsigned int*>(base + b_part + b_count);
 }
 
-template <int G, bool kMerge, bool kShard>
+template <int G, int DH, bool kMerge, bool kShard>
 static cudaError_t launch_decode_g(const DecodeArgs& a, const DecodeExtra& x, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   // q viewed as B*Hq rows of D; K, V as [B, Smax, Hkv, D]; 64-column boxes, 128-byte swizzle
@@ -753,7 +762,7 @@ static cudaError_t launch_decode_g(const DecodeArgs& a, const DecodeExtra& x, cu
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
   geo.units = (int)units;
   const size_t smem = sizeof(DecSmem<G>) + 1024;
-  auto kern = decode_kernel<G, kMerge, kShard>;
+  auto kern = decode_kernel<G, DH, kMerge, kShard>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = num_sms();
@@ -765,14 +774,18 @@ cudaError_t launch_decode_partial(const DecodeArgs& a, const DecodeExtra& x, cud
   const int G = a.Hq / a.Hkv;
   if (!decode_group_supported(G)) return cudaErrorNotSupported;
   const int mode = (x.out != nullptr ? 2 : 0) + (x.shard_lens != nullptr ? 1 : 0);
-  auto pick = [&](auto g) -> cudaError_t {
-    constexpr int GG = decltype(g)::value;
+  auto pick_d = [&](auto g, auto d) -> cudaError_t {
+    constexpr int GG = decltype(g)::value, DD = decltype(d)::value;
     switch (mode) {
-      case 0: return launch_decode_g<GG, false, false>(a, x, st);
-      case 1: return launch_decode_g<GG, false, true>(a, x, st);
-      case 2: return launch_decode_g<GG, true, false>(a, x, st);
-      default: return launch_decode_g<GG, true, true>(a, x, st);
+      case 0: return launch_decode_g<GG, DD, false, false>(a, x, st);
+      case 1: return launch_decode_g<GG, DD, false, true>(a, x, st);
+      case 2: return launch_decode_g<GG, DD, true, false>(a, x, st);
+      default: return launch_decode_g<GG, DD, true, true>(a, x, st);
     }
+  };
+  auto pick = [&](auto g) -> cudaError_t {
+    if (a.D == 64) return pick_d(g, std::integral_constant<int, 64>{});
+    return pick_d(g, std::integral_constant<int, 128>{});
   };
   switch (G) {
     case 1: return pick(std::integral_constant<int, 1>{});
@@ -840,7 +853,7 @@ extern "C" ring_status ring_attn_decode_partial_noalloc(const void* q, const voi
   if (!(scale > 0.f) || scale != scale || scale == __builtin_huge_valf()) return RING_EINVAL;
   if (dtype != RING_BF16 && dtype != RING_FP32) return RING_EINVAL;
   if ((long long)B * Smax * Hkv * D >= (1LL << 42)) return RING_EINVAL;
-  if (dtype != RING_BF16 || D != 128) return RING_EUNSUPPORTED;
+  if (dtype != RING_BF16 || (D != 64 && D != 128)) return RING_EUNSUPPORTED;
   const int G = Hq / Hkv;
   if (!decode_group_supported(G)) return RING_EUNSUPPORTED;
   const size_t need = decode_workspace_bytes(B, Hq, Hkv, Smax, D, P);

@@ -260,8 +260,9 @@ ring_status ring_attn_step_bwd(const void* q_shard, const void* kchunk, const vo
  *
  * Returns RING_EINVAL for null/misaligned pointers, Smax % P != 0, shapes < 1,
  * Hq % Hkv != 0, workspace too small; RING_EUNSUPPORTED unless dtype ==
- * RING_BF16, D == 128 and Hq / Hkv is 1, 2, 4, 8 or 16 (the query heads of a
- * kv head are the columns of the kernel's tensor-core products, padded to 16);
+ * RING_BF16, D is 64 or 128 and Hq / Hkv is 1, 2, 4, 8 or 16 (the query heads
+ * of a kv head are the columns of the kernel's tensor-core products, padded to
+ * 16);
  * RING_ECUDA on launch failure.
  */
 ring_status ring_attn_decode_partial(const void* q, const void* k, const void* v,

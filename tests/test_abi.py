@@ -131,7 +131,7 @@ def test_decode_and_merge_argument_checks():
     assert dec(Smax=1000) == ra.RING_EINVAL
     assert dec(wsb=ws - 1) == ra.RING_EINVAL
     assert dec(ws=FAKE + 16) == ra.RING_EINVAL          # workspace must be 256-byte aligned
-    assert dec(D=64) == ra.RING_EUNSUPPORTED
+    assert dec(D=96) == ra.RING_EUNSUPPORTED             # head dimensions 64 and 128 are built
     assert dec(dtype=1) == ra.RING_EUNSUPPORTED
     assert dec(Hq=24) == ra.RING_EUNSUPPORTED            # GQA group of 3 is not built (1, 2, 4, 8, 16 are)
     assert L.ring_attn_merge(FAKE, FAKE, None, None, 1, 1, 1, 128, 0, None) == ra.RING_EINVAL

@@ -108,6 +108,27 @@ def test_decode_ignores_rows_past_the_length(fused):
         assert abs(host(out_lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
         assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
 
+
+@pytest.mark.parametrize("Hq,Hkv,P", [(8, 2, 3), (16, 2, 1)])
+@pytest.mark.parametrize("fused", [False, True])
+def test_decode_head_dim_64(Hq, Hkv, P, fused):
+    # D = 64: one 64-column block per K/V row; with P = 1 the 24576-row chunk spans 3 sub-splits
+    need_cuda()
+    lens = [1, 300, 8192, 8193, 20000, 24576]
+    cfg = W.Decode("d64", len(lens), Hq, Hkv, 64, 24576, P, 97, fixed_lens=tuple(lens))
+    q, k, v, sl = W.decode_inputs(cfg, "cuda")
+    ws = ra.decode_workspace(cfg.B, Hq, Hkv, cfg.capacity, 64, P)
+    if fused:
+        out, out_lse = ra.ring_attn_decode_fused(q, k, v, P, seqlens=sl, scale=cfg.scale, workspace=ws)
+    else:
+        out, out_lse = ra.ring_attn_decode(q, k, v, sl, P, cfg.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale)
+    for (b, h), ro in ref_o.items():
+        assert abs(host(out_lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
+        assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+
 def test_merge_kernel_against_oracle_formula():
     need_cuda()
     g = torch.Generator(device="cuda").manual_seed(71)
