@@ -407,7 +407,7 @@ def run_ours(args):
                    "ms_per_step": round(dec_avg, 3), "bytes_per_step": dbytes,
                    "roofline": {"bound": "hbm", "achieved": round(achieved_gb, 1), "peak": pk["hbm_gbs"],
                                 "unit": "GB/s", "frac": round(achieved_gb / pk["hbm_gbs"], 4),
-                                "traffic": traffic.get("decode"), "kernel": "decode_kernel<4> + merge_kernel",
+                                "traffic": traffic.get("decode"), "kernel": "decode_kernel<4, 128> + merge_kernel",
                                 "peak_kind": f"{pk_kind} HBM copy"}},
         "prefill_ms_per_step": round(pre_avg, 3),
         "e2e": e2e,
