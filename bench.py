@@ -16,7 +16,7 @@ timed as the max over ranks.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
-same workload (the reference arm of this build).
+same workload, on the host cores, with the same metric and config.
 """
 from __future__ import annotations
 
