@@ -8,7 +8,8 @@ the next one is arriving from rank r-1 (a double buffer: the transfer of the
 next block overlaps the step).  Blocks land in this GPU's own memory before a
 kernel reads them: every kernel reads local memory only.  The backward runs
 the same loop with ring_attn_step_bwd; the dK, dV sums of a block travel with
-it and take one last hop home.
+it and take one last hop home.  helix_decode is the decode's
+exchange: per-shard partials, one all-gather, and the merge on every rank.
 
 The chunk ownership follows the splits of ring_attn_fwd (see split_chunks);
 the step functions default to this package's kernels and can be replaced
@@ -135,3 +136,36 @@ def ring_backward(q_shard, k_block, v_block, out_shard, lse_shard, dout_shard, l
             if t < P - 1:
                 kv, kv_nxt = kv_nxt, kv
     return dq.to(q_shard.dtype), gr[0].to(k_block.dtype), gr[1].to(v_block.dtype)
+
+
+def helix_decode(q, k_shard, v_shard, shard_len, scale=None, group=None, partial=None, merge=None):
+    """Split-KV single-token decode across GPUs ("NVIDIA unveils Helix
+    Parallelism", Phase 1, KV parallelism): rank r holds shard r of every
+    sequence's KV cache and computes, over its shard, the normalised partial
+    (O_r, lse_r) of every query head; the ranks exchange the partials with one
+    all-gather of B*Hq*(D+1) floats each, and every rank merges them with the
+    section-3 update of "Lesson 8" applied to whole partial states:
+        lse = m* + ln sum_r e^(lse_r - m*),  out = sum_r e^(lse_r - lse) O_r.
+
+    q [B, Hq, D] (the same on every rank); k_shard, v_shard [B, C, Hkv, D]
+    with the first shard_len[b] rows of sequence b valid (int32 [B], e.g. the
+    fill counts of ring_attn_kv_append); an empty shard gives lse_r = -inf and
+    O_r = 0.  Returns (out [B, Hq, D], lse [B, Hq]), the same on every rank.
+    The step functions default to this package's kernels (the decode over one
+    chunk, and the merge) and can be replaced (tests run the exchange on CPU
+    ranks with stand-ins)."""
+    from . import ring_attn_decode_partial, ring_attn_merge
+    if partial is None:
+        def partial(q_, k_, v_, lens_, scale_):
+            return ring_attn_decode_partial(q_, k_, v_, lens_, 1, scale_)
+    if merge is None:
+        def merge(parts_, lses_):
+            return ring_attn_merge(parts_, lses_, dtype=q.dtype)
+    world = dist.get_world_size(group)
+    part, plse = partial(q, k_shard, v_shard, shard_len, scale)          # [B, Hq, 1, D], [B, Hq, 1]
+    B, Hq, D = part.shape[0], part.shape[1], part.shape[-1]
+    mine = torch.cat([part.reshape(B, Hq, D), plse.reshape(B, Hq, 1)], dim=-1).contiguous()
+    gathered = [torch.empty_like(mine) for _ in range(world)]
+    dist.all_gather(gathered, mine, group=group)
+    allp = torch.stack(gathered, dim=2)                                   # [B, Hq, P, D + 1]
+    return merge(allp[..., :D].contiguous(), allp[..., D].contiguous())
