@@ -109,6 +109,62 @@ def test_helix_exchange_on_cpu_ranks(world):
                 np.testing.assert_allclose(lse[b, g * G:(g + 1) * G], rl, atol=1e-12, rtol=0)
 
 
+
+def _rank_round_robin(rank, world, block, port, q_out):
+    # every sequence's tokens dealt to the ranks block by block, as ring_attn_kv_append places
+    # them ("NVIDIA unveils Helix Parallelism", KV cache growth; oracle.helix simulates it)
+    from oracle import helix
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        q, k, v, lens = _inputs(world, seed=43)
+        cap = k.shape[1]
+        ks = np.zeros((B, cap, HKV, D), np.float32)
+        vs = np.zeros_like(ks)
+        shard_len = np.zeros(B, np.int32)
+        for b in range(B):
+            shards, _, _, dropped = helix.simulate_appends([[] for _ in range(world)], 0, list(range(lens[b])),
+                                                           block, world, cap)
+            assert dropped == 0
+            mine = shards[rank]
+            ks[b, :len(mine)] = k[b, mine]
+            vs[b, :len(mine)] = v[b, mine]
+            shard_len[b] = len(mine)
+        out, lse = R.helix_decode(torch.from_numpy(q), torch.from_numpy(ks), torch.from_numpy(vs),
+                                  torch.from_numpy(shard_len), scale=0.3, partial=fake_partial, merge=fake_merge)
+        q_out.put((rank, out.numpy(), lse.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,block", [(2, 4), (3, 1), (4, 8)])
+def test_helix_exchange_over_round_robin_shards(world, block):
+    # a single query attends to the union of the shards in any order: the exchange over
+    # round-robin shards equals attention over every token of the sequence
+    import oracle
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_round_robin, args=(r, world, block, port, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [qq.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    q, k, v, lens = _inputs(world, seed=43)
+    G = HQ // HKV
+    for b in range(B):
+        for g in range(HKV):
+            rows = [(0, i, 0) for i in range(G)]
+            ro, rl = oracle.attention_rows(q[b:b + 1, None, g * G:(g + 1) * G], k[b:b + 1, :, g:g + 1],
+                                           v[b:b + 1, :, g:g + 1], rows, scale=0.3, causal=False,
+                                           kv_len=np.array([lens[b]]))
+            for rank, out, lse in res:
+                np.testing.assert_allclose(out[b, g * G:(g + 1) * G], ro, atol=1e-12, rtol=0)
+                np.testing.assert_allclose(lse[b, g * G:(g + 1) * G], rl, atol=1e-12, rtol=0)
+
 def _gpu_rank(port, q_out):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
