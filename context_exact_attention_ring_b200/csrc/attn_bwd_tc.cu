@@ -6,35 +6,40 @@
 // with P recomputed tile by tile from the forward's lse.  Two launches of one
 // kernel template, neither with atomics:
 //   kKvMajor = true   a work item is a 128-key K/V tile of one kv head; its
-//                     steps are the 128-row query tiles (of every query head
+//                     steps are the 64-row query tiles (of every query head
 //                     of the group) that the block meets as it travels round
 //                     the ring ("Lesson 8: Context Parallelism", section 2):
 //                       T1 = K Q^T, T2 = V dO^T      (SS: K, V, Q, dO in smem)
 //                       P^T, dS^T from T1, T2          (two elementwise groups)
 //                       dV += P^T dO, dK += dS^T Q    (TS: P^T, dS^T in tmem)
 //   kKvMajor = false  a work item is a 128-row query tile of one head; its
-//                     steps are the K/V tiles in the rank's ring order:
+//                     steps are the 128-key K/V tiles in the rank's ring order:
 //                       T1 = Q K^T, T2 = dO V^T,  dS from T1, T2,
 //                       dQ += dS K                    (TS)
-// Every MMA is 128 x 128 (x 16), the shapes of the forward kernel; the
-// shared-memory tiles are the forward's 128-row, 128-byte-swizzled boxes,
-// read K-major by the SS products and MN-major by the TS products.
+// Every product has M = 128: the K/V-major launch's T1, T2 are 128 x 64 (64
+// query rows per step), every other product 128 x 128 or 128 x D.  The
+// shared-memory tiles are the forward's 128-byte-swizzled boxes, read K-major
+// by the SS products and MN-major by the TS products.
 //
-// Each step covers 64 query rows (K/V-major) or 64 keys (Q-major), so tensor
-// memory holds two T1/T2 pairs beside the accumulators and the two
-// elementwise groups ping-pong: while one turns its pair into P / dS, the
-// tensor cores accumulate the other's and compute the next pair
-// (issue order T(0) T(1) | TS(0) T(2) | TS(1) T(3) | ...), as the forward
-// kernel does with its two query tiles.
+// K/V-major: each step covers 64 query rows, so tensor memory holds two T1/T2
+// pairs beside dK and dV, and the two elementwise groups ping-pong: while one
+// turns its pair into P / dS, the tensor cores accumulate the other's and
+// compute the next pair (issue order T(0) T(1) | TS(0) T(2) | TS(1) T(3) | ...),
+// as the forward kernel does with its two query tiles.
+// Q-major: each step covers 128 keys and both groups work on it (group g on the
+// columns [64g, 64g + 64)).  Three 128-column regions rotate between S and dP
+// beside dQ, so S(i+1), dP(i+1) and S(i+2) are computed around the
+// elementwise pass of step i.
 //
 // Warp roles (12 warps): warp 0 TMA producer (the whole warp also stages the
 // step's lse and delta in the K/V-major kernel), warp 1 MMA issuer and
-// tensor-memory owner, warps 4-7 and 8-11 the two elementwise groups (group
-// g takes the steps i with i % 2 == g of every item; thread t owns row t of
-// its T1/T2 pair).  Tensor memory (512 columns): T1 pair [0,64) [64,128),
-// T2 pair [128,192) [192,256), accumulators [256, 256 + 2D); the bf16 P / dS
-// of a step overwrite the first 32 columns of its T1 / T2 once read.  Every
-// wait is bounded (as in the forward kernel).
+// tensor-memory owner, warps 4-7 and 8-11 the two elementwise groups (K/V-major:
+// group g takes the steps i with i % 2 == g of every item; thread t owns row t
+// of its tiles).  Tensor memory (512 columns): K/V-major: T1 pair [0,64)
+// [64,128), T2 pair [128,192) [192,256), dK, dV [256, 256 + 2D); Q-major:
+// regions [0,128) [128,256) [384,512) and dQ [256, 256 + D).  The bf16 P / dS of
+// a step overwrite the first 32 columns of the group's part of T1 / T2 once
+// read.  Every wait is bounded (as in the forward kernel).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
