@@ -201,3 +201,71 @@ def test_ring_loop_one_gpu_rank_runs_the_kernels():
     # one rank: the loop is one step of the tensor-core step kernel against the fused ring kernel
     assert errs[0] <= 2e-2 and errs[1] <= 1e-3
     assert max(errs[2:]) <= 3e-2
+
+
+
+def _rank_fails(rank, world, port, fail_rank, fail_step, q_out):
+    # a rank whose step raises part-way round the ring; the process group has a short timeout, so
+    # a rank that waits on it for a block must end with an error instead of waiting for good
+    import time
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    B, S, Hq, Hkv, D = 1, 16 * world, 2, 1, 8
+    q, k, v, _ = _inputs(B, S, Hq, Hkv, D, 22)
+    rows = R.shard_rows(S, world, "zigzag", rank).numpy()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows]))
+    calls = [0]
+
+    def step(*args, **kw):
+        if rank == fail_rank and calls[0] == fail_step:
+            raise RuntimeError("planted failure in the step")
+        calls[0] += 1
+        return fake_step(*args, **kw)
+
+    t0 = time.monotonic()
+    try:
+        out, lse = R.ring_forward(t(q), t(k), t(v), layout="zigzag", causal=True, scale=0.4, step=step,
+                                  new_state=fake_new_state, finalize=fake_finalize)
+        q_out.put((rank, None, time.monotonic() - t0, rows, out.numpy(), lse.numpy()))
+    except Exception as e:                                    # noqa: BLE001 -- any error ends the rank
+        q_out.put((rank, f"{type(e).__name__}: {e}"[:200], time.monotonic() - t0, rows, None, None))
+    # no destroy_process_group: a peer may be gone, and the process exits here
+
+
+@pytest.mark.parametrize("world,fail_rank,fail_step", [(3, 1, 0), (4, 3, 1), (4, 0, 0), (2, 0, 0), (3, 2, 2)])
+def test_a_rank_failing_mid_ring_never_leaves_the_others_waiting(world, fail_rank, fail_step):
+    # Rank f posts the send of the block it holds at step t before running that step, so when its
+    # step t raises, rank f+1 still gets that block (its step t+1) but never the next one (its step
+    # t+2): rank f+1 must end with an error when t + 2 <= P - 1.  Every other rank either ends with
+    # an error or finishes with the exact result; none waits past the process group's timeout.
+    import oracle
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_fails, args=(r, world, port, fail_rank, fail_step, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((qq.get(timeout=90) for _ in range(world)), key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(30)
+            if p.is_alive():
+                p.kill()                      # this test's own child, by its handle
+                p.join(10)
+    B, S, Hq, Hkv, D = 1, 16 * world, 2, 1, 8
+    q, k, v, _ = _inputs(B, S, Hq, Hkv, D, 22)
+    ro, rl = oracle.attention_rows(q, k, v, oracle.all_rows(B, Hq, S), scale=0.4, causal=True)
+    ro = ro.reshape(B, Hq, S, D).transpose(0, 2, 1, 3)
+    rl = rl.reshape(B, Hq, S)
+    starved = (fail_rank + 1) % world if fail_step + 2 <= world - 1 else None
+    for rank, err, secs, rows, out, lse in res:
+        assert secs < 60, (rank, secs)
+        if rank == fail_rank:
+            assert err is not None and "planted failure" in err
+        elif rank == starved:
+            assert err is not None, f"rank {rank} finished without the block rank {fail_rank} never sent"
+        if err is None:
+            np.testing.assert_allclose(out, ro[:, rows], atol=1e-12, rtol=0)
+            np.testing.assert_allclose(lse, rl[:, :, rows], atol=1e-12, rtol=0)
