@@ -195,3 +195,54 @@ def test_helix_exchange_one_gpu_rank_runs_the_kernels():
     p.join(60)
     assert p.exitcode == 0
     assert max(errs) == 0.0, errs      # one rank: the same kernels on the same data
+
+
+def _rank_fails(rank, world, port, fail_rank, q_out):
+    # a rank whose partial raises before the exchange; the others wait in the all-gather, and must
+    # end with an error (its connection closes, or the process group's 5 s timeout runs out)
+    import time
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    q, k, v, lens = _inputs(world)
+    sl = slice(rank * C, (rank + 1) * C)
+    shard_len = torch.from_numpy(np.clip(lens - rank * C, 0, C).astype(np.int32))
+
+    def partial(*a):
+        if rank == fail_rank:
+            raise RuntimeError("planted failure in the partial")
+        return fake_partial(*a)
+
+    t0 = time.monotonic()
+    try:
+        R.helix_decode(torch.from_numpy(q), torch.from_numpy(np.ascontiguousarray(k[:, sl])),
+                       torch.from_numpy(np.ascontiguousarray(v[:, sl])), shard_len, scale=0.3,
+                       partial=partial, merge=fake_merge)
+        q_out.put((rank, None, time.monotonic() - t0))
+    except Exception as e:                                    # noqa: BLE001 -- any error ends the rank
+        q_out.put((rank, f"{type(e).__name__}: {e}"[:200], time.monotonic() - t0))
+    # no destroy_process_group: a peer is gone, and the process exits here
+
+
+@pytest.mark.parametrize("world,fail_rank", [(2, 1), (3, 0)])
+def test_a_rank_failing_before_the_exchange_ends_every_rank_with_an_error(world, fail_rank):
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_fails, args=(r, world, port, fail_rank, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted(qq.get(timeout=90) for _ in range(world))
+    finally:
+        for p in procs:
+            p.join(30)
+            if p.is_alive():
+                p.kill()                      # this test's own child, by its handle
+                p.join(10)
+    for rank, err, secs in res:
+        # nobody can merge without every shard's partial
+        assert err is not None, f"rank {rank} merged without rank {fail_rank}'s partial"
+        if rank == fail_rank:
+            assert "planted failure" in err
+        assert secs < 60, (rank, secs)
