@@ -134,6 +134,18 @@ def test_positions_select_the_same_keys_as_the_causal_rule():
     np.testing.assert_allclose(dq_part, a[0][:, 8:], atol=1e-13, rtol=0)
 
 
+
+def test_keys_moved_with_their_positions_give_the_same_gradients():
+    # the causal rule reads a key's position, not its row: permuting the key/value rows together
+    # with their positions leaves dq unchanged and permutes dk, dv the same way
+    q, k, v, dout = _inputs(1, 24, 4, 2, 8, 19)
+    perm = np.random.default_rng(20).permutation(24)
+    a = oracle.attention_bwd(q, k, v, dout, scale=0.5, causal=True)
+    b = oracle.attention_bwd(q, k[:, perm], v[:, perm], dout, scale=0.5, causal=True, kpos=perm)
+    np.testing.assert_allclose(b[0], a[0], atol=1e-13, rtol=0)
+    np.testing.assert_allclose(b[1], a[1][:, perm], atol=1e-13, rtol=0)
+    np.testing.assert_allclose(b[2], a[2][:, perm], atol=1e-13, rtol=0)
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_sampled_dq_rows_equal_the_full_backward(causal):
     # the row-at-a-time dq (for large problems) against the full backward pinned above

@@ -50,6 +50,9 @@ MUTATIONS = [
     ("query positions ignored", "attn_fp64.c",
      "const int64_t qp = J->qpos ? J->qpos[i] : i;\n  const int64_t nkeys",
      "const int64_t qp = i;\n  const int64_t nkeys", ATTN),
+    ("key positions ignored", "attn_fp64.c",
+     "const int64_t kp = J->kpos ? J->kpos[j] : j;\n    const int allowed",
+     "const int64_t kp = j;\n    const int allowed", ATTN),
     # attn_fp64.c, backward: the calculus of the same definition
     ("softmax derivative drops delta", "attn_fp64.c",
      "const double ds = p * (dp[j] - delta);", "const double ds = p * dp[j];", BWD),
@@ -62,6 +65,12 @@ MUTATIONS = [
      "            dqi[d] -= J->scale * ds * (double)kj[d];\n            dkj", BWD),
     ("backward causal rule drops the diagonal", "attn_fp64.c",
      "if (J->causal && kp > qp)", "if (J->causal && kp >= qp)", BWD),
+    ("backward ignores query positions", "attn_fp64.c",
+     "const int64_t qp = J->qpos ? J->qpos[i] : i;\n        double m",
+     "const int64_t qp = i;\n        double m", BWD),
+    ("backward ignores key positions", "attn_fp64.c",
+     "const int64_t kp = J->kpos ? J->kpos[j] : j;\n          if (J->causal",
+     "const int64_t kp = j;\n          if (J->causal", BWD),
     ("sampled dQ rows drop the diagonal key", "attn_fp64.c",
      "const int nj = J->causal ? i + 1 : J->S;", "const int nj = J->causal ? i : J->S;", BWD),
     ("sampled dQ rows drop delta", "attn_fp64.c",
