@@ -46,13 +46,12 @@
 
 #include "kernels.h"
 #include "ptx.cuh"
+#include "bwd_sched.h"
 #include "ring_sched.h"
 
 namespace ra {
 
 namespace tb {
-constexpr int BR = 128;                 // rows of an item tile (and of T1/T2)
-constexpr int BS = 64;                  // rows of a K/V-major step (query rows)
 constexpr int THREADS = 384;
 constexpr int SLAB = 128 * 64 * 2;      // one 128-row x 64-column bf16 box
 constexpr uint32_t TMEM_COLS = 512;
@@ -84,111 +83,6 @@ struct BwdTcParams {
   int items;
   unsigned int* err;
 };
-
-// ---------------------------------------------------------------- work items
-// K/V-major item: one 128-key tile of chunk slot ks, kv head g, batch b.
-struct KvItem {
-  int b, g, ks, k_off, nk, srank;
-};
-__device__ __forceinline__ KvItem kv_item(const Plan& p, int L) {
-  const int tpk = cdiv(p.C, tb::BR);
-  const int per_bg = p.nkc * tpk;
-  KvItem it;
-  const int bg = L / per_bg, r = L - bg * per_bg;
-  it.b = bg / p.Hkv;
-  it.g = bg - it.b * p.Hkv;
-  it.ks = r / tpk;
-  it.k_off = (r - it.ks * tpk) * tb::BR;
-  it.nk = imin(tb::BR, p.C - it.k_off);
-  it.srank = p.mode == kModeRing ? chunk_owner(p, it.ks) : 0;
-  return it;
-}
-
-// One step of a K/V-major item: a 64-row query tile of head h in chunk qs.
-struct QStep {
-  int h, qs, q_off, nq, q0, k0;
-};
-struct QStepIter {
-  int h, n, qt;
-};
-__device__ __forceinline__ bool qstep_next(const Plan& p, const KvItem& it, QStepIter& s, QStep& out) {
-  const int G = p.Hq / p.Hkv, tpq = cdiv(p.C, tb::BS);
-  while (s.h < G) {
-    if (s.n >= p.nqc) {
-      s.n = 0;
-      ++s.h;
-      continue;
-    }
-    if (s.qt >= tpq) {
-      s.qt = 0;
-      ++s.n;
-      continue;
-    }
-    // the block of rank srank meets ranks srank, srank+1, ... (ring mode); buffer order (step mode)
-    const int qs = p.mode == kModeRing ? rank_chunk(p, (it.srank + s.n / p.cpr) % p.P, s.n % p.cpr) : s.n;
-    const int qb = q_pos_base(p, qs);
-    const int k0 = kv_pos_base(p, q_gid(p, qs), it.ks) + it.k_off;
-    if (s.qt == 0 && p.causal) {
-      // tiles whose last query precedes the first key are never met: start at the first one that is
-      if (qb + p.C - 1 < k0) {
-        s.qt = tpq;
-        continue;
-      }
-      s.qt = imax(0, (k0 - qb + 1 + tb::BS - 1) / tb::BS - 1);
-    }
-    const int q_off = s.qt * tb::BS;
-    const int nq = imin(tb::BS, p.C - q_off);
-    const int q0 = qb + q_off;
-    ++s.qt;
-    if (p.causal && k0 > q0 + nq - 1) continue;   // every key after every query of the tile
-    out.h = it.g * G + s.h;
-    out.qs = qs;
-    out.q_off = q_off;
-    out.nq = nq;
-    out.q0 = q0;
-    out.k0 = k0;
-    return true;
-  }
-  return false;
-}
-
-__device__ __forceinline__ int qstep_count(const Plan& p, const KvItem& it) {
-  const int G = p.Hq / p.Hkv, tpq = cdiv(p.C, tb::BS);
-  int n = 0;
-  for (int c = 0; c < p.nqc; ++c) {
-    const int qs = p.mode == kModeRing ? rank_chunk(p, (it.srank + c / p.cpr) % p.P, c % p.cpr) : c;
-    const int qb = q_pos_base(p, qs);
-    const int k0 = kv_pos_base(p, q_gid(p, qs), it.ks) + it.k_off;
-    if (!p.causal) {
-      n += tpq;
-    } else if (qb + p.C - 1 >= k0) {
-      int t = imax(0, (k0 - qb + 1 + tb::BS - 1) / tb::BS - 1);
-      if (qb + imin((t + 1) * tb::BS, p.C) - 1 < k0) ++t;   // (defensive: the formula already lands here)
-      n += tpq - t;
-    }
-  }
-  return n * G;
-}
-
-// Q-major item: one 128-row query tile of head h (longest work first).
-struct QItem {
-  int b, h, g, qs, q_off, nq, q0;
-};
-__device__ __forceinline__ QItem q_item(const Plan& p, int L) {
-  const int tpq = cdiv(p.C, tb::BR);
-  const int per_bh = p.nqc * tpq;
-  QItem it;
-  const int bh = L / per_bh, r = L - bh * per_bh;
-  it.b = bh / p.Hq;
-  it.h = bh - it.b * p.Hq;
-  it.g = it.h / (p.Hq / p.Hkv);
-  const int k = r / tpq;
-  it.qs = q_slot_by_rank(p, k);
-  it.q_off = (tpq - 1 - (r - k * tpq)) * tb::BR;
-  it.nq = imin(tb::BR, p.C - it.q_off);
-  it.q0 = q_pos_base(p, it.qs) + it.q_off;
-  return it;
-}
 
 // TMA load of one ROWS-row tile (D/64 boxes of ROWS x 64, slab after slab) at
 // row x of chunk slot `slot`

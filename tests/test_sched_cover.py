@@ -1,15 +1,18 @@
-"""The prefill kernels' scheduler (csrc/ring_sched.h), walked on the host.
+"""The attention kernels' schedulers (csrc/ring_sched.h, csrc/bwd_sched.h),
+walked on the host.
 
-tests/sched_cover.cpp includes the scheduler header the kernels use, builds
-with g++ and walks every work item and K/V tile as the tensor-core kernel
-does.  For every split, rank count, chunk count, ragged chunk length, GQA
-grouping, tile shape and mask, it checks the following:
+tests/sched_cover.cpp includes the scheduler headers the kernels use, builds
+with g++ and walks every work item and step as the kernels do: the forward
+tensor-core kernel, and both launches of the tensor-core backward (K/V-major
+for dK and dV, Q-major for dQ).  For every split, rank count, chunk count,
+ragged chunk length, GQA grouping, tile shape and mask, it checks the
+following:
 - each pair the causal rule allows is computed exactly once, and no other
   pair is;
 - each output row has exactly one owner, so no two CTAs write the same row;
 - every index stays inside its buffer;
-- the tile count the MMA warp expects equals the tile count the producer
-  sends.
+- the step count the MMA warp expects equals the step count the producer
+  walks.
 This stands in on the CPU for the bounds and race checks a sanitizer would
 make on the GPU.
 """
@@ -31,15 +34,19 @@ def walker(tmp_path_factory):
                            os.path.join(HERE, "sched_cover.cpp")])
     lib = ctypes.CDLL(so)
     i, p = ctypes.c_int, ctypes.c_void_p
-    lib.sched_cover_ring.argtypes = [i] * 10 + [p, ctypes.c_char_p]
-    lib.sched_cover_step.argtypes = [i] * 5 + [p, i, p, i, i, i, i, p, ctypes.c_char_p]
+    lib.sched_cover_ring.argtypes = [i] * 11 + [p, ctypes.c_char_p]
+    lib.sched_cover_step.argtypes = [i] * 5 + [p, i, p, i, i, i, i, i, p, ctypes.c_char_p]
     return lib
 
 
-def _ring(lib, B, Hq, Hkv, S, P, layout, cpr, causal, BM=128, BN=128):
+FORWARD, BACKWARD_KV, BACKWARD_Q = 0, 1, 2
+
+
+def _ring(lib, B, Hq, Hkv, S, P, layout, cpr, causal, which=FORWARD, BM=128, BN=128):
     stats = np.zeros(3, np.int64)
     msg = ctypes.create_string_buffer(256)
-    rc = lib.sched_cover_ring(B, Hq, Hkv, S, P, LAYOUT[layout], cpr, int(causal), BM, BN, stats.ctypes.data, msg)
+    rc = lib.sched_cover_ring(B, Hq, Hkv, S, P, LAYOUT[layout], cpr, int(causal), which, BM, BN, stats.ctypes.data,
+                              msg)
     assert rc == 0, (rc, msg.value.decode())
     return stats
 
@@ -54,12 +61,13 @@ for layout, cprs in (("contiguous", (1, 2, 3)), ("zigzag", (2, 3, 4, 8)), ("stri
                 CASES.append((layout, cpr, P, C))
 
 
+@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("layout,cpr,P,C", CASES)
-def test_ring_mode_covers_each_allowed_pair_once(walker, layout, cpr, P, C, causal):
+def test_ring_mode_covers_each_allowed_pair_once(walker, layout, cpr, P, C, causal, which):
     S = P * cpr * C
     for Hq, Hkv in ((2, 1), (3, 3)):             # even group: head pairs; odd group: two row tiles per item
-        stats = _ring(walker, 1, Hq, Hkv, S, P, layout, cpr, causal)
+        stats = _ring(walker, 1, Hq, Hkv, S, P, layout, cpr, causal, which)
         allowed = S * (S + 1) // 2 if causal else S * S
         assert stats[2] == Hq * allowed
 
@@ -67,24 +75,32 @@ def test_ring_mode_covers_each_allowed_pair_once(walker, layout, cpr, P, C, caus
 @pytest.mark.parametrize("BM,BN", [(128, 128), (128, 64), (64, 128)])
 def test_tile_shapes_batches_and_gqa(walker, BM, BN):
     for (Hq, Hkv) in ((8, 2), (6, 3), (5, 1), (4, 4)):
-        _ring(walker, 2, Hq, Hkv, 4 * 2 * 200, 4, "zigzag", 2, True, BM, BN)
-        _ring(walker, 2, Hq, Hkv, 3 * 130, 3, "striped", 1, True, BM, BN)
+        _ring(walker, 2, Hq, Hkv, 4 * 2 * 200, 4, "zigzag", 2, True, FORWARD, BM, BN)
+        _ring(walker, 2, Hq, Hkv, 3 * 130, 3, "striped", 1, True, FORWARD, BM, BN)
 
 
-def _step(lib, C, qid, kid, stripes, causal, Hq=2, Hkv=1):
+def test_backward_batches_and_gqa(walker):
+    for which in (BACKWARD_KV, BACKWARD_Q):
+        for (Hq, Hkv) in ((8, 2), (6, 3), (5, 1)):
+            _ring(walker, 2, Hq, Hkv, 4 * 2 * 200, 4, "zigzag", 2, True, which)
+            _ring(walker, 2, Hq, Hkv, 3 * 130, 3, "striped", 1, True, which)
+
+
+def _step(lib, C, qid, kid, stripes, causal, Hq=2, Hkv=1, which=FORWARD):
     stats = np.zeros(3, np.int64)
     msg = ctypes.create_string_buffer(256)
     q = (ctypes.c_int * len(qid))(*qid)
     k = (ctypes.c_int * len(kid))(*kid)
     rc = lib.sched_cover_step(1, Hq, Hkv, C, len(qid), ctypes.cast(q, ctypes.c_void_p), len(kid),
-                              ctypes.cast(k, ctypes.c_void_p), stripes, int(causal), 128, 128, stats.ctypes.data,
-                              msg)
+                              ctypes.cast(k, ctypes.c_void_p), stripes, int(causal), which, 128, 128,
+                              stats.ctypes.data, msg)
     assert rc == 0, (rc, msg.value.decode())
     return stats
 
 
+@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q])
 @pytest.mark.parametrize("causal", [True, False])
-def test_step_mode_covers_each_allowed_pair_of_the_held_block_once(walker, causal):
+def test_step_mode_covers_each_allowed_pair_of_the_held_block_once(walker, causal, which):
     # every (query shard, held block) pair of a zig-zag ring with P = 4 (8 chunks), chunk length 200,
     # and shards given in either chunk order
     P = 4
@@ -92,18 +108,19 @@ def test_step_mode_covers_each_allowed_pair_of_the_held_block_once(walker, causa
     for r in range(P):
         for s in range(P):
             for q_ids in (own[r], own[r][::-1]):
-                st = _step(walker, 200, q_ids, own[s], 0, causal)
+                st = _step(walker, 200, q_ids, own[s], 0, causal, which=which)
                 qt = [c * 200 + x for c in q_ids for x in range(200)]
                 kt = [c * 200 + y for c in own[s] for y in range(200)]
                 expect = sum(1 for a in qt for b in kt if b <= a) if causal else len(qt) * len(kt)
                 assert st[2] == 2 * expect
 
 
-def test_step_mode_stripes(walker):
+@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q])
+def test_step_mode_stripes(walker, which):
     P, C = 5, 150
     for r in range(P):
         for s in range(P):
-            st = _step(walker, C, [r], [s], P, True, Hq=3, Hkv=3)
+            st = _step(walker, C, [r], [s], P, True, Hq=3, Hkv=3, which=which)
             expect = sum(1 for x in range(C) for y in range(C) if y * P + s <= x * P + r)
             assert st[2] == 3 * expect
 
@@ -115,8 +132,11 @@ def test_the_walk_catches_a_wrong_mask(walker, tmp_path):
     old = "if (it.kt >= tpc || (p.causal && pos0 > qhi)) {"
     assert src.count(old) == 1
     (tmp_path / "ring_sched.h").write_text(src.replace(old, "if (it.kt >= tpc || (p.causal && pos0 + BN > qhi)) {"))
+    csrc = os.path.join(HERE, "..", "context_exact_attention_ring_b200", "csrc")
+    (tmp_path / "bwd_sched.h").write_text(open(os.path.join(csrc, "bwd_sched.h")).read())
     cpp = open(os.path.join(HERE, "sched_cover.cpp")).read().replace(
-        '"../context_exact_attention_ring_b200/csrc/ring_sched.h"', '"ring_sched.h"')
+        '"../context_exact_attention_ring_b200/csrc/ring_sched.h"', '"ring_sched.h"').replace(
+        '"../context_exact_attention_ring_b200/csrc/bwd_sched.h"', '"bwd_sched.h"')
     (tmp_path / "sched_cover.cpp").write_text(cpp)
     so = str(tmp_path / "libbad.so")
     subprocess.check_call(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-o", so, str(tmp_path / "sched_cover.cpp")])
@@ -124,6 +144,29 @@ def test_the_walk_catches_a_wrong_mask(walker, tmp_path):
     bad.sched_cover_ring.argtypes = walker.sched_cover_ring.argtypes
     stats = np.zeros(3, np.int64)
     msg = ctypes.create_string_buffer(256)
-    rc = bad.sched_cover_ring(1, 2, 1, 4 * 2 * 200, 4, 1, 2, 1, 128, 128, stats.ctypes.data, msg)
+    rc = bad.sched_cover_ring(1, 2, 1, 4 * 2 * 200, 4, 1, 2, 1, FORWARD, 128, 128, stats.ctypes.data, msg)
     # skipping tiles that straddle the diagonal drops allowed pairs; the kv_count check sees it first
+    assert rc in (12, 14), (rc, msg.value)
+
+
+def test_the_walk_catches_a_wrong_backward_step_filter(walker, tmp_path):
+    # a copy of the backward's step walk that starts one query tile late under the causal rule
+    # misses the diagonal tiles' first rows: the walk must fail
+    csrc = os.path.join(HERE, "..", "context_exact_attention_ring_b200", "csrc")
+    src = open(os.path.join(csrc, "bwd_sched.h")).read()
+    old = "s.qt = imax(0, (k0 - qb + 1 + tb::BS - 1) / tb::BS - 1);"
+    assert src.count(old) == 1
+    (tmp_path / "bwd_sched.h").write_text(src.replace(old, "s.qt = imax(0, (k0 - qb + 1 + tb::BS - 1) / tb::BS);"))
+    (tmp_path / "ring_sched.h").write_text(open(os.path.join(csrc, "ring_sched.h")).read())
+    cpp = open(os.path.join(HERE, "sched_cover.cpp")).read().replace(
+        '"../context_exact_attention_ring_b200/csrc/ring_sched.h"', '"ring_sched.h"').replace(
+        '"../context_exact_attention_ring_b200/csrc/bwd_sched.h"', '"bwd_sched.h"')
+    (tmp_path / "sched_cover.cpp").write_text(cpp)
+    so = str(tmp_path / "libbad_bwd.so")
+    subprocess.check_call(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-o", so, str(tmp_path / "sched_cover.cpp")])
+    bad = ctypes.CDLL(so)
+    bad.sched_cover_ring.argtypes = walker.sched_cover_ring.argtypes
+    stats = np.zeros(3, np.int64)
+    msg = ctypes.create_string_buffer(256)
+    rc = bad.sched_cover_ring(1, 2, 1, 4 * 2 * 200, 4, 1, 2, 1, BACKWARD_KV, 128, 128, stats.ctypes.data, msg)
     assert rc in (12, 14), (rc, msg.value)
