@@ -160,3 +160,39 @@ def test_sched_stats_zigzag_closed_form():
         assert per == [2 * P + 1] * P
         per, *_ = ra.ring_attn_sched_stats(64 * P, P, True, "contiguous")
         assert per == [r + 1 for r in range(P)]
+
+
+def test_header_builds_as_c_and_cxx_and_links_every_symbol(tmp_path):
+    # a C99 program that includes the header, takes the address of every declared function (so
+    # the linker must resolve each against the library) and calls the host-only entry points
+    import subprocess
+    names = declared_functions()
+    lib_dir = os.path.dirname(ra.LIB_PATH)
+    src = tmp_path / "use_abi.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"ring_attn.h\"\n"
+        "typedef void (*fn_t)(void);\n"
+        "int main(void) {\n"
+        "  const fn_t fns[] = {" + ", ".join(f"(fn_t)&{n}" for n in names) + "};\n"
+        "  size_t i, n = sizeof(fns) / sizeof(fns[0]);\n"
+        "  int64_t per[4], f = 0, p = 0, s = 0;\n"
+        "  for (i = 0; i < n; ++i) if (!fns[i]) return 2;\n"
+        "  if (ring_attn_sched_stats(1024, 4, 1, RING_ZIGZAG, 128, 128, per, &f, &p, &s) != RING_OK) return 3;\n"
+        "  printf(\"%d|%d|%s|%lld|%lld|%lld|%lld\\n\", ring_attn_version(), ring_attn_built_arch(),\n"
+        "         ring_attn_strerror(RING_EINVAL), (long long)per[0], (long long)f, (long long)p, (long long)s);\n"
+        "  return 0;\n}\n")
+    exe = str(tmp_path / "use_abi")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                           os.path.join(ROOT, "include"), str(src), "-o", exe, "-L", lib_dir, "-lringattn_sm100a",
+                           f"-Wl,-rpath,{lib_dir}"])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    ver, arch, err, per0, f, p, s = out.stdout.strip().split("|")
+    assert int(arch) == 100 and int(ver) >= 1 and err == ra.strerror(ra.RING_EINVAL)
+    # zig-zag, S = 1024, P = 4, 128-token tiles: 8 tiles per side, 2P+1 = 9 pairs per rank
+    assert (int(per0), int(f), int(p), int(s)) == (9, 28, 8, 28)
+    # the same header as C++ (its extern "C" block)
+    cxx = tmp_path / "use_abi.cpp"
+    cxx.write_text("#include \"ring_attn.h\"\nint main() { return ring_attn_version() > 0 ? 0 : 1; }\n")
+    subprocess.check_call(["g++", "-std=c++11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                           os.path.join(ROOT, "include"), "-fsyntax-only", str(cxx)])
