@@ -269,3 +269,46 @@ def test_a_rank_failing_mid_ring_never_leaves_the_others_waiting(world, fail_ran
         if err is None:
             np.testing.assert_allclose(out, ro[:, rows], atol=1e-12, rtol=0)
             np.testing.assert_allclose(lse, rl[:, :, rows], atol=1e-12, rtol=0)
+
+
+def _rank_groups(rank, world, port, q_out):
+    # two rings on interleaved ranks, {0, 2} and {1, 3}: a ring's neighbours are found through the
+    # group's own rank order, so a block must go to global rank 2 from 0, never to 1
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        groups = [dist.new_group([0, 2]), dist.new_group([1, 3])]   # every rank creates both, in one order
+        mine = rank % 2
+        ring = R.Ring(groups[mine])
+        B, S, Hq, Hkv, D = 1, 64, 2, 1, 8
+        q, k, v, _ = _inputs(B, S, Hq, Hkv, D, 30 + mine)           # each ring its own problem
+        rows = R.shard_rows(S, 2, "zigzag", ring.rank).numpy()
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows]))
+        out, lse = R.ring_forward(t(q), t(k), t(v), layout="zigzag", causal=True, scale=0.4, ring=ring,
+                                  step=fake_step, new_state=fake_new_state, finalize=fake_finalize)
+        q_out.put((rank, mine, rows, out.numpy(), lse.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rings_on_process_subgroups():
+    import oracle
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_groups, args=(r, 4, port, qq)) for r in range(4)]
+    for p in procs:
+        p.start()
+    res = [qq.get(timeout=120) for _ in range(4)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    B, S, Hq, Hkv, D = 1, 64, 2, 1, 8
+    for rank, mine, rows, out, lse in res:
+        q, k, v, _ = _inputs(B, S, Hq, Hkv, D, 30 + mine)
+        ro, rl = oracle.attention_rows(q, k, v, oracle.all_rows(B, Hq, S), scale=0.4, causal=True)
+        ro = ro.reshape(B, Hq, S, D).transpose(0, 2, 1, 3)
+        rl = rl.reshape(B, Hq, S)
+        np.testing.assert_allclose(out, ro[:, rows], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(lse, rl[:, :, rows], atol=1e-12, rtol=0)
