@@ -92,3 +92,24 @@ def test_package_sources_never_reach_the_oracle():
                     if pat.search(line) and ("import" in line or "oracle/" in line or "oracle." in line):
                         hits.append(f"{os.path.relpath(path, PKG)}:{n}: {line.strip()}")
     assert not hits, "\n".join(hits)
+
+
+def test_bench_reaches_the_oracle_only_in_its_cpu_baseline():
+    # bench.py may run the oracle only for the timed CPU baseline (its cpu_baseline leg and the
+    # reference arm, which calls it); every import of oracle must sit inside that function
+    import ast
+    root = os.path.dirname(PKG)
+    tree = ast.parse(open(os.path.join(root, "bench.py"), encoding="utf-8").read())
+    owners = []
+
+    def visit(node, fn):
+        for child in ast.iter_child_nodes(node):
+            name = child.name if isinstance(child, (ast.FunctionDef, ast.AsyncFunctionDef)) else fn
+            if isinstance(child, ast.Import) and any(a.name.split(".")[0] == "oracle" for a in child.names):
+                owners.append(fn)
+            if isinstance(child, ast.ImportFrom) and (child.module or "").split(".")[0] == "oracle":
+                owners.append(fn)
+            visit(child, name)
+
+    visit(tree, None)
+    assert owners and set(owners) == {"cpu_baseline"}, owners
