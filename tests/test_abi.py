@@ -196,3 +196,70 @@ def test_header_builds_as_c_and_cxx_and_links_every_symbol(tmp_path):
     cxx.write_text("#include \"ring_attn.h\"\nint main() { return ring_attn_version() > 0 ? 0 : 1; }\n")
     subprocess.check_call(["g++", "-std=c++11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
                            os.path.join(ROOT, "include"), "-fsyntax-only", str(cxx)])
+
+
+def test_backward_argument_checks():
+    # every case fails a check before the first launch (the plan, then pointers, then the workspace)
+    L = ra.lib()
+    ws_need = L.ring_attn_bwd_workspace_bytes(1, 2, 256)
+    assert ws_need == 2048 and L.ring_attn_bwd_workspace_bytes(0, 2, 256) == 0
+
+    def bwd(fn=L.ring_attn_bwd, **kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, Hq=2, Hkv=2,
+                 S=256, D=64, P=4, causal=1, layout=0, scale=0.125, dtype=0, ws=FAKE * 16, wsb=ws_need)
+        a.update(kw)
+        return fn(a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"], a["dq"], a["dk"], a["dv"], a["B"], a["Hq"],
+                  a["Hkv"], a["S"], a["D"], a["P"], a["causal"], a["layout"], a["scale"], a["dtype"], a["ws"], a["wsb"],
+                  None)
+    for fn in (L.ring_attn_bwd, L.ring_attn_bwd_simt):
+        assert bwd(fn, dout=None) == ra.RING_EINVAL
+        assert bwd(fn, dq=FAKE + 8) == ra.RING_EINVAL
+        assert bwd(fn, ws=None) == ra.RING_EINVAL
+        assert bwd(fn, ws=FAKE + 16) == ra.RING_EINVAL          # 256-byte alignment
+        assert bwd(fn, wsb=ws_need - 1) == ra.RING_EINVAL
+        assert bwd(fn, S=250) == ra.RING_EINVAL
+        assert bwd(fn, Hq=3) == ra.RING_EINVAL
+        assert bwd(fn, D=96) == ra.RING_EUNSUPPORTED
+    assert L.ring_attn_bwd_delta(None, FAKE, FAKE, 1, 2, 256, 64, 0, None) == ra.RING_EINVAL
+    assert L.ring_attn_bwd_delta(FAKE, FAKE, FAKE, 0, 2, 256, 64, 0, None) == ra.RING_EINVAL
+    assert L.ring_attn_bwd_delta(FAKE, FAKE, FAKE, 1, 2, 256, 64, 5, None) == ra.RING_EINVAL
+    ids = ra.ChunkIds()
+    ids.n_q, ids.n_kv, ids.chunk_len, ids.causal = 1, 1, 64, 1
+    step = lambda i, dout=FAKE, D=64: L.ring_attn_step_bwd(FAKE, FAKE, FAKE, dout, FAKE, FAKE, FAKE, FAKE, FAKE, i, 1,
+                                                          2, 2, D, 0.125, 0, None)
+    assert step(None) == ra.RING_EINVAL
+    assert step(ctypes.byref(ids), dout=FAKE + 4) == ra.RING_EINVAL
+    assert step(ctypes.byref(ids), D=96) == ra.RING_EUNSUPPORTED
+
+
+def test_fused_decode_and_append_argument_checks():
+    L = ra.lib()
+    ws = ra.ring_attn_decode_workspace_bytes(2, 8, 2, 4096, 128, 4)
+
+    def fused(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, sl=FAKE, shard=None, part=FAKE, plse=FAKE, out=FAKE, olse=FAKE, B=2, Hq=8,
+                 Hkv=2, Smax=4096, D=128, P=4, scale=0.088, dtype=0, ws=FAKE * 16, wsb=ws)
+        a.update(kw)
+        return L.ring_attn_decode_fused(a["q"], a["k"], a["v"], a["sl"], a["shard"], a["part"], a["plse"], a["out"],
+                                        a["olse"], a["B"], a["Hq"], a["Hkv"], a["Smax"], a["D"], a["P"], a["scale"],
+                                        a["dtype"], a["ws"], a["wsb"], None)
+    assert fused(sl=None) == ra.RING_EINVAL                     # no source of lengths
+    assert fused(shard=FAKE) == ra.RING_EINVAL                  # two sources of lengths
+    assert fused(out=None) == ra.RING_EINVAL
+    assert fused(olse=FAKE + 2) == ra.RING_EINVAL
+    assert fused(wsb=ws - 1) == ra.RING_EINVAL
+    assert fused(Hq=6) == ra.RING_EUNSUPPORTED                  # GQA group of 3
+
+    def append(**kw):
+        a = dict(kc=FAKE, vc=FAKE, kn=FAKE, vn=FAKE, sl=FAKE, na=FAKE, B=2, T=3, Hkv=2, Smax=4096, D=128, P=4, block=16,
+                 dtype=0)
+        a.update(kw)
+        return L.ring_attn_kv_append(a["kc"], a["vc"], a["kn"], a["vn"], a["sl"], a["na"], a["B"], a["T"], a["Hkv"],
+                                     a["Smax"], a["D"], a["P"], a["block"], a["dtype"], None)
+    assert append(sl=None) == ra.RING_EINVAL
+    assert append(kn=FAKE + 8) == ra.RING_EINVAL
+    assert append(block=0) == ra.RING_EINVAL
+    assert append(Smax=4095) == ra.RING_EINVAL                  # Smax % P
+    assert append(T=0) == ra.RING_EINVAL
+    assert append(dtype=5) == ra.RING_EINVAL
+    assert append(Hkv=1, D=4) == ra.RING_EUNSUPPORTED           # a row of 8 bytes: rows move in 16-byte pieces
