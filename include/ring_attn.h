@@ -255,8 +255,11 @@ ring_status ring_attn_step_bwd(const void* q_shard, const void* kchunk, const vo
  * recombined with the same update; `workspace` (device, at least
  * ring_attn_decode_workspace_bytes(...) bytes, 256-byte aligned) holds those
  * sub-results and per-chunk arrival counters.  The counters must be zero
- * before the first call on a workspace; every call leaves them zero again.
- * Calls that share a workspace must not overlap on the GPU.
+ * before the first call on a workspace; every call that completes leaves them
+ * zero again.  A call cut short by an expired wait (ring_attn_device_error
+ * returns RING_ETIMEOUT) may leave them non-zero: zero the workspace again
+ * before its next use.  Calls that share a workspace must not overlap on the
+ * GPU.
  *
  * Returns RING_EINVAL for null/misaligned pointers, Smax % P != 0, shapes < 1,
  * Hq % Hkv != 0, workspace too small; RING_EUNSUPPORTED unless dtype ==
@@ -350,8 +353,9 @@ ring_status ring_attn_decode(const void* q, const void* k, const void* v, const 
  * out [B,Hq,D] bf16 and out_lse [B,Hq] float (may be NULL) the merged
  * result.  The workspace is ring_attn_decode_workspace_bytes(...) bytes,
  * 256-byte aligned; its counters must be zero before the first call on it and
- * every call leaves them zero.  Calls that share a workspace must not overlap
- * on the GPU.  Errors as ring_attn_decode_partial, plus RING_EINVAL unless
+ * every call that completes leaves them zero (after RING_ETIMEOUT, zero it
+ * again).  Calls that share a workspace must not overlap on the GPU.  Errors
+ * as ring_attn_decode_partial, plus RING_EINVAL unless
  * exactly one of seqlens / shard_lens is given, or for a null or misaligned
  * out.
  */
