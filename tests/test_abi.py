@@ -263,3 +263,26 @@ def test_fused_decode_and_append_argument_checks():
     assert append(T=0) == ra.RING_EINVAL
     assert append(dtype=5) == ra.RING_EINVAL
     assert append(Hkv=1, D=4) == ra.RING_EUNSUPPORTED           # a row of 8 bytes: rows move in 16-byte pieces
+
+
+def test_sched_stats_random_sweep_equals_oracle_enumeration():
+    # seeded random splits, rank counts, ragged chunk lengths and odd tile sizes
+    import numpy as np
+    rng = np.random.default_rng(77)
+    layouts = ["contiguous", "contiguous2", "contiguous3", "zigzag", "zigzag3", "zigzag4", "zigzag6", "striped"]
+    n = 0
+    while n < 60:
+        layout = layouts[rng.integers(len(layouts))]
+        P = int(rng.integers(1, 7))
+        k = sch.parse_layout(layout)[1]
+        C = int(rng.integers(1, 300))
+        S = P * k * C
+        if S > 3000:
+            continue
+        tq, tk = int(rng.choice([16, 32, 48, 64, 100, 128])), int(rng.choice([16, 32, 64, 96, 128]))
+        causal = bool(rng.integers(2))
+        per, full, partial, skipped = ra.ring_attn_sched_stats(S, P, causal, layout, tq, tk)
+        o_full, o_partial, o_skipped, _ = sch.tile_classes(S, P, layout, causal, tq, tk)
+        assert (full, partial, skipped) == (o_full, o_partial, o_skipped), (S, P, layout, causal, tq, tk)
+        assert per == sch.per_rank_pairs(P, layout, causal, S), (S, P, layout, causal)
+        n += 1
