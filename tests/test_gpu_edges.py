@@ -7,7 +7,6 @@ import pytest
 import torch
 
 import context_exact_attention_ring_b200 as ra
-import oracle
 import workloads as W
 from oracle import merge as omerge
 from tests.helpers import TOL_BF16_LSE, TOL_BF16_OUT, TOL_FP32, check_rows, host, need_cuda, oracle_rows

@@ -11,7 +11,7 @@ import torch
 import context_exact_attention_ring_b200 as ra
 import workloads as W
 from oracle import schedule as sch
-from tests.helpers import (TOL_BF16_LSE, TOL_BF16_OUT, TOL_FP32, check_rows, host, need_cuda, oracle_rows)
+from tests.helpers import (TOL_BF16_LSE, TOL_BF16_OUT, TOL_FP32, check_rows, need_cuda, oracle_rows)
 from tests.test_gpu_simt import ring_by_steps
 
 pytestmark = pytest.mark.gpu
