@@ -211,11 +211,6 @@ def tile_classes(S: int, P: int, layout: str, causal: bool, tile_q: int, tile_k:
     return full, partial, skipped, per_rank
 
 
-def rank_of_chunk(P: int, layout: str) -> dict[int, int]:
-    """Owner rank of each global chunk."""
-    return {c: r for r, cs in layout_assignment(P, layout).items() for c in cs}
-
-
 def kv_visit_order(P: int, layout: str, rank: int) -> list[int]:
     """Global K/V chunk indices in the order rank ``rank`` meets them during
     one ring loop (for zig-zag, both chunks of the source rank at each step,
