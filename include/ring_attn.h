@@ -20,7 +20,9 @@
  *
  * Conventions shared by every entry point.
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
- *     allocates no memory and keeps no state except one device error word.
+ *     allocates no memory and keeps no state except one device error word and
+ *     the fixed scratch array of ring_attn_decode_partial_noalloc (reserved
+ *     when the library is loaded; see that entry).
  *   - Row-major layouts, last index contiguous:
  *       q, out        [B, S, Hq, D]        k, v  [B, S, Hkv, D]
  *       lse           [B, Hq, S]  float, natural log: lse = m + ln l
