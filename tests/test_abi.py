@@ -286,3 +286,17 @@ def test_sched_stats_random_sweep_equals_oracle_enumeration():
         assert (full, partial, skipped) == (o_full, o_partial, o_skipped), (S, P, layout, causal, tq, tk)
         assert per == sch.per_rank_pairs(P, layout, causal, S), (S, P, layout, causal)
         n += 1
+
+
+def test_state_init_and_finalize_argument_checks():
+    L = ra.lib()
+    assert L.ring_attn_state_init(None, FAKE, FAKE, 1, 2, 64, 64, None) == ra.RING_EINVAL
+    assert L.ring_attn_state_init(FAKE, FAKE + 4, FAKE, 1, 2, 64, 64, None) == ra.RING_EINVAL
+    assert L.ring_attn_state_init(FAKE, FAKE, FAKE, 1, 2, 0, 64, None) == ra.RING_EINVAL
+    assert L.ring_attn_state_init(FAKE, FAKE, FAKE, 1, 2, 64, 66, None) == ra.RING_EINVAL    # D % 4
+    fin = lambda **kw: L.ring_attn_state_finalize(*[kw.get(n, FAKE) for n in ("m", "l", "O", "out", "lse")],
+                                                  kw.get("B", 1), 2, 64, 64, kw.get("dtype", 0), None)
+    assert fin(lse=None) == ra.RING_EINVAL
+    assert fin(out=FAKE + 2) == ra.RING_EINVAL
+    assert fin(B=0) == ra.RING_EINVAL
+    assert fin(dtype=3) == ra.RING_EINVAL
