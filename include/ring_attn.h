@@ -369,9 +369,9 @@ ring_status ring_attn_decode_fused(const void* q, const void* k, const void* v, 
 /*
  * ring_attn_kv_append -- append T new tokens per sequence to a KV cache
  * sharded over P KV-parallel ranks, round-robin by blocks ("NVIDIA unveils
- * Helix Parallelism", on growing the KV cache: the first block of new tokens
- * goes to rank 0, the next to rank 1, and so on, so that every rank's share
- * grows evenly).
+ * Helix Parallelism", on growing the KV cache: successive blocks of new
+ * tokens go to successive ranks, wrapping after the last, so every rank's
+ * share grows at the same pace).
  *
  * k_cache, v_cache [B,Smax,Hkv,D]: rank p's shard is rows [p*C, (p+1)*C),
  * C = Smax/P, of which the first shard_lens[b*P+p] are filled.  k_new, v_new

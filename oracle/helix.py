@@ -3,11 +3,12 @@
 TEST INFRASTRUCTURE (see the package docstring).
 
 Source: "NVIDIA unveils Helix Parallelism", on growing the KV cache during
-decoding: writing every new token to one GPU would make a memory hotspot, so
-new tokens are dealt out by blocks -- the first block to GPU 0, the next to
-GPU 1, and so on -- and every KV-parallel rank's share grows evenly.
+decoding.  To keep one GPU from becoming a memory hotspot, appended tokens
+are placed in blocks that rotate over the KV-parallel GPUs (block 0 on GPU 0,
+block 1 on GPU 1, continuing in turn), so every rank's share grows at the
+same pace.
 
-Reading: "and so on" wraps around after the last rank (block i goes to rank
+Reading: the rotation wraps after the last rank (block i goes to rank
 i mod P), a block is `block` consecutive appended tokens of one sequence, and
 inside a rank's shard tokens keep their arrival order.
 

@@ -2,8 +2,8 @@
 
 TEST INFRASTRUCTURE (see the package docstring).  Used only to pin that the
 blockwise recurrence reaches the plain definition computed by attn_fp64.c
-("numerically identical" after a full loop: "Sequence parallelism and ring
-attention", FAQ; "Lesson 8: Context Parallelism", section 3).
+(after a full loop the result is exact attention: "Sequence parallelism and
+ring attention", FAQ; "Lesson 8: Context Parallelism", section 3).
 
 The update follows "Lesson 8", section 3, in its notation: when a new K/V
 block arrives with scores S_new,

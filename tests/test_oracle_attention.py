@@ -9,7 +9,7 @@ Pins used, none of which re-types the oracle's own formula:
   * a library routine: torch's scaled_dot_product_attention in float64;
   * brute force: the numpy full-matrix oracle, written separately;
   * invariants: key permutation (non-causal), split / rotation independence of
-    the ring recurrence ("numerically identical": "Sequence parallelism and
+    the ring recurrence (exact after a full loop: "Sequence parallelism and
     ring attention", FAQ; "Lesson 8: Context Parallelism", section 3).
 """
 import itertools

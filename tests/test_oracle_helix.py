@@ -18,7 +18,7 @@ def test_printed_first_blocks(P, block):
     for blk, gpu in GOLD["printed_first_blocks"]:
         for n in range(blk * block, (blk + 1) * block):
             assert helix.append_rank(n, block, P) == gpu
-    # ... "and so on": after the last rank the deal starts again at rank 0
+    # the rotation continues past the last rank: the deal starts again at rank 0
     assert helix.append_rank(P * block, block, P) == 0
 
 
