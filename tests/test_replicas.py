@@ -61,3 +61,32 @@ def test_cpu_baseline_small_sample():
     cfg = W.Prefill("tiny", "bf16", True, "zigzag", 1, 2, 1, 512, 64, 2, 3)
     r = bench.cpu_baseline(cfg, seconds=0.2)
     assert r["kind"] == "oracle" and r["cores"] >= 1 and r["value"] > 0 and r["unit"] == "TFLOP/s"
+
+
+
+def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    # a copy of the kernel sources with traffic.json hashes matching them reports every kernel's
+    # bytes; changing one byte of one kernel's source turns that kernel's traffic into None
+    import hashlib
+    import json
+    import shutil
+    d = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for e in d.values():
+        if not isinstance(e, dict):
+            continue
+        m = hashlib.sha256()
+        for src in e["sources"]:
+            dst = tmp_path / src
+            dst.parent.mkdir(parents=True, exist_ok=True)
+            shutil.copy(os.path.join(bench.ROOT, src), dst)
+            m.update(dst.read_bytes())
+        e["source_sha256"] = m.hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(d))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    cur = bench.load_traffic()
+    assert cur["attn_tc"] == d["attn_tc"]["bytes"] and cur["decode"] == d["decode"]["bytes"]
+    f = tmp_path / "context_exact_attention_ring_b200" / "csrc" / "decode.cu"
+    f.write_text(f.read_text() + "\n")
+    changed = bench.load_traffic()
+    assert changed["decode"] is None and changed["attn_tc"] == cur["attn_tc"]
