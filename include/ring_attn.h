@@ -132,7 +132,8 @@ ring_status ring_attn_fwd_counted(const void* q, const void* k, const void* v, v
 /*
  * ring_attn_fwd_simt -- the same computation as ring_attn_fwd on CUDA cores
  * with float32 FMA for both dtypes (bf16 inputs are widened exactly).  Slow;
- * it exists to cross-check the tensor-core path on the GPU.
+ * it exists to cross-check the tensor-core path on the GPU.  Arguments and
+ * errors as ring_attn_fwd.
  */
 ring_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse,
                                int B, int Hq, int Hkv, int S, int D, int P, int causal, int layout,
@@ -141,7 +142,9 @@ ring_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void
 /*
  * ring_attn_state_init -- set a ring state to its starting value
  * m = -inf, l = 0, O = 0 ("Lesson 8", section 3, before the first block).
- * m, l [B,Hq,S_loc] float; O [B,S_loc,Hq,D] float.
+ * m, l [B,Hq,S_loc] float; O [B,S_loc,Hq,D] float.  Returns RING_EINVAL for
+ * null/misaligned pointers, sizes < 1 or D % 4 != 0; RING_ECUDA on launch
+ * failure.
  */
 ring_status ring_attn_state_init(float* m, float* l, float* O, int B, int Hq, int S_loc, int D,
                                  void* stream);
@@ -174,7 +177,9 @@ ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* 
 /*
  * ring_attn_state_finalize -- out = O (cast to dtype), lse = m + ln l, for a
  * state produced by ring_attn_step.  out [B,S_loc,Hq,D]; lse [B,Hq,S_loc].
- * A row with l == 0 gets out = 0 and lse = -inf.
+ * A row with l == 0 gets out = 0 and lse = -inf.  Returns RING_EINVAL for
+ * null/misaligned pointers, sizes < 1 or a dtype out of range; RING_ECUDA on
+ * launch failure.
  */
 ring_status ring_attn_state_finalize(const float* m, const float* l, const float* O, void* out,
                                      float* lse, int B, int Hq, int S_loc, int D, int dtype,
@@ -198,7 +203,9 @@ size_t ring_attn_bwd_workspace_bytes(int B, int Hq, int S);
 
 /*
  * ring_attn_bwd_delta -- delta[b,h,i] = sum_d dout[b,i,h,d] * out[b,i,h,d]
- * for out, dout [B,S,Hq,D] of `dtype`; delta [B,Hq,S] float.
+ * for out, dout [B,S,Hq,D] of `dtype`; delta [B,Hq,S] float.  Returns
+ * RING_EINVAL for null/misaligned pointers, sizes < 1 or a dtype out of
+ * range; RING_ECUDA on launch failure.
  */
 ring_status ring_attn_bwd_delta(const void* out, const void* dout, float* delta, int B, int Hq, int S, int D,
                                 int dtype, void* stream);
@@ -402,6 +409,8 @@ ring_status ring_attn_kv_append(void* k_cache, void* v_cache, const void* k_new,
  * cut inside each chunk pair (full: no mask needed; partial: masked;
  * skipped: fully masked, never issued).  `layout` as for ring_attn_fwd.
  * per_rank_pairs has room for P values.  Any output pointer may be NULL.
+ * Returns RING_EINVAL for S, P, tile_q or tile_k < 1, or a split out of range
+ * or not dividing S; it touches no device.
  */
 ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile_q, int tile_k,
                                   int64_t* per_rank_pairs, int64_t* full, int64_t* partial,
@@ -426,10 +435,12 @@ ring_status ring_attn_device_error(int* where);
  */
 ring_status ring_attn_selftest_wait(int limit_us, void* stream);
 
-/* A static, human-readable name for a status code. */
+/* A static, human-readable name for a status code; an unknown code gives
+ * "unknown status".  Never fails. */
 const char* ring_attn_strerror(ring_status status);
 
-/* Library version and the SM architecture it was compiled for (e.g. 100). */
+/* Library version and the SM architecture it was compiled for (e.g. 100).
+ * Both are constants of the build and never fail. */
 int ring_attn_version(void);
 int ring_attn_built_arch(void);
 
