@@ -300,3 +300,13 @@ def test_state_init_and_finalize_argument_checks():
     assert fin(out=FAKE + 2) == ra.RING_EINVAL
     assert fin(B=0) == ra.RING_EINVAL
     assert fin(dtype=3) == ra.RING_EINVAL
+
+
+def test_every_declared_function_documents_its_errors():
+    # the comment above each declaration says what the call returns on failure (or that it cannot fail)
+    text = open(HEADER).read()
+    documented = {}
+    for m in re.finditer(r"/\*(.*?)\*/\s*(?:#define[^\n]*\n)?([^;/]*?\b(ring_attn_[a-z0-9_]+)\s*\([^;]*;)", text, re.S):
+        documented[m.group(3)] = bool(re.search(r"RING_E|[Ee]rrors|Returns|0 on bad|[Nn]ever fail", m.group(1)))
+    assert set(declared_functions()) <= set(documented) | {"ring_attn_built_arch"}
+    assert [n for n, ok in documented.items() if not ok] == []
