@@ -124,6 +124,9 @@ ring_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out
  * Tiles are 128 query rows x 128 keys cut inside each chunk pair (the last
  * tile of a chunk may be shorter).  Only dtype RING_BF16 counts; other
  * arguments and errors as ring_attn_fwd.
+ * Instrumentation of the scheduler: the per-rank pair counts are those of
+ * "Lesson 8", section 4B (2P+1 per zig-zag rank) and section 4A (r+1 per
+ * contiguous rank).
  */
 ring_status ring_attn_fwd_counted(const void* q, const void* k, const void* v, void* out, float* lse,
                                   int B, int Hq, int Hkv, int S, int D, int P, int causal, int layout,
@@ -134,6 +137,7 @@ ring_status ring_attn_fwd_counted(const void* q, const void* k, const void* v, v
  * with float32 FMA for both dtypes (bf16 inputs are widened exactly).  Slow;
  * it exists to cross-check the tensor-core path on the GPU.  Arguments and
  * errors as ring_attn_fwd.
+ * The computation is that of "Lesson 8", sections 2-4.
  */
 ring_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse,
                                int B, int Hq, int Hkv, int S, int D, int P, int causal, int layout,
@@ -180,6 +184,8 @@ ring_status ring_attn_step(const void* q_shard, const void* kchunk, const void* 
  * A row with l == 0 gets out = 0 and lse = -inf.  Returns RING_EINVAL for
  * null/misaligned pointers, sizes < 1 or a dtype out of range; RING_ECUDA on
  * launch failure.
+ * "Lesson 8", section 3 keeps (m, l); lse = m + ln l is this library's
+ * reading of the log-sum-exp of that state.
  */
 ring_status ring_attn_state_finalize(const float* m, const float* l, const float* O, void* out,
                                      float* lse, int B, int Hq, int S_loc, int D, int dtype,
@@ -206,6 +212,7 @@ size_t ring_attn_bwd_workspace_bytes(int B, int Hq, int S);
  * for out, dout [B,S,Hq,D] of `dtype`; delta [B,Hq,S] float.  Returns
  * RING_EINVAL for null/misaligned pointers, sizes < 1 or a dtype out of
  * range; RING_ECUDA on launch failure.
+ * The pages give no backward (see the backward pass above).
  */
 ring_status ring_attn_bwd_delta(const void* out, const void* dout, float* delta, int B, int Hq, int S, int D,
                                 int dtype, void* stream);
@@ -217,6 +224,7 @@ ring_status ring_attn_bwd_delta(const void* out, const void* dout, float* delta,
  * errors as ring_attn_fwd; workspace (ring_attn_bwd_workspace_bytes bytes,
  * 256-byte aligned) receives delta.  dq, dk, dv are overwritten; the results
  * do not depend on the launch order of tiles (no atomics).
+ * The pages give no backward (see the backward pass above).
  */
 ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                           const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
@@ -228,6 +236,7 @@ ring_status ring_attn_bwd(const void* q, const void* k, const void* v, const voi
  * dtypes (the bf16 ring_attn_bwd runs on the tensor cores: tcgen05 products
  * of 128 x 128 tiles, fp32 accumulation in tensor memory).  Slow; it exists
  * to cross-check the tensor-core path.  Arguments and errors as ring_attn_bwd.
+ * The pages give no backward (see the backward pass above).
  */
 ring_status ring_attn_bwd_simt(const void* q, const void* k, const void* v, const void* out, const float* lse,
                                const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
@@ -244,6 +253,8 @@ ring_status ring_attn_bwd_simt(const void* q, const void* k, const void* v, cons
  * shard's dQ) and dk_acc, dv_acc [B, n_kv*C, Hkv, D] float (the shard's share
  * of the block's dK, dV, which travel with the block).  Errors as
  * ring_attn_step.
+ * The pages give no backward; the hop mirrors the forward's ring step
+ * ("Lesson 8", section 2).
  */
 ring_status ring_attn_step_bwd(const void* q_shard, const void* kchunk, const void* vchunk, const void* dout_shard,
                                const float* lse, const float* delta, float* dq_acc, float* dk_acc, float* dv_acc,
@@ -283,7 +294,8 @@ ring_status ring_attn_decode_partial(const void* q, const void* k, const void* v
                                      int dtype, void* workspace, size_t workspace_bytes,
                                      void* stream);
 
-/* Bytes of workspace ring_attn_decode_partial needs for these sizes (0 on bad sizes). */
+/* Bytes of workspace ring_attn_decode_partial needs for these sizes (0 on bad sizes).
+ * A library helper; the pages have no counterpart. */
 size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Smax, int D, int P);
 
 /*
@@ -336,6 +348,7 @@ ring_status ring_attn_merge(const float* partials, const float* part_lse, void* 
  * the caller's buffers for the per-chunk results (as above); out [B,Hq,D]
  * bf16 and out_lse [B,Hq] float (may be NULL) receive attention over all
  * seqlens[b] keys.  Errors as the two calls.
+ * The split-KV decode of "NVIDIA unveils Helix Parallelism", Phase 1.
  */
 ring_status ring_attn_decode(const void* q, const void* k, const void* v, const int32_t* seqlens, float* partials,
                              float* part_lse, void* out, float* out_lse, int B, int Hq, int Hkv, int Smax, int D,
@@ -423,6 +436,7 @@ ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile
  * dropped a token because its shard was full, RING_ECUDA if the device
  * reports an error, else RING_OK.  `where` (may be NULL) receives the code
  * of the site that recorded the error (0 if none).
+ * A library helper; the pages have no counterpart.
  */
 ring_status ring_attn_device_error(int* where);
 
@@ -432,15 +446,18 @@ ring_status ring_attn_device_error(int* where);
  * every wait inside the library's kernels gives up after its own limit.  The
  * next ring_attn_device_error() then reports RING_ETIMEOUT.  No fault, trap
  * or hang is involved; it exists to test the error path.
+ * A library helper; the pages have no counterpart.
  */
 ring_status ring_attn_selftest_wait(int limit_us, void* stream);
 
 /* A static, human-readable name for a status code; an unknown code gives
- * "unknown status".  Never fails. */
+ * "unknown status".  Never fails.
+ * A library helper; the pages have no counterpart. */
 const char* ring_attn_strerror(ring_status status);
 
 /* Library version and the SM architecture it was compiled for (e.g. 100).
- * Both are constants of the build and never fail. */
+ * Both are constants of the build and never fail.
+ * Library helpers; the pages have no counterpart. */
 int ring_attn_version(void);
 int ring_attn_built_arch(void);
 

@@ -310,3 +310,11 @@ def test_every_declared_function_documents_its_errors():
         documented[m.group(3)] = bool(re.search(r"RING_E|[Ee]rrors|Returns|0 on bad|[Nn]ever fail", m.group(1)))
     assert set(declared_functions()) <= set(documented) | {"ring_attn_built_arch"}
     assert [n for n, ok in documented.items() if not ok] == []
+
+
+def test_every_declared_function_cites_its_passage_or_says_it_has_none():
+    text = open(HEADER).read()
+    uncited = [m.group(3) for m in re.finditer(
+        r"/\*(.*?)\*/\s*(?:#define[^\n]*\n)?([^;/]*?\b(ring_attn_[a-z0-9_]+)\s*\([^;]*;)", text, re.S)
+        if not re.search(r"Lesson 8|Sequence parallelism|Helix|pages", m.group(1))]
+    assert uncited == []
