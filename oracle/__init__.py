@@ -43,7 +43,10 @@ _lib = None
 
 def build(force: bool = False) -> str:
     """Compile attn_fp64.c with gcc (plain -O2, no fast-math: the oracle keeps
-    IEEE double semantics).  Returns the path of the shared library."""
+    IEEE double semantics).  Returns the path of the shared library.
+
+    Plumbing (builds the C oracle); no passage.
+    """
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
@@ -80,7 +83,10 @@ def _load():
 
 
 def cores() -> int:
-    """Host cores available to the oracle's threads."""
+    """Host cores available to the oracle's threads.
+
+    Plumbing; no passage.
+    """
     return int(_load().oracle_cores())
 
 
@@ -100,6 +106,9 @@ def attention_rows(q, k, v, rows, *, scale: float, causal: bool,
     ``qpos``/``kpos`` give global token positions (default: the row index),
     ``kv_len`` [B] limits the keys of each batch entry.
     Returns (out [n,D] float64, lse [n] float64); lse is the natural log.
+
+    Follows the definition of attention in "Lesson 8: Context Parallelism",
+    section 1, with the causal rule of section 4 (attn_fp64.c).
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
     B, Sq, Hq, D = q.shape
@@ -133,6 +142,9 @@ def attention_bwd(q, k, v, dout, *, scale: float, causal: bool, qpos=None, kpos=
 
     q, dout [B,Sq,Hq,D], k/v [B,Skv,Hkv,D] (read as float32).  Returns
     (dq [B,Sq,Hq,D], dk [B,Skv,Hkv,D], dv [B,Skv,Hkv,D]) float64.
+
+    The pages give no backward: this is the calculus of the definition of
+    "Lesson 8", section 1 (attn_fp64.c).
     """
     q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
     B, Sq, Hq, D = q.shape
@@ -160,7 +172,11 @@ def attention_bwd(q, k, v, dout, *, scale: float, causal: bool, qpos=None, kpos=
 
 def attention_bwd_dq_rows(q, k, v, dout, rows, *, scale: float, causal: bool, threads: int = 0):
     """fp64 dq of the requested query rows (b, h, i) only: each row needs just
-    its own scores, so large problems can be sampled.  Returns [n, D] float64."""
+    its own scores, so large problems can be sampled.  Returns [n, D] float64.
+
+    The pages give no backward: the calculus of "Lesson 8", section 1, one
+    query row at a time (attn_fp64.c).
+    """
     q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
     B, S, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
@@ -176,7 +192,10 @@ def attention_bwd_dq_rows(q, k, v, dout, rows, *, scale: float, causal: bool, th
 
 
 def all_rows(B: int, H: int, S: int) -> np.ndarray:
-    """Every (b, h, i) triple, in (b, h, i) order."""
+    """Every (b, h, i) triple, in (b, h, i) order.
+
+    Plumbing; no passage.
+    """
     b, h, i = np.meshgrid(np.arange(B), np.arange(H), np.arange(S), indexing="ij")
     return np.stack([b.ravel(), h.ravel(), i.ravel()], axis=1).astype(np.int32)
 
@@ -184,7 +203,10 @@ def all_rows(B: int, H: int, S: int) -> np.ndarray:
 def attention_full(q, k, v, *, scale: float, causal: bool, qpos=None, kpos=None,
                    kv_len=None, threads: int = 0):
     """fp64 attention for every query row.
-    Returns out [B,Sq,Hq,D] and lse [B,Hq,Sq] (float64)."""
+    Returns out [B,Sq,Hq,D] and lse [B,Hq,Sq] (float64).
+
+    As attention_rows ("Lesson 8", sections 1 and 4), for every row.
+    """
     B, Sq, Hq, D = np.asarray(q).shape
     rows = all_rows(B, Hq, Sq)
     out, lse = attention_rows(q, k, v, rows, scale=scale, causal=causal, qpos=qpos,

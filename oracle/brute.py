@@ -12,7 +12,11 @@ import numpy as np
 
 
 def brute(q, k, v, *, scale: float, causal: bool, qpos=None, kpos=None, kv_len=None):
-    """Returns (out [B,Sq,Hq,D], lse [B,Hq,Sq]) in float64."""
+    """Returns (out [B,Sq,Hq,D], lse [B,Hq,Sq]) in float64.
+
+    Follows "Lesson 8: Context Parallelism", section 1, with the causal rule of
+    section 4.
+    """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)

@@ -20,7 +20,10 @@ from __future__ import annotations
 
 def append_rank(n: int, block: int, P: int) -> int:
     """Rank that receives the n-th appended token (n = 0, 1, ...): block
-    n // block, dealt to the ranks in turn."""
+    n // block, dealt to the ranks in turn.
+
+    Follows "NVIDIA unveils Helix Parallelism", on KV cache growth.
+    """
     return (n // block) % P
 
 
@@ -31,6 +34,8 @@ def simulate_appends(shards: list[list], n_appended: int, tokens: list, block: i
     A token whose shard already holds `capacity` rows is dropped.  Returns
     (shards, n_appended_after, placements, dropped), where placements[j] is
     (rank, row) for token j, or None if it was dropped.
+
+    Follows "NVIDIA unveils Helix Parallelism", on KV cache growth.
     """
     shards = [list(s) for s in shards]
     placements, dropped = [], 0

@@ -21,7 +21,12 @@ import numpy as np
 
 
 def merge(partials, part_lse):
-    """partials [..., P, D], part_lse [..., P] -> (out [..., D], lse [...])."""
+    """partials [..., P, D], part_lse [..., P] -> (out [..., D], lse [...]).
+
+    The update of "Lesson 8: Context Parallelism", section 3, applied to
+    whole partial states (the merge of "NVIDIA unveils Helix Parallelism",
+    Phase 1).
+    """
     O = np.asarray(partials, dtype=np.float64)
     L = np.asarray(part_lse, dtype=np.float64)
     m = L.max(axis=-1, keepdims=True)

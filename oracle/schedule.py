@@ -33,7 +33,11 @@ _DEFAULT_K = {"contiguous": 1, "zigzag": 2, "striped": 1}
 
 def parse_layout(layout: str) -> tuple[str, int]:
     """Split name and chunks per rank: 'contiguous' | 'zigzag' | 'striped',
-    optionally followed by k ('zigzag4' = four chunks per rank)."""
+    optionally followed by k ('zigzag4' = four chunks per rank).
+
+    Plumbing (names the splits of "Lesson 8", sections 4A and 4B, and the
+    striped variant); no arithmetic.
+    """
     name = layout.rstrip("0123456789")
     if name not in _DEFAULT_K:
         raise ValueError(layout)
@@ -69,7 +73,11 @@ def zigzag_assignment(P: int, chunks_per_rank: int = 2) -> dict[int, list[int]]:
 
 
 def striped_tokens(S: int, P: int) -> dict[int, list[int]]:
-    """Striped split: rank r holds tokens r, r+P, r+2P, ... in that order."""
+    """Striped split: rank r holds tokens r, r+P, r+2P, ... in that order.
+
+    Reading of the striped variant named in "Sequence parallelism and ring
+    attention", outlook.
+    """
     return {r: list(range(r, S, P)) for r in range(P)}
 
 
@@ -87,7 +95,10 @@ def layout_assignment(P: int, layout: str) -> dict[int, list[int]]:
 
 
 def chunk_positions(S: int, P: int, layout: str) -> dict[int, list[int]]:
-    """Global token positions of every chunk, in the chunk's row order."""
+    """Global token positions of every chunk, in the chunk's row order.
+
+    Chunks of "Lesson 8", sections 4A and 4B (stripes for the striped split).
+    """
     name, _ = parse_layout(layout)
     if name == "striped":
         if S % P:
@@ -127,7 +138,10 @@ def ring_pairs(P: int, layout: str, causal: bool, S: int | None = None) -> list[
     """Every (rank, step, q chunk, kv chunk) the ring loop meets, classified
     under the causal rule.  Chunked splits: kv < q full, kv == q diagonal,
     kv > q skipped.  Striped split (S needed): from the token positions, full
-    if every key precedes every query, skipped if none does, else 'diag'."""
+    if every key precedes every query, skipped if none does, else 'diag'.
+
+    Rotation of "Lesson 8", section 2; causal rule of section 4.
+    """
     own = layout_assignment(P, layout)
     striped = parse_layout(layout)[0] == "striped"
     pos = chunk_positions(S, P, layout) if striped else None
@@ -155,7 +169,10 @@ def ring_pairs(P: int, layout: str, causal: bool, S: int | None = None) -> list[
 
 
 def per_rank_pairs(P: int, layout: str, causal: bool, S: int | None = None) -> list[int]:
-    """Unmasked chunk pairs per rank (a diagonal pair counts as one)."""
+    """Unmasked chunk pairs per rank (a diagonal pair counts as one).
+
+    Counting of "Lesson 8", section 4B (a diagonal pair counts once).
+    """
     cnt = [0] * P
     for p in ring_pairs(P, layout, causal, S):
         if p.kind != "skip":
@@ -164,7 +181,10 @@ def per_rank_pairs(P: int, layout: str, causal: bool, S: int | None = None) -> l
 
 
 def chunk_len(S: int, P: int, layout: str) -> int:
-    """Rows per chunk (per stripe for the striped split)."""
+    """Rows per chunk (per stripe for the striped split).
+
+    Chunk length of "Lesson 8", sections 4A and 4B.
+    """
     name, k = parse_layout(layout)
     n = P * k
     if S % n:
@@ -183,6 +203,8 @@ def tile_classes(S: int, P: int, layout: str, causal: bool, tile_q: int, tile_k:
     else 'partial' (causal); all tiles are full otherwise.
     Returns (full, partial, skipped, per_rank_processed[P]) where processed
     counts full + partial tiles by the rank owning the queries.
+
+    Causal rule of "Lesson 8", section 4, applied tile by tile.
     """
     pos = {c: np.asarray(v, dtype=np.int64) for c, v in chunk_positions(S, P, layout).items()}
 
@@ -214,6 +236,9 @@ def tile_classes(S: int, P: int, layout: str, causal: bool, tile_q: int, tile_k:
 def kv_visit_order(P: int, layout: str, rank: int) -> list[int]:
     """Global K/V chunk indices in the order rank ``rank`` meets them during
     one ring loop (for zig-zag, both chunks of the source rank at each step,
-    in the order that rank owns them)."""
+    in the order that rank owns them).
+
+    Rotation of "Lesson 8", section 2.
+    """
     own = layout_assignment(P, layout)
     return [c for src in ring_rotation(P, rank) for c in own[src]]

@@ -21,6 +21,8 @@ import numpy as np
 
 
 def init_state(n_rows: int, D: int):
+    """The starting state of "Lesson 8", section 3: m = -inf, l = 0, O = 0.
+    """
     return (np.full(n_rows, -np.inf), np.zeros(n_rows), np.zeros((n_rows, D)))
 
 
@@ -29,6 +31,8 @@ def update(state, s_new: np.ndarray, v_new: np.ndarray):
 
     s_new [n, Lk] scaled scores of the new block (-inf where masked),
     v_new [Lk, D] its value rows.  Returns the new (m, l, O) with O normalised.
+
+    The update of "Lesson 8", section 3.
     """
     m, l, O = state
     blk_max = s_new.max(axis=1) if s_new.shape[1] else np.full(s_new.shape[0], -np.inf)
@@ -50,7 +54,10 @@ def ring_attention_rows(q, k, v, *, scale: float, causal: bool, chunks_in_order,
                         q_rows, qpos, h: int, b: int = 0):
     """Run the recurrence for query rows ``q_rows`` (positions ``qpos``) of head
     h over the K/V chunks given in visiting order.  q [B,S,Hq,D], k/v
-    [B,S,Hkv,D].  Returns (out, lse, m, l) per row."""
+    [B,S,Hkv,D].  Returns (out, lse, m, l) per row.
+
+    The ring loop of "Lesson 8", sections 2 and 3.
+    """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
