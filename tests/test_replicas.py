@@ -90,3 +90,26 @@ def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monk
     f.write_text(f.read_text() + "\n")
     changed = bench.load_traffic()
     assert changed["decode"] is None and changed["attn_tc"] == cur["attn_tc"]
+
+
+def test_profile_summaries_name_commands_the_bench_accepts():
+    # every command a profile summary cites runs committed code: bench.py with options it
+    # defines and profile cases it has
+    import glob
+    import re
+    import shlex
+    lines = []
+    for f in glob.glob(os.path.join(bench.ROOT, "profiles", "*.md")):
+        for line in open(f, encoding="utf-8"):
+            if "python bench.py" in line:
+                lines.append(line[line.index("python bench.py"):].strip())
+    assert lines
+    parser_src = open(os.path.join(bench.ROOT, "bench.py"), encoding="utf-8").read()
+    options = set(re.findall(r'add_argument\("(--[a-z0-9-]+)"', parser_src))
+    for cmd in lines:
+        words = shlex.split(cmd)[2:]
+        for i, w in enumerate(words):
+            if w.startswith("--"):
+                assert w in options, (cmd, w)
+            if w == "--profile":
+                assert words[i + 1] in bench.PROFILE_CASES, cmd
