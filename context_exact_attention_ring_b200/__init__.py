@@ -12,7 +12,8 @@ Names follow the C ABI:
   ring_attn_state_init, ring_attn_step, ring_attn_state_finalize,
   ring_attn_decode_partial, ring_attn_merge, ring_attn_decode,
   ring_attn_decode_workspace_bytes, ring_attn_decode_fused,
-  ring_attn_kv_append, ring_attn_sched_stats, ring_attn_device_error.
+  ring_attn_kv_append, ring_attn_sched_stats, ring_attn_device_error;
+and ring_attention (RingAttnFunction), the forward and backward under autograd.
 """
 from __future__ import annotations
 
@@ -457,6 +458,32 @@ def ring_attn_kv_append(k_cache, v_cache, k_new, v_new, shard_lens, n_appended, 
                                    _ptr(n_appended), B, T, Hkv, Smax, D, int(P), int(block),
                                    _dtype_code(k_cache), _stream())
     _check(st, "ring_attn_kv_append")
+
+
+class RingAttnFunction(torch.autograd.Function):
+    """Autograd over the whole ring: forward is ring_attn_fwd, backward is
+    ring_attn_bwd on the saved q, k, v, out and lse.  Only marshalling: both
+    passes run in the library's kernels."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, P, causal=True, layout="zigzag", scale=None):
+        out, lse = ring_attn_fwd(q, k, v, P, causal, layout, scale)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.cfg = (P, causal, layout, scale)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        P, causal, layout, scale = ctx.cfg
+        dq, dk, dv = ring_attn_bwd(q, k, v, out, lse, dout.to(q.dtype).contiguous(), P, causal, layout, scale)
+        return dq, dk, dv, None, None, None, None
+
+
+def ring_attention(q, k, v, P, causal=True, layout="zigzag", scale=None):
+    """out = ring attention of q, k, v that autograd can differentiate
+    (RingAttnFunction)."""
+    return RingAttnFunction.apply(q, k, v, P, causal, layout, scale)
 
 
 def ring_attn_sched_stats(S, P, causal, layout, tile_q=128, tile_k=128):
