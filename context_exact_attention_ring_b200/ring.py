@@ -10,6 +10,7 @@ kernel reads them: every kernel reads local memory only.  The backward runs
 the same loop with ring_attn_step_bwd; the dK, dV sums of a block travel with
 it and take one last hop home.  helix_decode is the decode's
 exchange: per-shard partials, one all-gather, and the merge on every rank.
+ring_attention puts the forward and backward loops under torch autograd.
 
 The chunk ownership follows the splits of ring_attn_fwd (see split_chunks);
 the step functions default to this package's kernels and can be replaced
@@ -94,14 +95,17 @@ def ring_forward(q_shard, k_block, v_block, layout="zigzag", causal=True, scale=
     B, S_loc, Hq, D = q_shard.shape
     m, l, O = (new_state or _new_state)(B, Hq, S_loc, D, device=q_shard.device)
     cur = [k_block.contiguous(), v_block.contiguous()]
-    nxt = [torch.empty_like(x) for x in cur]
+    # received blocks alternate between two buffers of the loop's own: the caller's block is
+    # only ever sent, never overwritten
+    bufs = [[torch.empty_like(x) for x in cur] for _ in range(min(2, P - 1))]
     for t in range(P):
         src = (r - t) % P
+        nxt = bufs[t % 2] if t < P - 1 else None
         reqs = ring.shift(cur, nxt) if t < P - 1 else []
         step(q_shard, cur[0], cur[1], m, l, O, own[r], own[src], C, causal=causal, scale=scale, stripes=stripes)
         _wait(reqs)
         if t < P - 1:
-            cur, nxt = nxt, cur
+            cur = nxt
     return (finalize or ring_attn_state_finalize)(m, l, O, dtype=q_shard.dtype)
 
 
@@ -121,11 +125,14 @@ def ring_backward(q_shard, k_block, v_block, out_shard, lse_shard, dout_shard, l
     f32 = dict(device=q_shard.device, dtype=torch.float32)
     dq = torch.zeros(q_shard.shape, **f32)
     kv = [k_block.contiguous(), v_block.contiguous()]
-    kv_nxt = [torch.empty_like(x) for x in kv]
+    # as in ring_forward: the caller's block is only sent; received blocks alternate between two
+    # buffers of the loop's own
+    kv_bufs = [[torch.empty_like(x) for x in kv] for _ in range(min(2, P - 1))]
     gr = [torch.zeros(k_block.shape, **f32), torch.zeros(v_block.shape, **f32)]
     gr_nxt = [torch.empty_like(x) for x in gr]
     for t in range(P):
         src = (r - t) % P
+        kv_nxt = kv_bufs[t % 2] if t < P - 1 else None
         reqs = ring.shift(kv, kv_nxt) if t < P - 1 else []   # the next block arrives during the step
         step(q_shard, kv[0], kv[1], dout_shard, lse_shard, delta, dq, gr[0], gr[1], own[r], own[src], C,
              causal=causal, scale=scale, stripes=stripes)
@@ -134,8 +141,37 @@ def ring_backward(q_shard, k_block, v_block, out_shard, lse_shard, dout_shard, l
         if P > 1:
             gr, gr_nxt = gr_nxt, gr
             if t < P - 1:
-                kv, kv_nxt = kv_nxt, kv
+                kv = kv_nxt
     return dq.to(q_shard.dtype), gr[0].to(k_block.dtype), gr[1].to(v_block.dtype)
+
+
+class RingAttention(torch.autograd.Function):
+    """Autograd over the cross-GPU ring: forward is ring_forward, backward is
+    ring_backward on the saved shard, out and lse (the dK, dV of this rank's
+    block come home with it).  fwd_kw / bwd_kw pass the optional step
+    functions of the two loops."""
+
+    @staticmethod
+    def forward(ctx, q_shard, k_block, v_block, layout, causal, scale, ring, fwd_kw, bwd_kw):
+        out, lse = ring_forward(q_shard, k_block, v_block, layout, causal, scale, ring, **(fwd_kw or {}))
+        ctx.save_for_backward(q_shard, k_block, v_block, out, lse)
+        ctx.cfg = (layout, causal, scale, ring, bwd_kw or {})
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q_shard, k_block, v_block, out, lse = ctx.saved_tensors
+        layout, causal, scale, ring, bwd_kw = ctx.cfg
+        dq, dk, dv = ring_backward(q_shard, k_block, v_block, out, lse, dout.to(q_shard.dtype).contiguous(), layout,
+                                   causal, scale, ring, **bwd_kw)
+        return dq, dk, dv, None, None, None, None, None, None
+
+
+def ring_attention(q_shard, k_block, v_block, layout="zigzag", causal=True, scale=None, ring=None, fwd_kw=None,
+                   bwd_kw=None):
+    """This rank's output of the cross-GPU ring, differentiable by autograd
+    (RingAttention).  Every rank calls it, and later its backward, in step."""
+    return RingAttention.apply(q_shard, k_block, v_block, layout, causal, scale, ring, fwd_kw, bwd_kw)
 
 
 def helix_decode(q, k_shard, v_shard, shard_len, scale=None, group=None, partial=None, merge=None):

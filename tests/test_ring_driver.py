@@ -312,3 +312,87 @@ def test_rings_on_process_subgroups():
         rl = rl.reshape(B, Hq, S)
         np.testing.assert_allclose(out, ro[:, rows], atol=1e-12, rtol=0)
         np.testing.assert_allclose(lse, rl[:, :, rows], atol=1e-12, rtol=0)
+
+
+def _rank_autograd(rank, world, port, q_out):
+    # the ring under autograd: loss = sum(out * dout) per rank, backward through the ring loop
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        B, S, Hq, Hkv, D = 1, 32 * world, 4, 2, 8
+        q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 25)
+        rows = R.shard_rows(S, world, "zigzag", rank).numpy()
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows])).double().requires_grad_()
+        qs, ks, vs = t(q), t(k), t(v)
+        out = R.ring_attention(qs, ks, vs, "zigzag", True, 0.4,
+                               fwd_kw=dict(step=fake_step, new_state=fake_new_state, finalize=fake_finalize),
+                               bwd_kw=dict(step=fake_step_bwd, delta_fn=fake_delta))
+        (out * torch.from_numpy(np.ascontiguousarray(dout[:, rows])).double()).sum().backward()
+        q_out.put((rank, rows, out.detach().numpy(), qs.grad.numpy(), ks.grad.numpy(), vs.grad.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_attention_under_autograd_on_cpu_ranks():
+    import oracle
+    world = 3
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_autograd, args=(r, world, port, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [qq.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    B, S, Hq, Hkv, D = 1, 32 * world, 4, 2, 8
+    q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 25)
+    ro, _ = oracle.attention_rows(q, k, v, oracle.all_rows(B, Hq, S), scale=0.4, causal=True)
+    ro = ro.reshape(B, Hq, S, D).transpose(0, 2, 1, 3)
+    dq_ref, dk_ref, dv_ref = oracle.attention_bwd(q, k, v, dout, scale=0.4, causal=True)
+    for rank, rows, out, dq, dk, dv in res:
+        np.testing.assert_allclose(out, ro[:, rows], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(dq, dq_ref[:, rows], atol=2e-6, rtol=0)
+        np.testing.assert_allclose(dk, dk_ref[:, rows], atol=2e-6, rtol=0)
+        np.testing.assert_allclose(dv, dv_ref[:, rows], atol=2e-6, rtol=0)
+
+
+def _rank_inputs_kept(rank, world, port, q_out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        B, S, Hq, Hkv, D = 1, 16 * world, 2, 1, 8
+        q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 27)
+        rows = R.shard_rows(S, world, "zigzag", rank).numpy()
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows])).double()
+        qs, ks, vs, ds = t(q), t(k), t(v), t(dout)
+        before = [x.clone() for x in (qs, ks, vs, ds)]
+        out, lse = R.ring_forward(qs, ks, vs, layout="zigzag", causal=True, scale=0.4, step=fake_step,
+                                  new_state=fake_new_state, finalize=fake_finalize)
+        after_fwd = all(torch.equal(a, b) for a, b in zip(before, (qs, ks, vs, ds)))
+        R.ring_backward(qs, ks, vs, out, lse, ds, layout="zigzag", causal=True, scale=0.4, step=fake_step_bwd,
+                        delta_fn=fake_delta)
+        after_bwd = all(torch.equal(a, b) for a, b in zip(before, (qs, ks, vs, ds)))
+        q_out.put((rank, after_fwd and after_bwd))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [3, 4])
+def test_the_loops_leave_the_callers_shards_unchanged(world):
+    # the forward's shards are the backward's inputs: a loop that received a later block into the
+    # caller's own K/V buffer would corrupt the gradients
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_inputs_kept, args=(r, world, port, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [qq.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    assert all(ok for _, ok in res), res
