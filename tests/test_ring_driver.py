@@ -314,7 +314,7 @@ def test_rings_on_process_subgroups():
         np.testing.assert_allclose(lse, rl[:, :, rows], atol=1e-12, rtol=0)
 
 
-def _rank_autograd(rank, world, port, q_out):
+def _rank_autograd(rank, world, port, layout, q_out):
     # the ring under autograd: loss = sum(out * dout) per rank, backward through the ring loop
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -322,10 +322,10 @@ def _rank_autograd(rank, world, port, q_out):
     try:
         B, S, Hq, Hkv, D = 1, 32 * world, 4, 2, 8
         q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 25)
-        rows = R.shard_rows(S, world, "zigzag", rank).numpy()
+        rows = R.shard_rows(S, world, layout, rank).numpy()
         t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows])).double().requires_grad_()
         qs, ks, vs = t(q), t(k), t(v)
-        out = R.ring_attention(qs, ks, vs, "zigzag", True, 0.4,
+        out = R.ring_attention(qs, ks, vs, layout, True, 0.4,
                                fwd_kw=dict(step=fake_step, new_state=fake_new_state, finalize=fake_finalize),
                                bwd_kw=dict(step=fake_step_bwd, delta_fn=fake_delta))
         (out * torch.from_numpy(np.ascontiguousarray(dout[:, rows])).double()).sum().backward()
@@ -334,13 +334,14 @@ def _rank_autograd(rank, world, port, q_out):
         dist.destroy_process_group()
 
 
-def test_ring_attention_under_autograd_on_cpu_ranks():
+@pytest.mark.parametrize("layout", ["zigzag", "striped", "contiguous2"])
+def test_ring_attention_under_autograd_on_cpu_ranks(layout):
     import oracle
     world = 3
     ctx = mp.get_context("spawn")
     qq = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_autograd, args=(r, world, port, qq)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_autograd, args=(r, world, port, layout, qq)) for r in range(world)]
     for p in procs:
         p.start()
     res = [qq.get(timeout=120) for _ in range(world)]
