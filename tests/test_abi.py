@@ -318,3 +318,29 @@ def test_every_declared_function_cites_its_passage_or_says_it_has_none():
         r"/\*(.*?)\*/\s*(?:#define[^\n]*\n)?([^;/]*?\b(ring_attn_[a-z0-9_]+)\s*\([^;]*;)", text, re.S)
         if not re.search(r"Lesson 8|Sequence parallelism|Helix|pages", m.group(1))]
     assert uncited == []
+
+
+def test_binding_signatures_match_the_header():
+    # the ctypes argument list of every bound function has the header's arity, with pointers where
+    # the header has pointers, float where it has float and size_t where it has size_t
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    L = ra.lib()
+    checked = 0
+    for m in re.finditer(r"\b(ring_attn_[a-z0-9_]+)\s*\(([^;]*?)\)\s*;", text, flags=re.S):
+        name, params = m.group(1), " ".join(m.group(2).split())
+        fn = getattr(L, name)
+        if fn.argtypes is None:
+            continue
+        params = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        assert len(params) == len(fn.argtypes), (name, params, fn.argtypes)
+        for p, a in zip(params, fn.argtypes):
+            if "*" in p:
+                assert a in (ctypes.c_void_p,) or issubclass(a, ctypes._Pointer), (name, p, a)
+            elif p.startswith("float "):
+                assert a is ctypes.c_float, (name, p, a)
+            elif p.startswith("size_t "):
+                assert a is ctypes.c_size_t, (name, p, a)
+            else:
+                assert a is ctypes.c_int, (name, p, a)
+        checked += 1
+    assert checked >= 20
