@@ -467,6 +467,7 @@ class RingAttnFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, P, causal=True, layout="zigzag", scale=None):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()   # views (e.g. transposes) are copied once
         out, lse = ring_attn_fwd(q, k, v, P, causal, layout, scale)
         ctx.save_for_backward(q, k, v, out, lse)
         ctx.cfg = (P, causal, layout, scale)

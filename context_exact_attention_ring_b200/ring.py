@@ -153,6 +153,7 @@ class RingAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q_shard, k_block, v_block, layout, causal, scale, ring, fwd_kw, bwd_kw):
+        q_shard, k_block, v_block = q_shard.contiguous(), k_block.contiguous(), v_block.contiguous()
         out, lse = ring_forward(q_shard, k_block, v_block, layout, causal, scale, ring, **(fwd_kw or {}))
         ctx.save_for_backward(q_shard, k_block, v_block, out, lse)
         ctx.cfg = (layout, causal, scale, ring, bwd_kw or {})

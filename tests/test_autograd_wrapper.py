@@ -57,6 +57,22 @@ def test_gradients_flow_through_the_two_calls(monkeypatch):
         torch.testing.assert_close(a, b, rtol=0, atol=1e-12)
 
 
+def test_views_reach_the_library_as_contiguous_tensors(monkeypatch):
+    seen = []
+
+    def fake_fwd(q, k, v, P, causal=True, layout="zigzag", scale=None, out=None, lse=None):
+        seen.extend(x.is_contiguous() for x in (q, k, v))
+        with torch.no_grad():
+            return _attn(q, k, v, causal, scale), torch.zeros(q.shape[0], q.shape[2], q.shape[1], dtype=q.dtype)
+
+    monkeypatch.setattr(ra, "ring_attn_fwd", fake_fwd)
+    base = torch.randn(2, 4, 48, 16, dtype=torch.float64)
+    q = base.transpose(1, 2)                                  # [B, S, H, D] view, not contiguous
+    assert not q.is_contiguous()
+    ra.ring_attention(q, q, q, 4, True)
+    assert seen == [True, True, True]
+
+
 def test_host_tensors_are_refused():
     q = torch.zeros(1, 256, 2, 64, dtype=torch.bfloat16, requires_grad=True)
     k = torch.zeros(1, 256, 2, 64, dtype=torch.bfloat16)
