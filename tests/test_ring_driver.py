@@ -101,7 +101,7 @@ def _inputs(B, S, Hq, Hkv, D, seed):
     return f(B, S, Hq, D), f(B, S, Hkv, D), f(B, S, Hkv, D), f(B, S, Hq, D)
 
 
-def _rank(rank, world, port, layout, q_out):
+def _rank(rank, world, port, layout, q_out, causal=True):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
@@ -111,24 +111,25 @@ def _rank(rank, world, port, layout, q_out):
         q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 21)
         rows = R.shard_rows(S, world, layout, rank).numpy()
         t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows]))
-        out, lse = R.ring_forward(t(q), t(k), t(v), layout=layout, causal=True, scale=scale, step=fake_step,
+        out, lse = R.ring_forward(t(q), t(k), t(v), layout=layout, causal=causal, scale=scale, step=fake_step,
                                   new_state=fake_new_state, finalize=fake_finalize)
         dq, dk, dv = R.ring_backward(t(q).double(), t(k).double(), t(v).double(), out, lse, t(dout).double(),
-                                     layout=layout, causal=True, scale=scale, step=fake_step_bwd,
+                                     layout=layout, causal=causal, scale=scale, step=fake_step_bwd,
                                      delta_fn=fake_delta)
         q_out.put((rank, rows, out.numpy(), lse.numpy(), dq.numpy(), dk.numpy(), dv.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,layout", [(2, "zigzag"), (3, "contiguous"), (2, "striped"), (3, "zigzag3"),
-                                          (4, "zigzag"), (4, "striped")])
-def test_ring_loop_on_cpu_ranks(world, layout):
+@pytest.mark.parametrize("world,layout,causal", [(2, "zigzag", True), (3, "contiguous", True), (2, "striped", True),
+                                                 (3, "zigzag3", True), (4, "zigzag", True), (4, "striped", True),
+                                                 (3, "zigzag", False)])
+def test_ring_loop_on_cpu_ranks(world, layout, causal):
     import oracle
     ctx = mp.get_context("spawn")
     qq = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, layout, qq)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, layout, qq, causal)) for r in range(world)]
     for p in procs:
         p.start()
     res = [qq.get(timeout=120) for _ in range(world)]
@@ -138,10 +139,10 @@ def test_ring_loop_on_cpu_ranks(world, layout):
     B, S, Hq, Hkv, D = 1, 48 * world, 4, 2, 8
     q, k, v, dout = _inputs(B, S, Hq, Hkv, D, 21)
     rows_all = oracle.all_rows(B, Hq, S)
-    ro, rl = oracle.attention_rows(q, k, v, rows_all, scale=0.4, causal=True)
+    ro, rl = oracle.attention_rows(q, k, v, rows_all, scale=0.4, causal=causal)
     ro = ro.reshape(B, Hq, S, D).transpose(0, 2, 1, 3)
     rl = rl.reshape(B, Hq, S)
-    dq_ref, dk_ref, dv_ref = oracle.attention_bwd(q, k, v, dout, scale=0.4, causal=True)
+    dq_ref, dk_ref, dv_ref = oracle.attention_bwd(q, k, v, dout, scale=0.4, causal=causal)
     for rank, rows, out, lse, dq, dk, dv in res:
         np.testing.assert_allclose(out, ro[:, rows], atol=1e-12, rtol=0)
         np.testing.assert_allclose(lse, rl[:, :, rows], atol=1e-12, rtol=0)
