@@ -39,6 +39,11 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's published B200 figures: dense bf16 tensor throughput (half the 2:4-sparsity
+# figure of the datasheet) and HBM3e bandwidth of the HGX part.  Reported beside the
+# measured peaks so a reader can judge a fraction against either.
+PUBLISHED = {"bf16_tflops": 2250.0, "hbm_gbs": 7700.0,
+             "source": "NVIDIA B200 datasheet: 2.25 PFLOP/s dense bf16, 7.7 TB/s HBM3e (HGX)"}
 
 
 def peaks():
@@ -177,6 +182,35 @@ def step_ring(ra, cfg, q, k, v, dev):
             ra.ring_attn_state_finalize(m, l, O, dtype=q.dtype, out=o_r, lse=lse_r)
 
     return run, P * (P + 2), o_r, rows[P - 1]
+
+
+def merge_bytes(mc) -> float:
+    """Algorithmic bytes of one merge: the partials and their lse read once,
+    the bf16 output and its lse written."""
+    return float(mc.B * mc.Hq * (mc.P * (mc.D + 1) * 4 + mc.D * 2 + 4))
+
+
+def time_merge_only(ra, dev, reps=20):
+    """ring_attn_merge alone on an HBM-bound shape (W.MERGE_ONLY).  A 256 MB
+    write flushes L2 before every launch; each launch is timed with its own
+    CUDA events on the launching stream.  Returns (mean ms, GB/s)."""
+    mc = W.MERGE_ONLY
+    part, plse = W.merge_inputs(mc, dev)
+    out = torch.empty((mc.B, mc.Hq, mc.D), device=dev, dtype=torch.bfloat16)
+    olse = torch.empty((mc.B, mc.Hq), device=dev, dtype=torch.float32)
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
+    st = torch.cuda.current_stream()
+    for _ in range(3):
+        ra.ring_attn_merge(part, plse, out=out, out_lse=olse)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(st)
+        ra.ring_attn_merge(part, plse, out=out, out_lse=olse)
+        e1.record(st)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    return ms, merge_bytes(mc) / (ms / 1e3) / 1e9
 
 
 def run_ours(args):
@@ -374,6 +408,21 @@ def run_ours(args):
                     "frac": round(step_tf / world / peak_s, 4), "max_abs_diff_vs_fused_out": round(diff, 5)}
         del srun, so
 
+    # ---------------------------------------------------------------- the merge alone, HBM-bound
+    merge_only = None
+    if not args.no_merge:
+        barrier(dist)
+        m_ms, m_gbs = time_merge_only(ra, dev)
+        m_ms = max_over_ranks(dist, m_ms)
+        m_gbs = merge_bytes(W.MERGE_ONLY) / (m_ms / 1e3) / 1e9
+        merge_only = {"metric": "ring_attn_merge GB/s of algorithmic bytes, L2 flushed before each launch",
+                      "workload": W.MERGE_ONLY.name, "value": round(m_gbs * world, 1), "unit": "GB/s",
+                      "ms_per_launch": round(m_ms, 4), "bytes_per_launch": merge_bytes(W.MERGE_ONLY),
+                      "roofline": {"bound": "hbm", "achieved": round(m_gbs, 1), "peak": pk["hbm_gbs"],
+                                   "unit": "GB/s", "frac": round(m_gbs / pk["hbm_gbs"], 4),
+                                   "kernel": "merge_kernel<bf16>", "peak_kind": f"{pk_kind} HBM copy",
+                                   "frac_of_published": round(m_gbs / PUBLISHED["hbm_gbs"], 4)}}
+
     # ---------------------------------------------------------------- roofline of the dominant kernel
     pre_avg = statistics.mean(pre_ms)
     achieved_tf = flops / (pre_avg / 1e3) / 1e12
@@ -401,13 +450,19 @@ def run_ours(args):
                    "decode_workload": dcfg.name, "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(achieved_tf / peak_tf, 4), "traffic": traffic.get("attn_tc"),
-                     "kernel": "attn_tc_kernel<128>", "peak_kind": f"{pk_kind} bf16 dense, sustained"},
+                     "kernel": "attn_tc_kernel<128>", "peak_kind": f"{pk_kind} bf16 dense, sustained",
+                     "frac_of_burst": round(achieved_tf / pk["bf16_tflops"], 4),
+                     "frac_of_published": round(achieved_tf / PUBLISHED["bf16_tflops"], 4),
+                     "published_peak": PUBLISHED["bf16_tflops"], "published_source": PUBLISHED["source"]},
         "decode": {"metric": "split-KV decode GB/s", "value": round(dvalue, 1), "unit": "GB/s",
                    "ms_per_step": round(dec_avg, 3), "bytes_per_step": dbytes,
                    "roofline": {"bound": "hbm", "achieved": round(achieved_gb, 1), "peak": pk["hbm_gbs"],
                                 "unit": "GB/s", "frac": round(achieved_gb / pk["hbm_gbs"], 4),
                                 "traffic": traffic.get("decode"), "kernel": "decode_kernel<4, 128> + merge_kernel",
-                                "peak_kind": f"{pk_kind} HBM copy"}},
+                                "peak_kind": f"{pk_kind} HBM copy",
+                                "frac_of_published": round(achieved_gb / PUBLISHED["hbm_gbs"], 4),
+                                "published_peak": PUBLISHED["hbm_gbs"]},
+                   "merge_only": merge_only},
         "prefill_ms_per_step": round(pre_avg, 3),
         "e2e": e2e,
         "backward": bwd,
@@ -539,6 +594,8 @@ PROFILE_CASES = {
     "decode_full": W.CFG5,
     # the same decode in one launch (partials plus the last-CTA merge)
     "decode_full_fused": W.CFG5,
+    # the merge alone: B*Hq = 8192 rows of 32 float32 partials of 128 dims (134 MB > L2)
+    "merge": W.MERGE_ONLY,
 }
 
 
@@ -573,6 +630,12 @@ def run_profile(args):
         fn = lambda: ra.ring_attn_fwd(q, k, v, cfg.P, causal=cfg.causal, layout=cfg.layout, scale=cfg.scale,
                                       out=out, lse=lse)
         work, unit = cfg.flops() / 1e12, "TFLOP/s"
+    elif isinstance(cfg, W.Merge):
+        part, plse = W.merge_inputs(cfg, dev)
+        out = torch.empty((cfg.B, cfg.Hq, cfg.D), device=dev, dtype=torch.bfloat16)
+        olse = torch.empty((cfg.B, cfg.Hq), device=dev, dtype=torch.float32)
+        fn = lambda: ra.ring_attn_merge(part, plse, out=out, out_lse=olse)
+        work, unit = merge_bytes(cfg) / 1e9, "GB/s"
     else:
         q, k, v, sl = W.decode_inputs(cfg, dev)
         lens = sl.cpu().numpy().astype(np.int64)
@@ -616,6 +679,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward timing after the main region")
     ap.add_argument("--no-step", action="store_true", help="skip the step-API timing after the main region")
+    ap.add_argument("--no-merge", action="store_true", help="skip the merge-only timing after the main region")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)

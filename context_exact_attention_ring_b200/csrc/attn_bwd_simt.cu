@@ -54,6 +54,58 @@ __global__ void bwd_delta_kernel(const T* __restrict__ out, const T* __restrict_
   if (lane == 0) delta[((size_t)b * Hq + h) * S + i] = acc;
 }
 
+// The same rowsum, HBM-bound, for D*sizeof(T) a multiple of 16 bytes: a warp
+// takes 32 consecutive rows of delta's own [B, Hq, S] order (so its result
+// leaves as one coalesced 128-byte store); LPR lanes share a row, each loading
+// 16 bytes of out and of dout, and the warp covers 32 / LPR rows per
+// iteration.  The iterations are unrolled so every lane has several
+// independent loads in flight.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) bwd_delta_vec_kernel(const T* __restrict__ out, const T* __restrict__ dout,
+                                                            float* __restrict__ delta, int B, int Hq, int S) {
+  constexpr int EPV = 16 / (int)sizeof(T);   // elements per 16-byte load
+  constexpr int LPR = D / EPV;               // lanes per row
+  constexpr int RPI = 32 / LPR;              // rows per warp iteration
+  static_assert(D % EPV == 0 && LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "unsupported row size");
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)B * Hq * S;
+  const long long r0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32;
+  if (r0 >= nrows) return;
+  const int sub = lane / LPR, part = lane % LPR;
+  // position of row r0 in (b*Hq + h, i) form; later rows advance i and wrap
+  const long long bh0 = r0 / S;
+  const int i0 = (int)(r0 - bh0 * S);
+  float mine = 0.f;
+#pragma unroll
+  for (int it = 0; it < LPR; ++it) {
+    const int k = it * RPI + sub;   // row r0 + k
+    float acc = 0.f;
+    if (r0 + k < nrows) {
+      long long bh = bh0;
+      int i = i0 + k;
+      while (i >= S) {
+        i -= S;
+        ++bh;
+      }
+      const long long b = bh / Hq;
+      const int h = (int)(bh - b * Hq);
+      const size_t off = (((size_t)b * S + i) * Hq + h) * D + (size_t)part * EPV;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(out + off));
+      const uint4 g = __ldg(reinterpret_cast<const uint4*>(dout + off));
+      const T* av = reinterpret_cast<const T*>(&a);
+      const T* gv = reinterpret_cast<const T*>(&g);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) acc = fmaf(bld(av + e), bld(gv + e), acc);
+    }
+#pragma unroll
+    for (int o = LPR / 2; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    // every lane of group `sub` now holds row k's sum; lane L collects row L
+    const float v = __shfl_sync(0xffffffffu, acc, (lane % RPI) * LPR);
+    if (lane / RPI == it) mine = v;
+  }
+  if (r0 + lane < nrows) delta[r0 + lane] = mine;
+}
+
 // S = Q K^T and dP = dO V^T for a 64 x 64 tile: thread (ty, tx) owns rows
 // ty + 16*ii and keys tx + 16*jj; writes P and dS to shared memory.
 template <int D>
@@ -295,8 +347,25 @@ static cudaError_t launch_bwd_t(const Plan& p, const BwdArgs& a, cudaStream_t st
 cudaError_t launch_bwd_delta(const void* out, const void* dout, float* delta, int B, int Hq, int S, int D, bool bf16,
                              cudaStream_t st) {
   const long long rows = (long long)B * S * Hq;
-  const int per = 8;   // warps (rows) per block
-  const long long blocks = (rows + per - 1) / per;
+  const int per = 8;   // warps per block
+  if (D == 64 || D == 128) {
+    const long long blocks = (rows + 32LL * per - 1) / (32LL * per);   // 32 rows per warp
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const unsigned nb = (unsigned)blocks;
+    if (bf16) {
+      auto o = static_cast<const __nv_bfloat16*>(out);
+      auto g = static_cast<const __nv_bfloat16*>(dout);
+      if (D == 128) bwd_delta_vec_kernel<__nv_bfloat16, 128><<<nb, 32 * per, 0, st>>>(o, g, delta, B, Hq, S);
+      else bwd_delta_vec_kernel<__nv_bfloat16, 64><<<nb, 32 * per, 0, st>>>(o, g, delta, B, Hq, S);
+    } else {
+      auto o = static_cast<const float*>(out);
+      auto g = static_cast<const float*>(dout);
+      if (D == 128) bwd_delta_vec_kernel<float, 128><<<nb, 32 * per, 0, st>>>(o, g, delta, B, Hq, S);
+      else bwd_delta_vec_kernel<float, 64><<<nb, 32 * per, 0, st>>>(o, g, delta, B, Hq, S);
+    }
+    return cudaGetLastError();
+  }
+  const long long blocks = (rows + per - 1) / per;   // one warp per row
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   if (bf16)
     bwd_delta_kernel<__nv_bfloat16><<<(unsigned)blocks, 32 * per, 0, st>>>(

@@ -55,7 +55,11 @@ namespace tb {
 constexpr int THREADS = 384;
 constexpr int SLAB = 128 * 64 * 2;      // one 128-row x 64-column bf16 box
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int REG_LOW = 96, REG_HIGH = 184;
+// Register split: 120 for the producer / MMA warpgroup (96 made the K/V-major
+// launch spill there), 184 for the elementwise warpgroups.  128*120 + 256*184 =
+// 62,464 must not exceed 384 threads x the registers a thread is launched with
+// (the launcher checks REG_NEED against the built kernel before every launch).
+constexpr int REG_LOW = 120, REG_HIGH = 184;
 constexpr int REG_NEED = (128 * REG_LOW + 256 * REG_HIGH + THREADS - 1) / THREADS;
 }  // namespace tb
 

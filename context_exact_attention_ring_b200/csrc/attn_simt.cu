@@ -247,13 +247,40 @@ cudaError_t launch_state_finalize(const float* m, const float* l, const float* O
 }
 
 // ---------------------------------------------------------------------------
-// (O, lse) merge: one warp per (b, hq); lanes own 4 consecutive dims at a
-// time (128-bit loads, coalesced across the warp).
+// (O, lse) merge, HBM-bound: one warp per (b, hq) row.  Lane j computes the
+// weight e^(lse_p - lse) of parts p = j, j+32, ... once per block of 32 parts
+// and the accumulation loop broadcasts it by shuffle.  Lanes own 4
+// consecutive dims (one 16-byte load per part, a warp reads 512 contiguous
+// bytes of a part), and kUnroll parts are loaded before any is used, so each
+// lane keeps kUnroll independent loads in flight.  A part whose weight is 0
+// (an empty part, lse = -inf) is not read.  The output row leaves as one
+// vector store per lane.
 // ---------------------------------------------------------------------------
+namespace merge {
+constexpr int kUnroll = 8;
+}
+
+__device__ __forceinline__ void st_vec4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void st_vec4(__nv_bfloat16* p, float4 v) {
+  uint2 w;
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  w.x = *reinterpret_cast<uint32_t*>(&lo);
+  w.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p) = w;
+}
+
+__device__ __forceinline__ void fma4(float w, const float4& x, float4& acc) {
+  acc.x = fmaf(w, x.x, acc.x);
+  acc.y = fmaf(w, x.y, acc.y);
+  acc.z = fmaf(w, x.z, acc.z);
+  acc.w = fmaf(w, x.w, acc.w);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) merge_kernel(const float* __restrict__ part, const float* __restrict__ plse,
                                                     T* __restrict__ out, float* __restrict__ out_lse, int n_rows,
                                                     int P, int D) {
+  using merge::kUnroll;
   const int w = (int)(((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= n_rows) return;
@@ -270,22 +297,36 @@ __global__ void __launch_bounds__(256) merge_kernel(const float* __restrict__ pa
   for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   const float inv_z = live ? 1.f / z : 0.f;
   const float* Ob = part + (size_t)w * P * D;
-  for (int d0 = lane * 4; d0 < D; d0 += 128) {
+  for (int d0 = 0; d0 < D; d0 += 128) {
+    const int d = d0 + lane * 4;
+    const bool mine = d < D;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < P; ++i) {
-      const float wt = expf(L[i] - base) * inv_z;
-      if (wt == 0.f) continue;
-      const float4 x = __ldg(reinterpret_cast<const float4*>(Ob + (size_t)i * D + d0));
-      acc.x = fmaf(wt, x.x, acc.x);
-      acc.y = fmaf(wt, x.y, acc.y);
-      acc.z = fmaf(wt, x.z, acc.z);
-      acc.w = fmaf(wt, x.w, acc.w);
+    for (int c = 0; c < P; c += 32) {
+      const int nb = min(32, P - c);
+      const float wt = lane < nb ? expf(L[c + lane] - base) * inv_z : 0.f;
+      const float* src = Ob + (size_t)c * D + d;
+      int j = 0;
+      for (; j + kUnroll <= nb; j += kUnroll) {
+        float wj[kUnroll];
+        float4 x[kUnroll];
+if (mine) {
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) x[u] = __ldg(reinterpret_cast<const float4*>(src + (size_t)(j + u) * D));
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) wj[u] = __shfl_sync(0xffffffffu, wt, j + u);
+        if (mine) {
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u)
+            if (wj[u] != 0.f) fma4(wj[u], x[u], acc);   // an empty part's O may hold anything
+        }
+      }
+      for (; j < nb; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, wt, j);
+        if (mine && wj != 0.f) fma4(wj, __ldg(reinterpret_cast<const float4*>(src + (size_t)j * D)), acc);
+      }
     }
-    T* o = out + (size_t)w * D + d0;
-    st_val(o + 0, acc.x);
-    st_val(o + 1, acc.y);
-    st_val(o + 2, acc.z);
-    st_val(o + 3, acc.w);
+    if (mine) st_vec4(out + (size_t)w * D + d, acc);
   }
   if (lane == 0 && out_lse) out_lse[w] = live ? mx + logf(z) : -CUDART_INF_F;
 }

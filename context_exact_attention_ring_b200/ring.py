@@ -113,7 +113,13 @@ def ring_backward(q_shard, k_block, v_block, out_shard, lse_shard, dout_shard, l
                   scale=None, ring=None, step=None, delta_fn=None):
     """Gradients (dq, dk, dv) of this rank's shard.  dK, dV of a block are
     summed by every rank it visits, then sent home.  float32 sums; the results
-    take the dtype of q."""
+    take the dtype of q.
+
+    A block's running sums travel one hop behind it: at step t this rank
+    computes its own contribution to the block it holds into a fresh buffer
+    while the sums the previous ranks made for that block arrive from rank
+    r-1; it then adds the two and sends them on to rank r+1, where they arrive
+    during the next step.  Only the last hop home is not hidden behind a step."""
     from . import ring_attn_bwd_delta, ring_attn_step_bwd
     ring = ring or Ring()
     step = step or ring_attn_step_bwd
@@ -128,21 +134,35 @@ def ring_backward(q_shard, k_block, v_block, out_shard, lse_shard, dout_shard, l
     # as in ring_forward: the caller's block is only sent; received blocks alternate between two
     # buffers of the loop's own
     kv_bufs = [[torch.empty_like(x) for x in kv] for _ in range(min(2, P - 1))]
-    gr = [torch.zeros(k_block.shape, **f32), torch.zeros(v_block.shape, **f32)]
-    gr_nxt = [torch.empty_like(x) for x in gr]
+    # this step's contribution to the held block's dK, dV (two buffers: the one sent at step t is
+    # not touched before that send has completed, at step t+1), and the sums arriving for it
+    mine = [[torch.empty(k_block.shape, **f32), torch.empty(v_block.shape, **f32)] for _ in range(min(2, P))]
+    g_in = [torch.empty(k_block.shape, **f32), torch.empty(v_block.shape, **f32)]
+    g_reqs = []
     for t in range(P):
         src = (r - t) % P
         kv_nxt = kv_bufs[t % 2] if t < P - 1 else None
         reqs = ring.shift(kv, kv_nxt) if t < P - 1 else []   # the next block arrives during the step
-        step(q_shard, kv[0], kv[1], dout_shard, lse_shard, delta, dq, gr[0], gr[1], own[r], own[src], C,
+        g = mine[t % 2]
+        g[0].zero_()
+        g[1].zero_()
+        step(q_shard, kv[0], kv[1], dout_shard, lse_shard, delta, dq, g[0], g[1], own[r], own[src], C,
              causal=causal, scale=scale, stripes=stripes)
-        reqs += ring.shift(gr, gr_nxt)                        # this block's sums follow it (home after step P-1)
-        _wait(reqs)
+        if t > 0:
+            _wait(g_reqs)                  # the sums of this block from the ranks it visited before
+            g[0].add_(g_in[0])
+            g[1].add_(g_in[1])
         if P > 1:
-            gr, gr_nxt = gr_nxt, gr
-            if t < P - 1:
-                kv = kv_nxt
-    return dq.to(q_shard.dtype), gr[0].to(k_block.dtype), gr[1].to(v_block.dtype)
+            # the block's sums follow it to rank r+1 (home after step P-1); the sums of the block
+            # held at step t+1 come from rank r-1
+            g_reqs = ring.shift(g, g_in)
+        _wait(reqs)
+        if t < P - 1:
+            kv = kv_nxt
+    if P > 1:
+        _wait(g_reqs)                      # this rank's own block, summed by every rank
+        g = g_in
+    return dq.to(q_shard.dtype), g[0].to(k_block.dtype), g[1].to(v_block.dtype)
 
 
 class RingAttention(torch.autograd.Function):
@@ -175,7 +195,7 @@ def ring_attention(q_shard, k_block, v_block, layout="zigzag", causal=True, scal
     return RingAttention.apply(q_shard, k_block, v_block, layout, causal, scale, ring, fwd_kw, bwd_kw)
 
 
-def helix_decode(q, k_shard, v_shard, shard_len, scale=None, group=None, partial=None, merge=None):
+def helix_decode(q, k_shard, v_shard, shard_len, scale=None, group=None, partial=None, merge=None, gather=None):
     """Split-KV single-token decode across GPUs ("NVIDIA unveils Helix
     Parallelism", Phase 1, KV parallelism): rank r holds shard r of every
     sequence's KV cache and computes, over its shard, the normalised partial
@@ -190,7 +210,8 @@ def helix_decode(q, k_shard, v_shard, shard_len, scale=None, group=None, partial
     O_r = 0.  Returns (out [B, Hq, D], lse [B, Hq]), the same on every rank.
     The step functions default to this package's kernels (the decode over one
     chunk, and the merge) and can be replaced (tests run the exchange on CPU
-    ranks with stand-ins)."""
+    ranks with stand-ins).  gather(t) returns every rank's t in rank order; it
+    defaults to one all_gather over `group`."""
     from . import ring_attn_decode_partial, ring_attn_merge
     if partial is None:
         def partial(q_, k_, v_, lens_, scale_):
@@ -198,11 +219,13 @@ def helix_decode(q, k_shard, v_shard, shard_len, scale=None, group=None, partial
     if merge is None:
         def merge(parts_, lses_):
             return ring_attn_merge(parts_, lses_, dtype=q.dtype)
-    world = dist.get_world_size(group)
+    if gather is None:
+        def gather(t):
+            got = [torch.empty_like(t) for _ in range(dist.get_world_size(group))]
+            dist.all_gather(got, t, group=group)
+            return got
     part, plse = partial(q, k_shard, v_shard, shard_len, scale)          # [B, Hq, 1, D], [B, Hq, 1]
     B, Hq, D = part.shape[0], part.shape[1], part.shape[-1]
     mine = torch.cat([part.reshape(B, Hq, D), plse.reshape(B, Hq, 1)], dim=-1).contiguous()
-    gathered = [torch.empty_like(mine) for _ in range(world)]
-    dist.all_gather(gathered, mine, group=group)
-    allp = torch.stack(gathered, dim=2)                                   # [B, Hq, P, D + 1]
+    allp = torch.stack(gather(mine), dim=2)                               # [B, Hq, P, D + 1]
     return merge(allp[..., :D].contiguous(), allp[..., D].contiguous())

@@ -10,6 +10,24 @@ TOL_BF16_OUT = 2e-2      # bf16 in / fp32 accumulate: out (after the bf16 roundi
 TOL_BF16_LSE = 1e-3      # bf16 path: lse
 
 
+# Every parity check made through margin() is recorded here; tests/conftest.py
+# prints the worst ratio of error to tolerance per check at the end of the run,
+# so a log shows the headroom of each configuration and not only pass / fail.
+MARGINS: list = []
+
+
+def margin(quantity: str, err, tol, what: str = "") -> float:
+    """Assert err <= tol for one parity check (max |gpu - reference| of
+    `quantity`) and record it under the running test's id."""
+    import os
+    err = float(err)
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0].replace("tests/", "")
+    name = test if (not what or what in test) else f"{test} {what}"
+    MARGINS.append((name, quantity, err, float(tol)))
+    assert err <= tol, f"{name}: max |{quantity} - reference| = {err:.3e} > {tol}"
+    return err
+
+
 def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
 
@@ -27,8 +45,8 @@ def check_rows(out, lse, rows, ref_out, ref_lse, tol_out, tol_lse, what=""):
     err_o = np.max(np.abs(o - ref_out))
     err_l = np.max(np.abs(l - ref_lse))
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(l)), what
-    assert err_o <= tol_out, f"{what}: max |out - oracle| = {err_o:.3e} > {tol_out}"
-    assert err_l <= tol_lse, f"{what}: max |lse - oracle| = {err_l:.3e} > {tol_lse}"
+    margin("out", err_o, tol_out, what)
+    margin("lse", err_l, tol_lse, what)
     return err_o, err_l
 
 

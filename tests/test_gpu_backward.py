@@ -10,7 +10,7 @@ import context_exact_attention_ring_b200 as ra
 import oracle
 import workloads as W
 from oracle import schedule as sch
-from tests.helpers import host, need_cuda
+from tests.helpers import margin, host, need_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +32,7 @@ def _check(grads, refs, tol, what):
         err = float(np.max(np.abs(host(x) - r)))
         bound = tol * max(1.0, float(np.max(np.abs(r))))
         assert np.all(np.isfinite(host(x))), f"{what} {name}"
-        assert err <= bound, f"{what}: max |{name} - oracle| = {err:.3e} > {bound:.3e}"
+        margin(name, err, bound, what)
 
 
 CASES = [
@@ -144,7 +144,7 @@ def test_tensor_core_backward_matches_cuda_cores(layout, S, P, Hq, Hkv, D):
     assert ra.ring_attn_device_error()[0] == ra.RING_OK
     for name, a, b in zip(("dq", "dk", "dv"), g1, g2):
         scale_ = max(1.0, b.float().abs().max().item())
-        assert (a.float() - b.float()).abs().max().item() <= TOL_BWD_BF16 * scale_, name
+        margin(str(name), (a.float() - b.float()).abs().max().item(), TOL_BWD_BF16 * scale_)
 
 
 def test_full_size_backward_sampled_rows_and_invariants():
@@ -164,7 +164,7 @@ def test_full_size_backward_sampled_rows_and_invariants():
     rows = np.array([r for r in W.sample_rows(cfg, 24) if r[1] in (0, 9, 22, 31)], dtype=np.int32)
     ref = oracle.attention_bwd_dq_rows(host(q), host(k), host(v), host(dout), rows, scale=cfg.scale, causal=True)
     got = host(dq)[rows[:, 0], rows[:, 2], rows[:, 1]]
-    assert np.max(np.abs(got - ref)) <= TOL_BWD_BF16 * max(1.0, float(np.max(np.abs(ref))))
+    margin("dq", np.max(np.abs(got - ref)), TOL_BWD_BF16 * max(1.0, float(np.max(np.abs(ref)))))
     G = cfg.Hq // cfg.Hkv
     dk64 = dk.double().sum(dim=1).cpu().numpy()                                  # [B, Hkv, D]
     dv64 = dv.double().sum(dim=1).cpu().numpy()
@@ -176,3 +176,29 @@ def test_full_size_backward_sampled_rows_and_invariants():
     rows_walk = lambda y: 4.0 * np.sqrt(cfg.S * G) * 2.0 ** -9 * float(y.float().pow(2).mean().sqrt().item())
     assert np.max(np.abs(dk64)) <= walk(dk) + cfg.scale * rows_walk(q) * 8.0
     assert np.max(np.abs(dv64 - do64)) <= walk(dv) + rows_walk(dout)
+
+
+@pytest.mark.parametrize("cfg", [
+    W.Prefill("autograd_bf16_zigzag_gqa", "bf16", True, "zigzag", 1, 8, 2, 2048, 128, 4, 621),
+    W.Prefill("autograd_bf16_striped_gqa", "bf16", True, "striped", 2, 4, 2, 1536, 128, 3, 622),
+    W.Prefill("autograd_fp32_zigzag_gqa", "fp32", True, "zigzag", 1, 4, 2, 1024, 64, 4, 623),
+    W.Prefill("autograd_fp32_striped", "fp32", True, "striped", 1, 2, 2, 768, 64, 3, 624),
+], ids=lambda c: c.name)
+def test_ring_attention_under_autograd_against_oracle(cfg):
+    # the training entry point: out = ring_attention(q, k, v, P) on leaf tensors, loss = sum(out * dout),
+    # loss.backward(); the leaves' gradients against the fp64 oracle
+    need_cuda()
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    dout = _dout(cfg, cfg.seed + 1)
+    lq, lk, lv = (x.clone().requires_grad_(True) for x in (q, k, v))
+    out = ra.ring_attention(lq, lk, lv, cfg.P, causal=cfg.causal, layout=cfg.layout, scale=cfg.scale)
+    (out.float() * dout.float()).sum().backward()
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    assert lq.grad.dtype == q.dtype and lk.grad.shape == k.shape and lv.grad.shape == v.shape
+    rows = oracle.all_rows(cfg.B, cfg.Hq, cfg.S)
+    ro, _ = oracle.attention_rows(host(q), host(k), host(v), rows, scale=cfg.scale, causal=cfg.causal)
+    ro = ro.reshape(cfg.B, cfg.Hq, cfg.S, cfg.D).transpose(0, 2, 1, 3)
+    margin("out", np.max(np.abs(host(out) - ro)), 1e-5 if cfg.dtype == "fp32" else 2e-2)
+    refs = oracle.attention_bwd(host(q), host(k), host(v), host(dout), scale=cfg.scale, causal=cfg.causal)
+    _check((lq.grad, lk.grad, lv.grad), refs, TOL_BWD_FP32 if cfg.dtype == "fp32" else TOL_BWD_BF16, cfg.name)

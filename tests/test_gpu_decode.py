@@ -8,7 +8,7 @@ import context_exact_attention_ring_b200 as ra
 import oracle
 import workloads as W
 from oracle import merge as omerge
-from tests.helpers import TOL_BF16_LSE, TOL_BF16_OUT, host, need_cuda
+from tests.helpers import margin, TOL_BF16_LSE, TOL_BF16_OUT, host, need_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -66,16 +66,16 @@ def test_decode_small(Hq, Hkv):
             if np.isneginf(rl):
                 assert np.isneginf(gl) and np.all(host(part)[b, h, p] == 0)
             else:
-                assert abs(gl - rl) <= TOL_BF16_LSE
-                assert np.max(np.abs(host(part)[b, h, p] - ro)) <= TOL_BF16_OUT
+                margin("lse", abs(gl - rl), TOL_BF16_LSE)
+                margin("out", np.max(np.abs(host(part)[b, h, p] - ro)), TOL_BF16_OUT)
     # merged result: attention over all valid keys
     ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale)
     for (b, h), ro in ref_o.items():
         if lens[b] == 0:
             assert np.isneginf(host(out_lse)[b, h]) and np.all(host(out)[b, h] == 0)
             continue
-        assert abs(host(out_lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
-        assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+        margin("lse", abs(host(out_lse)[b, h] - ref_l[(b, h)]), TOL_BF16_LSE)
+        margin("out", np.max(np.abs(host(out)[b, h] - ro)), TOL_BF16_OUT)
     # the arrival counters are back at zero: a second call on the same workspace agrees
     out2, lse2 = ra.ring_attn_decode(q, k, v, sl, P, cfg.scale, workspace=ws)
     torch.cuda.synchronize()
@@ -105,8 +105,8 @@ def test_decode_ignores_rows_past_the_length(fused):
     assert np.all(np.isfinite(host(out))) and np.all(np.isfinite(host(out_lse)))
     ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale)
     for (b, h), ro in ref_o.items():
-        assert abs(host(out_lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
-        assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+        margin("lse", abs(host(out_lse)[b, h] - ref_l[(b, h)]), TOL_BF16_LSE)
+        margin("out", np.max(np.abs(host(out)[b, h] - ro)), TOL_BF16_OUT)
 
 
 @pytest.mark.parametrize("Hq,Hkv,P", [(8, 2, 3), (16, 2, 1)])
@@ -126,8 +126,8 @@ def test_decode_head_dim_64(Hq, Hkv, P, fused):
     assert ra.ring_attn_device_error()[0] == ra.RING_OK
     ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale)
     for (b, h), ro in ref_o.items():
-        assert abs(host(out_lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
-        assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+        margin("lse", abs(host(out_lse)[b, h] - ref_l[(b, h)]), TOL_BF16_LSE)
+        margin("out", np.max(np.abs(host(out)[b, h] - ro)), TOL_BF16_OUT)
 
 def test_merge_kernel_against_oracle_formula():
     need_cuda()
@@ -141,10 +141,46 @@ def test_merge_kernel_against_oracle_formula():
         out, lse = ra.ring_attn_merge(part, plse, dtype=dt)
         ro, rl = omerge.merge(host(part), host(plse))
         tol = 1e-5 if dt == torch.float32 else TOL_BF16_OUT
-        assert np.max(np.abs(host(out) - ro)) <= tol
+        margin("out", np.max(np.abs(host(out) - ro)), tol)
         fin = np.isfinite(rl)
         assert np.max(np.abs(host(lse)[fin] - rl[fin])) <= 1e-5
         assert np.all(np.isneginf(host(lse)[~fin]))
+
+
+@pytest.mark.parametrize("P,D", [(1, 128), (7, 64), (32, 128), (37, 96), (100, 128)])
+def test_merge_part_counts_head_sizes_and_nan_in_empty_parts(P, D):
+    # part counts around the kernel's 32-part weight blocks and 8-deep load batches, head sizes
+    # that leave lanes idle (64, 96 dims for 32 lanes of 4), and empty parts (lse = -inf) whose O
+    # holds NaN: an empty part must not enter the sum whatever its O holds.  The oracle gets the
+    # same parts with those O set to zero (what the decode writes for an empty chunk).
+    need_cuda()
+    mc = W.Merge(f"merge_P{P}_D{D}", 3, 5, P, D, 72 + P, empty_frac=0.3)
+    part, plse = W.merge_inputs(mc, "cuda")
+    plse[1, 2, :] = float("-inf")            # one row with every part empty
+    part[1, 2] = float("nan")
+    ref_part = torch.nan_to_num(part, nan=0.0)
+    ro, rl = omerge.merge(host(ref_part), host(plse))
+    for dt in (torch.float32, torch.bfloat16):
+        out, lse = ra.ring_attn_merge(part, plse, dtype=dt)
+        torch.cuda.synchronize()
+        assert np.all(np.isfinite(host(out)))
+        margin("out", np.max(np.abs(host(out) - ro)), 1e-5 if dt == torch.float32 else TOL_BF16_OUT, str(dt))
+        fin = np.isfinite(rl)
+        margin("lse", np.max(np.abs(host(lse)[fin] - rl[fin])), 1e-5, str(dt))
+        assert np.all(np.isneginf(host(lse)[~fin])) and np.all(host(out)[~fin] == 0)
+
+
+def test_merge_only_workload_every_row():
+    # the merge alone at the size bench.py times (B*Hq = 8192 rows, P = 32, D = 128, 134 MB of
+    # partials), every row against the merge formula
+    need_cuda()
+    mc = W.MERGE_ONLY
+    part, plse = W.merge_inputs(mc, "cuda")
+    out, lse = ra.ring_attn_merge(part, plse, dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ro, rl = omerge.merge(host(part), host(plse))
+    margin("out", np.max(np.abs(host(out) - ro)), TOL_BF16_OUT)
+    margin("lse", np.max(np.abs(host(lse) - rl)), 1e-5)
 
 
 def test_cfg5_full_size_sampled():

@@ -9,7 +9,7 @@ import torch
 import context_exact_attention_ring_b200 as ra
 import workloads as W
 from oracle import merge as omerge
-from tests.helpers import TOL_BF16_LSE, TOL_BF16_OUT, TOL_FP32, check_rows, host, need_cuda, oracle_rows
+from tests.helpers import margin, TOL_BF16_LSE, TOL_BF16_OUT, TOL_FP32, check_rows, host, need_cuda, oracle_rows
 from tests.test_gpu_decode import oracle_decode
 from tests.test_gpu_simt import ring_by_steps
 
@@ -60,8 +60,8 @@ def test_decode_lengths_out_of_range_are_clamped():
         if eff[b] == 0:
             assert np.isneginf(host(lse)[b, h]) and np.all(host(out)[b, h] == 0)
         else:
-            assert abs(host(lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
-            assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+            margin("lse", abs(host(lse)[b, h] - ref_l[(b, h)]), TOL_BF16_LSE)
+            margin("out", np.max(np.abs(host(out)[b, h] - ro)), TOL_BF16_OUT)
 
 
 @pytest.mark.parametrize("cap,P,lens", [
@@ -83,8 +83,8 @@ def test_decode_partials_odd_chunks(cap, P, lens):
             if np.isneginf(rl):
                 assert np.isneginf(host(plse)[b, h, p])
             else:
-                assert abs(host(plse)[b, h, p] - rl) <= TOL_BF16_LSE
-                assert np.max(np.abs(host(part)[b, h, p] - ro)) <= TOL_BF16_OUT
+                margin("lse", abs(host(plse)[b, h, p] - rl), TOL_BF16_LSE)
+                margin("out", np.max(np.abs(host(part)[b, h, p] - ro)), TOL_BF16_OUT)
 
 
 def test_merge_single_part_is_identity():
@@ -94,6 +94,6 @@ def test_merge_single_part_is_identity():
     plse = torch.randn((2, 3, 1), generator=g, device="cuda")
     out, lse = ra.ring_attn_merge(part, plse, dtype=torch.float32)
     ro, rl = omerge.merge(host(part), host(plse))
-    assert np.max(np.abs(host(out) - ro)) <= TOL_FP32
-    assert np.max(np.abs(host(lse) - rl)) <= TOL_FP32
+    margin("out", np.max(np.abs(host(out) - ro)), TOL_FP32)
+    margin("lse", np.max(np.abs(host(lse) - rl)), TOL_FP32)
     np.testing.assert_allclose(host(out), host(part)[:, :, 0], atol=TOL_FP32)

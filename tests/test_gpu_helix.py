@@ -12,7 +12,7 @@ import context_exact_attention_ring_b200 as ra
 import oracle
 import workloads as W
 from oracle import helix
-from tests.helpers import TOL_BF16_LSE, TOL_BF16_OUT, host, need_cuda
+from tests.helpers import margin, TOL_BF16_LSE, TOL_BF16_OUT, host, need_cuda
 from tests.test_gpu_decode import oracle_decode
 
 pytestmark = pytest.mark.gpu
@@ -101,8 +101,8 @@ def _fused_vs_oracle(q, k, v, sl, P, scale, lens):
         if np.isneginf(ref_l[(b, h)]):
             assert np.isneginf(lh[b, h]) and not oh[b, h].any()
         else:
-            assert abs(lh[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
-            assert np.max(np.abs(oh[b, h] - ro)) <= TOL_BF16_OUT
+            margin("lse", abs(lh[b, h] - ref_l[(b, h)]), TOL_BF16_LSE)
+            margin("out", np.max(np.abs(oh[b, h] - ro)), TOL_BF16_OUT)
     return out, lse
 
 
@@ -152,8 +152,8 @@ def test_fused_decode_full_size_sampled():
     lens = host(sl).astype(int)
     ref_o, ref_l = oracle_decode(q, k, v, lens, cfg.scale, heads=heads)
     for (b, h), ro in ref_o.items():
-        assert abs(host(lse)[b, h] - ref_l[(b, h)]) <= TOL_BF16_LSE
-        assert np.max(np.abs(host(out)[b, h] - ro)) <= TOL_BF16_OUT
+        margin("lse", abs(host(lse)[b, h] - ref_l[(b, h)]), TOL_BF16_LSE)
+        margin("out", np.max(np.abs(host(out)[b, h] - ro)), TOL_BF16_OUT)
 
 
 @pytest.mark.parametrize("P,block,steps,T", [(4, 8, 6, 7), (8, 32, 3, 50), (2, 1, 5, 3)])
@@ -199,5 +199,5 @@ def test_decode_after_round_robin_appends(P, block, steps, T):
             o, l = oracle.attention_rows(qq, ks[:, :, gk:gk + 1], vs[:, :, gk:gk + 1],
                                          [(0, h, 0) for h in range(G)], scale=scale, causal=False)
             for h in range(G):
-                assert abs(host(lse)[b, gk * G + h] - l[h]) <= TOL_BF16_LSE
-                assert np.max(np.abs(host(out)[b, gk * G + h] - o[h])) <= TOL_BF16_OUT
+                margin("lse", abs(host(lse)[b, gk * G + h] - l[h]), TOL_BF16_LSE)
+                margin("out", np.max(np.abs(host(out)[b, gk * G + h] - o[h])), TOL_BF16_OUT)

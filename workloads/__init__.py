@@ -83,6 +83,18 @@ class Decode:
         return self.capacity // self.P
 
 
+@dataclass(frozen=True)
+class Merge:
+    """The (O, lse) merge alone: B*Hq rows of P normalised partials of D dims."""
+    name: str
+    B: int
+    Hq: int
+    P: int
+    D: int
+    seed: int
+    empty_frac: float = 0.0   # share of parts with lse = -inf (their O is filled with NaN)
+
+
 # The five workloads of the hot path.
 CFG1 = Prefill("ring_fp32_noncausal_B1_H2_S256_D64_P4", "fp32", False, "contiguous", 1, 2, 2, 256, 64, 4, 1)
 CFG2 = Prefill("ring_bf16_causal_contiguous_B1_H8_S8192_D128_P8", "bf16", True, "contiguous", 1, 8, 8, 8192, 128, 8, 2)
@@ -92,6 +104,9 @@ CFG4 = Prefill("ring_bf16_causal_zigzag_gqa_B1_Hq32_Hkv8_S131072_D128_P16", "bf1
                sample_rows=256)
 CFG5 = Decode("decode_splitkv_bf16_B8_Hq32_Hkv8_D128_ctx1M_P32", 8, 32, 8, 128, 1 << 20, 32, 5)
 CONFIGS = {c.name: c for c in (CFG1, CFG2, CFG3, CFG4, CFG5)}
+# The merge of workload 5's partials on its own, at a size that is HBM-bound
+# (134 MB of partials, above the 126 MB L2): B*Hq = 8192 rows, P = 32, D = 128.
+MERGE_ONLY = Merge("merge_fp32parts_bf16out_BHq8192_P32_D128", 256, 32, 32, 128, 6)
 
 
 def _dtype(name: str):
@@ -174,3 +189,19 @@ def decode_inputs(cfg: Decode, device="cpu"):
         v[b] = randn((cfg.capacity, cfg.Hkv, cfg.D), gen, device, torch.bfloat16)
     lens = decode_lengths(cfg).to(device)
     return q, k, v, lens
+
+
+def merge_inputs(cfg: Merge, device="cpu"):
+    """partials [B,Hq,P,D] float32 N(0,1) and part_lse [B,Hq,P] float32
+    N(0,1)*4.  With empty_frac > 0 that share of parts (seeded) gets
+    lse = -inf and an O of NaN: an empty part must contribute nothing,
+    whatever its O holds."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(cfg.seed)
+    part = torch.randn((cfg.B, cfg.Hq, cfg.P, cfg.D), generator=gen, device=device, dtype=torch.float32)
+    plse = torch.randn((cfg.B, cfg.Hq, cfg.P), generator=gen, device=device, dtype=torch.float32) * 4
+    if cfg.empty_frac > 0:
+        empty = torch.rand((cfg.B, cfg.Hq, cfg.P), generator=gen, device=device) < cfg.empty_frac
+        plse[empty] = float("-inf")
+        part[empty] = float("nan")
+    return part, plse
