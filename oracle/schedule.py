@@ -11,8 +11,8 @@ Sources (each function cites the passage it follows):
     r and 2P-1-r; the worked example also gives the sequential assignment of
     k consecutive chunks per rank.
   * same lesson, section 4 and the worked example: under the causal mask,
-    query chunk q attends K/V chunks 0..q, so a rank's workload is the sum of
-    (q + 1) over its query chunks.
+    query chunk q attends K/V chunks 0..q; a rank's workload is counted here
+    by walking its ring loop pair by pair (per_rank_pairs).
   * same lesson, code exercise: the general zig-zag rule for k chunks per rank
     (even slots count up from the front, odd slots down from the back).
   * "Sequence parallelism and ring attention", outlook: names the striped
@@ -47,29 +47,57 @@ def parse_layout(layout: str) -> tuple[str, int]:
     return name, k
 
 
-def sequential_assignment(P: int, chunks_per_rank: int) -> dict[int, list[int]]:
-    """Rank r owns chunks r*k .. r*k + k - 1 (worked example, sequential)."""
-    return {r: [r * chunks_per_rank + c for c in range(chunks_per_rank)] for r in range(P)}
+def _front_bands(k: int) -> int:
+    """Zig-zag split: the sequence of P*k chunks is read as k bands of P
+    consecutive chunks.  The first ceil(k/2) bands are dealt front to back in
+    order of rank; the others are mirrored (rank 0 takes the band's last
+    chunk), which is section 4B's pairing of an early chunk with a late one."""
+    return (k + 1) // 2
 
 
-def zigzag_assignment(P: int, chunks_per_rank: int = 2) -> dict[int, list[int]]:
-    """Zig-zag ownership (section 4B; general k from the code exercise).
+def chunk_owner(c: int, P: int, layout: str) -> int:
+    """Rank that owns global chunk c.
 
-    Slot c of rank r: even c takes chunk (c/2)*P + r, counting from the front;
-    odd c takes chunk total-1-(c//2)*P-r, counting from the back.  For k = 2
-    this is {r, 2P-1-r}.
+    Contiguous split (section 4A; k chunks per rank: the worked example's
+    sequential assignment): chunks r*k .. r*k+k-1 belong to rank r.  Zig-zag
+    split (section 4B; k per rank: the code exercise's rule, restated by
+    bands): chunk c sits in band c // P at place c mod P; a front band gives
+    it to rank (c mod P), a back band to rank P-1-(c mod P).  Striped split:
+    the one "chunk" of rank r is its stripe, numbered r.
     """
-    total = P * chunks_per_rank
-    out = {}
-    for r in range(P):
-        owned = []
-        for c in range(chunks_per_rank):
-            if c % 2 == 0:
-                owned.append((c // 2) * P + r)
-            else:
-                owned.append(total - 1 - (c // 2) * P - r)
-        out[r] = owned
-    return out
+    name, k = parse_layout(layout)
+    if name == "contiguous":
+        return c // k
+    if name == "striped":
+        return c
+    band, place = divmod(c, P)
+    return place if band < _front_bands(k) else P - 1 - place
+
+
+def layout_assignment(P: int, layout: str) -> dict[int, list[int]]:
+    """Chunks owned by each rank, in the rank's slot order.
+
+    Contiguous: ascending.  Zig-zag: the rank's chunk of the first front band,
+    then of the last back band, then of the second front band, of the
+    next-to-last back band, and so on (slot 2i from the front, slot 2i+1 from
+    the back: section 4B and the code exercise).  For 'striped' the one
+    "chunk" of rank r is its stripe, numbered r.  Every chunk's owner comes
+    from chunk_owner; this only fixes the order in which a rank lists them.
+    """
+    name, k = parse_layout(layout)
+    if name == "striped":
+        return {r: [r] for r in range(P)}
+    if name == "contiguous":
+        order = list(range(P * k))
+    else:
+        fronts = list(range(_front_bands(k)))
+        backs = list(range(k - 1, _front_bands(k) - 1, -1))
+        bands = [b for i in range(len(fronts)) for b in fronts[i:i + 1] + backs[i:i + 1]]
+        order = [c for b in bands for c in range(b * P, (b + 1) * P)]
+    held: dict[int, list[int]] = {r: [] for r in range(P)}
+    for c in order:
+        held[chunk_owner(c, P, layout)].append(c)
+    return held
 
 
 def striped_tokens(S: int, P: int) -> dict[int, list[int]]:
@@ -79,19 +107,6 @@ def striped_tokens(S: int, P: int) -> dict[int, list[int]]:
     attention", outlook.
     """
     return {r: list(range(r, S, P)) for r in range(P)}
-
-
-def layout_assignment(P: int, layout: str) -> dict[int, list[int]]:
-    """Chunks owned by each rank: 'contiguous' (section 4A; with k chunks per
-    rank the sequential assignment), 'zigzag' (section 4B; k per rank from the
-    code exercise).  For 'striped' the one "chunk" of rank r is its stripe,
-    numbered r."""
-    name, k = parse_layout(layout)
-    if name == "contiguous":
-        return sequential_assignment(P, k)
-    if name == "zigzag":
-        return zigzag_assignment(P, k)
-    return {r: [r] for r in range(P)}
 
 
 def chunk_positions(S: int, P: int, layout: str) -> dict[int, list[int]]:
@@ -109,20 +124,15 @@ def chunk_positions(S: int, P: int, layout: str) -> dict[int, list[int]]:
     return {c: list(range(c * C, (c + 1) * C)) for c in range(n)}
 
 
-def causal_workload(assign: dict[int, list[int]]) -> dict[int, int]:
-    """Causal chunk pairs per rank: query chunk q sees K/V chunks 0..q, so the
-    rank's count is the number of (q, kv) chunk pairs with kv <= q (section 4).
-    Enumerated pair by pair rather than summed in closed form."""
-    n_chunks = sum(len(v) for v in assign.values())
-    return {r: sum(1 for q in qs for kv in range(n_chunks) if kv <= q) for r, qs in assign.items()}
+def block_sources(P: int, rank: int, start: int | None = None) -> list[int]:
+    """The rank whose K/V block rank ``rank`` holds at steps t = 0..P-1.
 
-
-def ring_rotation(P: int, rank: int, start: int | None = None) -> list[int]:
-    """Which rank's K/V block rank ``rank`` holds at steps t = 0..P-1: blocks
-    move from rank r-1 to rank r each step, so at step t it is the block that
-    started on rank (start - t) mod P (section 2; start defaults to rank)."""
-    s = rank if start is None else start
-    return [(s - t) % P for t in range(P)]
+    Section 2: every step each block moves on to the next rank, so at step t
+    a rank holds the block that began t hops behind it, i.e. on rank
+    (start - t) mod P (start defaults to the rank itself).
+    """
+    first = rank if start is None else start
+    return [(first - hop) % P for hop in range(P)]
 
 
 @dataclass(frozen=True)
@@ -147,7 +157,7 @@ def ring_pairs(P: int, layout: str, causal: bool, S: int | None = None) -> list[
     pos = chunk_positions(S, P, layout) if striped else None
     out = []
     for r in range(P):
-        for t, src in enumerate(ring_rotation(P, r)):
+        for t, src in enumerate(block_sources(P, r)):
             for qc in own[r]:
                 for kc in own[src]:
                     if striped:
@@ -241,4 +251,4 @@ def kv_visit_order(P: int, layout: str, rank: int) -> list[int]:
     Rotation of "Lesson 8", section 2.
     """
     own = layout_assignment(P, layout)
-    return [c for src in ring_rotation(P, rank) for c in own[src]]
+    return [c for src in block_sources(P, rank) for c in own[src]]

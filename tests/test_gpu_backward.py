@@ -113,7 +113,7 @@ def test_step_backward_ring(dtype, layout, S, P):
         qs, ds = q[:, rr].contiguous(), dout[:, rr].contiguous()
         ls, dl = lse[:, :, rr].contiguous(), delta[:, :, rr].contiguous()
         dq_r = torch.zeros((B, len(rr), Hq, D), device="cuda")
-        for src in sch.ring_rotation(P, r):
+        for src in sch.block_sources(P, r):
             kr = rows[src]
             ra.ring_attn_step_bwd(qs, k[:, kr].contiguous(), v[:, kr].contiguous(), ds, ls, dl, dq_r, dk_acc[src],
                                   dv_acc[src], own[r], own[src], C, causal=True, scale=cfg.scale, stripes=stripes)

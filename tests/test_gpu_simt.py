@@ -71,7 +71,7 @@ def ring_by_steps(q, k, v, P, layout, causal, scale, order_fn=None, checkpoint_a
         rows = torch.tensor([t for c in qc for t in pos[c]], device=q.device)
         qs = q[:, rows].contiguous()
         m, l, O = ra.new_state(B, Hq, len(rows), D)
-        srcs = sch.ring_rotation(P, r)
+        srcs = sch.block_sources(P, r)
         if order_fn is not None:
             srcs = order_fn(srcs)
         for t, src in enumerate(srcs):
@@ -124,7 +124,7 @@ def test_step_state_is_attention_over_seen_keys():
     qs = q[:, rows].contiguous()
     m, l, O = ra.new_state(cfg.B, cfg.Hq, C, cfg.D)
     seen = []
-    for src in sch.ring_rotation(cfg.P, r):
+    for src in sch.block_sources(cfg.P, r):
         krows = np.arange(src * C, (src + 1) * C)
         ra.ring_attn_step(qs, k[:, krows].contiguous(), v[:, krows].contiguous(), m, l, O, [r], [src], C,
                           causal=False, scale=cfg.scale)

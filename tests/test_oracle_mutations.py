@@ -92,13 +92,14 @@ MUTATIONS = [
     ("recurrence masks the diagonal", "streaming.py",
      "ks[None, :] <= qpos[:, None]", "ks[None, :] < qpos[:, None]", ATTN),
     # schedule.py: ownership, rotation and pair classes ("Lesson 8", sections 2 and 4)
-    ("zig-zag back chunk mirrored wrongly", "schedule.py",
-     "owned.append(total - 1 - (c // 2) * P - r)", "owned.append(total - 1 - (c // 2) * P - (P - 1 - r))",
-     SCHED),
+    ("zig-zag back band not mirrored", "schedule.py",
+     "return place if band < _front_bands(k) else P - 1 - place",
+     "return place if band < _front_bands(k) else place", SCHED),
     ("ring turns the wrong way", "schedule.py",
-     "return [(s - t) % P for t in range(P)]", "return [(s + t) % P for t in range(P)]", SCHED),
-    ("causal workload drops the diagonal", "schedule.py",
-     "for kv in range(n_chunks) if kv <= q)", "for kv in range(n_chunks) if kv < q)", SCHED),
+     "return [(first - hop) % P for hop in range(P)]", "return [(first + hop) % P for hop in range(P)]", SCHED),
+    ("causal walk drops the diagonal", "schedule.py",
+     'elif kc == qc:\n                        kind = "diag"',
+     'elif kc == qc:\n                        kind = "skip"', SCHED),
     ("diagonal pair classed as full", "schedule.py",
      "elif not causal or kc < qc:", "elif not causal or kc <= qc:", SCHED),
     ("striped split dealt contiguously", "schedule.py",

@@ -22,28 +22,31 @@ def _keys_int(d):
 
 def test_printed_assignments():
     P = GOLD["P"]
-    assert sch.sequential_assignment(P, 2) == _keys_int(GOLD["sequential_2_per_rank"])
-    assert sch.zigzag_assignment(P, 2) == _keys_int(GOLD["zigzag"])
+    assert sch.layout_assignment(P, "contiguous2") == _keys_int(GOLD["sequential_2_per_rank"])
+    assert sch.layout_assignment(P, "zigzag") == _keys_int(GOLD["zigzag"])
+    # the owner of every chunk agrees with the printed assignment
+    for r, cs in _keys_int(GOLD["zigzag"]).items():
+        assert all(sch.chunk_owner(c, P, "zigzag") == r for c in cs)
 
 
 def test_printed_workloads():
+    # causal chunk pairs per rank, counted by walking each rank's ring loop
     P = GOLD["P"]
-    ws = sch.causal_workload(sch.sequential_assignment(P, 2))
-    wz = sch.causal_workload(sch.zigzag_assignment(P, 2))
+    ws = dict(enumerate(sch.per_rank_pairs(P, "contiguous2", True)))
+    wz = dict(enumerate(sch.per_rank_pairs(P, "zigzag", True)))
     assert ws == _keys_int(GOLD["sequential_workload"])
     assert wz == _keys_int(GOLD["zigzag_workload"])
     assert max(ws.values()) / min(ws.values()) == GOLD["sequential_max_over_min"]
 
 
 def test_printed_rotation():
-    assert sch.ring_rotation(GOLD["P"], 2, 2) == GOLD["rank2_rotation"]
+    assert sch.block_sources(GOLD["P"], 2, 2) == GOLD["rank2_rotation"]
 
 
 @pytest.mark.parametrize("P", list(range(1, 33)))
 def test_zigzag_closed_form(P):
     # section 4B: every rank does (r+1) + (2P-r) = 2P+1 causal chunk pairs
     assert sch.per_rank_pairs(P, "zigzag", True) == [2 * P + 1] * P
-    assert list(sch.causal_workload(sch.zigzag_assignment(P, 2)).values()) == [2 * P + 1] * P
 
 
 @pytest.mark.parametrize("P", list(range(1, 17)))
@@ -103,11 +106,13 @@ def test_kv_visit_order_covers_all_chunks_once():
 # --------------------------------------------------------------------------- split variants
 @pytest.mark.parametrize("P,k", [(p, k) for p in (1, 2, 3, 4, 8) for k in (2, 3, 4, 5, 8)])
 def test_general_zigzag_is_a_partition(P, k):
-    own = sch.zigzag_assignment(P, k)
+    own = sch.layout_assignment(P, f"zigzag{k}")
     assert sorted(c for cs in own.values() for c in cs) == list(range(P * k))
-    # slot 0 counts up from the front, slot 1 down from the back (the section 4B pair for k = 2)
+    # the code exercise's slot rule, as printed: even slot 2i counts up from the front (chunk
+    # iP + r), odd slot 2i+1 down from the back (chunk kP - 1 - iP - r); for k = 2 the section
+    # 4B pair {r, 2P-1-r}
     for r in range(P):
-        assert own[r][0] == r and own[r][1] == P * k - 1 - r
+        assert own[r] == [(j // 2) * P + r if j % 2 == 0 else P * k - 1 - (j // 2) * P - r for j in range(k)]
 
 
 @pytest.mark.parametrize("P,k", [(p, k) for p in (1, 2, 3, 4, 8, 16) for k in (2, 4, 6, 8)])
@@ -115,7 +120,6 @@ def test_general_zigzag_even_k_balanced_closed_form(P, k):
     # slots 2i and 2i+1 hold chunks iP+r and (k-i)P-1-r: (iP+r+1) + ((k-i)P-r) = kP+1 pairs,
     # so each rank does (k/2)(kP+1) causal chunk pairs whatever its index
     expect = [(k // 2) * (k * P + 1)] * P
-    assert list(sch.causal_workload(sch.zigzag_assignment(P, k)).values()) == expect
     assert sch.per_rank_pairs(P, f"zigzag{k}", True) == expect
 
 
