@@ -258,6 +258,9 @@ cudaError_t launch_state_finalize(const float* m, const float* l, const float* O
 // ---------------------------------------------------------------------------
 namespace merge {
 constexpr int kUnroll = 8;
+// Small blocks (4 rows each): as blocks finish, the SMs are refilled a few
+// rows at a time, so the last partial wave of a large merge stays short.
+constexpr int kThreads = 128;
 }
 
 __device__ __forceinline__ void st_vec4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
@@ -277,7 +280,7 @@ __device__ __forceinline__ void fma4(float w, const float4& x, float4& acc) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) merge_kernel(const float* __restrict__ part, const float* __restrict__ plse,
+__global__ void __launch_bounds__(merge::kThreads) merge_kernel(const float* __restrict__ part, const float* __restrict__ plse,
                                                     T* __restrict__ out, float* __restrict__ out_lse, int n_rows,
                                                     int P, int D) {
   using merge::kUnroll;
@@ -334,11 +337,12 @@ if (mine) {
 cudaError_t launch_merge(const float* part, const float* plse, void* out, float* out_lse, int B, int Hq, int P,
                          int D, bool bf16, cudaStream_t st) {
   const int rows = B * Hq;
-  const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+  const unsigned blocks = (unsigned)(((size_t)rows * 32 + merge::kThreads - 1) / merge::kThreads);
   if (bf16)
-    merge_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(part, plse, (__nv_bfloat16*)out, out_lse, rows, P, D);
+    merge_kernel<__nv_bfloat16><<<blocks, merge::kThreads, 0, st>>>(part, plse, (__nv_bfloat16*)out, out_lse, rows,
+                                                                    P, D);
   else
-    merge_kernel<float><<<blocks, 256, 0, st>>>(part, plse, (float*)out, out_lse, rows, P, D);
+    merge_kernel<float><<<blocks, merge::kThreads, 0, st>>>(part, plse, (float*)out, out_lse, rows, P, D);
   return cudaGetLastError();
 }
 

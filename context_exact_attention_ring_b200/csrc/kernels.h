@@ -30,6 +30,8 @@ struct TcArgs {
   unsigned int* err;             // device error word
 };
 cudaError_t launch_attn_tc(const Plan& p, const TcArgs& a, cudaStream_t st);
+// The same on CTA pairs (tcgen05 cta_group::2, M = 256), D = 128 only.
+cudaError_t launch_attn_tc_pair(const Plan& p, const TcArgs& a, cudaStream_t st);
 
 // Backward (CUDA cores).  Ring mode writes dq, dk, dv (input dtype); step
 // mode adds into the float32 sums dq_acc, dk_acc, dv_acc instead.

@@ -270,6 +270,102 @@ RA_HD Item item_at(const Plan& p, const ItemSpace& s, int BM, int L) {
   return it;
 }
 
+// ---------------------------------------------------------------------------
+// Work items of the CTA-pair kernel: four 128-row query tiles that share every
+// K/V tile, two in each CTA of the pair (tile x = 2*cta + i is tile i of CTA
+// cta; the pair's M = 256 products for tile i span both CTAs' tile i).  The
+// four tiles are four query heads of one kv head at the same rows when the
+// GQA group G is a multiple of 4 (identical masks); two heads of one kv head
+// at two consecutive row tiles (one row tile per CTA) when G is even; else
+// four consecutive row tiles of one head.  qhi is the last valid position
+// over all four tiles, so both CTAs walk the same K/V tiles; a tile whose rows
+// all precede a K/V tile of that walk gets it fully masked.  Ordering as in
+// item_at: head group by head group, longest first.
+// ---------------------------------------------------------------------------
+RA_HD ItemSpace item_space_pair(const Plan& p, int BM) {
+  ItemSpace s;
+  const int G = p.Hq / p.Hkv;
+  s.tq = cdiv(p.C, BM);
+  if (G % 4 == 0) {
+    s.head_pairs = 2;
+    s.per_chunk = s.tq;
+    s.nbh = p.B * p.Hkv * (G / 4);
+  } else if (G % 2 == 0) {
+    s.head_pairs = 1;
+    s.per_chunk = cdiv(s.tq, 2);
+    s.nbh = p.B * p.Hkv * (G / 2);
+  } else {
+    s.head_pairs = 0;
+    s.per_chunk = cdiv(s.tq, 4);
+    s.nbh = p.B * p.Hq;
+  }
+  s.count = s.nbh * p.nqc * s.per_chunk;
+  return s;
+}
+
+// The two tiles of item L that CTA `cta` (0 or 1) of the pair computes.
+RA_HD Item item_pair_at(const Plan& p, const ItemSpace& s, int BM, int L, int cta) {
+  Item it;
+  const int per_bh = p.nqc * s.per_chunk;
+  const int bh = L / per_bh;
+  const int pos_index = L - bh * per_bh;
+  const int slot_rank = pos_index / s.per_chunk;
+  const int within = s.per_chunk - 1 - (pos_index - slot_rank * s.per_chunk);
+  it.qslot = q_slot_by_rank(p, slot_rank);
+  const int G = p.Hq / p.Hkv;
+  int hs[4], ts[4];
+  if (s.head_pairs == 2) {
+    const int per_b = p.Hkv * (G / 4);
+    it.b = bh / per_b;
+    const int r = bh - it.b * per_b;
+    it.hkv = r / (G / 4);
+    const int quad = r - it.hkv * (G / 4);
+    for (int x = 0; x < 4; ++x) {
+      hs[x] = it.hkv * G + 4 * quad + x;
+      ts[x] = within;
+    }
+  } else if (s.head_pairs == 1) {
+    const int per_b = p.Hkv * (G / 2);
+    it.b = bh / per_b;
+    const int r = bh - it.b * per_b;
+    it.hkv = r / (G / 2);
+    const int pair = r - it.hkv * (G / 2);
+    for (int x = 0; x < 4; ++x) {
+      hs[x] = it.hkv * G + 2 * pair + (x & 1);
+      ts[x] = 2 * within + (x >> 1);
+    }
+  } else {
+    it.b = bh / p.Hq;
+    const int h = bh - it.b * p.Hq;
+    it.hkv = h / G;
+    for (int x = 0; x < 4; ++x) {
+      hs[x] = h;
+      ts[x] = 4 * within + x;
+    }
+  }
+  const int cbase_pos = q_pos_base(p, it.qslot);
+  it.qlo = 0x7fffffff;
+  it.qhi = -1;
+  for (int x = 0; x < 4; ++x) {
+    const int off = ts[x] * BM;
+    const int nrows = ts[x] < s.tq ? imin(BM, p.C - off) : 0;
+    if (nrows > 0) {
+      it.qlo = imin(it.qlo, cbase_pos + off);
+      it.qhi = imax(it.qhi, cbase_pos + off + nrows - 1);
+    }
+    if ((x >> 1) == cta) {
+      const int i = x & 1;
+      it.h[i] = hs[x];
+      it.tile_in_chunk[i] = ts[x];
+      it.qoff[i] = off;
+      it.qrow0[i] = buf_row(p, it.qslot, off);
+      it.qpos0[i] = cbase_pos + off;
+      it.nrows[i] = nrows;
+    }
+  }
+  return it;
+}
+
 // Causal class of a tile with valid query positions [q0,q1] and key positions
 // [k0,k1]: 0 full (no mask), 1 partial (mask), 2 skipped.
 RA_HD int tile_class(int causal, int q0, int q1, int k0, int k1) {

@@ -9,6 +9,11 @@
 //   forward        item_at over all items; for both query tiles of an item,
 //                  the K/V tiles of kv_next, with the element mask "key
 //                  position <= query position" and "column < valid keys";
+//   forward pair   item_pair_at over all items of the CTA-pair kernel, for
+//                  both CTAs and both tiles of each, walking the K/V tiles of
+//                  the item's shared qhi with the same element mask (both
+//                  CTAs must agree on the item's chunk, batch, kv head and
+//                  qhi, so they walk the same tiles);
 //   backward K/V   kv_item over all items; the query steps of qstep_next,
 //                  where key row r sees query column j iff k0 + r <= q0 + j
 //                  and j is a valid query of the step;
@@ -39,7 +44,7 @@ using namespace ra;
 
 namespace {
 
-enum { kForward = 0, kBackwardKv = 1, kBackwardQ = 2 };
+enum { kForward = 0, kBackwardKv = 1, kBackwardQ = 2, kForwardPair = 3 };
 
 struct Problem {
   Plan p;
@@ -120,6 +125,63 @@ struct Walk {
           }
       }
       if (n != kv_count(p, it.qslot, it.qhi, BN, tpc)) return fail(12, "kv_count disagrees with kv_next", L, n);
+    }
+    return 0;
+  }
+
+  int forward_pair(int BM, int BN) {
+    owner.assign((size_t)p.B * p.Hq * p.Sq, 0);
+    const ItemSpace sp = item_space_pair(p, BM);
+    const int tpc = cdiv(p.C, BN);
+    const int G = p.Hq / p.Hkv;
+    for (int L = 0; L < sp.count; ++L) {
+      Item its[2] = {item_pair_at(p, sp, BM, L, 0), item_pair_at(p, sp, BM, L, 1)};
+      ++items;
+      if (its[0].b != its[1].b || its[0].hkv != its[1].hkv || its[0].qslot != its[1].qslot ||
+          its[0].qhi != its[1].qhi)
+        return fail(17, "the two CTAs of a pair disagree on the item", L);
+      const Item& it0 = its[0];
+      if (it0.b < 0 || it0.b >= p.B || it0.hkv < 0 || it0.hkv >= p.Hkv) return fail(1, "item batch/kv head out of range", L);
+      if (it0.qslot < 0 || it0.qslot >= p.nqc) return fail(2, "item query chunk out of range", L, it0.qslot);
+      if (it0.qhi < 0) return fail(4, "item without a valid query row", L);
+      for (int c = 0; c < 2; ++c) {
+        const Item& it = its[c];
+        for (int i = 0; i < 2; ++i) {
+          if (it.h[i] < 0 || it.h[i] >= p.Hq || it.h[i] / G != it.hkv)
+            return fail(3, "query head not in the kv group", L, c, i);
+          if (it.nrows[i] < 0 || it.nrows[i] > BM || (it.nrows[i] > 0 && it.qoff[i] + it.nrows[i] > p.C))
+            return fail(4, "query tile rows out of range", L, i, it.nrows[i]);
+          if (it.nrows[i] > 0 && it.qpos0[i] + it.nrows[i] - 1 > it.qhi) return fail(4, "tile beyond qhi", L, c, i);
+          for (int r = 0; r < it.nrows[i]; ++r) {
+            const int row = buf_row(p, it.qslot, it.qoff[i] + r);
+            if (!p.strided && row != it.qrow0[i] + r) return fail(6, "qrow0 disagrees with buf_row", L, i, r);
+            if (int e = own(((size_t)it.b * p.Hq + it.h[i]) * p.Sq + row, L, row)) return e;
+          }
+        }
+      }
+      KvIter iter;
+      kv_begin(p, it0.qslot, iter);
+      KvTile t;
+      int n = 0;
+      while (kv_next(p, it0.qhi, BN, tpc, iter, t)) {
+        ++n;
+        ++steps;
+        if (t.slot < 0 || t.slot >= p.nkc || t.nvalid < 1 || t.nvalid > BN || t.k0 + t.nvalid > p.C)
+          return fail(8, "kv tile out of range", L, t.slot, t.k0);
+        for (int c = 0; c < 2; ++c)
+          for (int i = 0; i < 2; ++i)
+            for (int r = 0; r < its[c].nrows[i]; ++r) {
+              const int qpos = its[c].qpos0[i] + r;
+              for (int k = 0; k < t.nvalid; ++k) {
+                if (p.causal && t.pos0 + k > qpos) continue;           // the kernel's element mask
+                const int krow = buf_row(p, t.slot, t.k0 + k);
+                if (!p.strided && krow != t.row0 + k) return fail(10, "row0 disagrees with buf_row", L, k);
+                if (int e = mark(its[c].b, its[c].h[i], buf_row(p, its[c].qslot, its[c].qoff[i] + r), krow, L))
+                  return e;
+              }
+            }
+      }
+      if (n != kv_count(p, it0.qslot, it0.qhi, BN, tpc)) return fail(12, "kv_count disagrees with kv_next", L, n);
     }
     return 0;
   }
@@ -218,7 +280,10 @@ struct Walk {
 int run(const Problem& pr, int which, int BM, int BN, int64_t* stats, char* msg) {
   msg[0] = 0;
   Walk w(pr, msg);
-  int rc = which == kForward ? w.forward(BM, BN) : which == kBackwardKv ? w.backward_kv() : w.backward_q();
+  int rc = which == kForward       ? w.forward(BM, BN)
+           : which == kForwardPair ? w.forward_pair(BM, BN)
+           : which == kBackwardKv  ? w.backward_kv()
+                                   : w.backward_q();
   if (rc == 0) rc = w.finish();
   stats[0] = w.items;
   stats[1] = w.steps;
@@ -232,7 +297,8 @@ extern "C" {
 
 // Ring mode: the whole sequence of S tokens split into P ranks with `cpr` chunks each
 // (layout 0 contiguous, 1 zig-zag, 2 striped).  which: 0 forward (BM x BN tiles),
-// 1 backward K/V-major, 2 backward Q-major.  stats = {items, steps, pairs}.
+// 1 backward K/V-major, 2 backward Q-major, 3 forward of the CTA-pair kernel.
+// stats = {items, steps, pairs}.
 int sched_cover_ring(int B, int Hq, int Hkv, int S, int P, int layout, int cpr, int causal, int which, int BM,
                      int BN, int64_t* stats, char* msg) {
   Problem pr;

@@ -132,3 +132,39 @@ def test_p_independence():
     for o, l in outs[1:]:
         margin("out", (o - outs[0][0]).abs().max().item(), TOL_BF16_OUT)
         margin("lse", (l - outs[0][1]).abs().max().item(), TOL_BF16_LSE)
+
+
+# D = 128 runs on CTA pairs (tcgen05 cta_group::2) by default; RING_ATTN_TC_KERNEL=single selects
+# the one-CTA kernel.  Both are checked against the oracle on the item shapes the pair kernel
+# forms differently: four heads (group 4), two heads at two row tiles (group 2), four row tiles
+# (group 1 and 3), ragged chunks, the striped split, and the step API.
+BOTH = [
+    W.Prefill("pair_group4_zigzag", "bf16", True, "zigzag", 1, 8, 2, 2048, 128, 4, 131),
+    W.Prefill("pair_group2_ragged", "bf16", True, "zigzag", 2, 4, 2, 1200, 128, 3, 132),
+    W.Prefill("pair_group1_keysx8", "bf16", True, "zigzag", 1, 2, 2, 4096, 128, 4, 133, keys_x8=True),
+    W.Prefill("pair_group3_noncausal", "bf16", False, "contiguous", 1, 6, 2, 1024, 128, 2, 134),
+    W.Prefill("pair_striped_group4", "bf16", True, "striped", 1, 8, 2, 1536, 128, 3, 135),
+    W.Prefill("pair_tail_S200", "bf16", True, "zigzag", 1, 4, 1, 200, 128, 1, 136),
+]
+
+
+@pytest.mark.parametrize("kernel", ["pair", "single"])
+@pytest.mark.parametrize("cfg", BOTH, ids=lambda c: c.name)
+def test_both_tensor_core_kernels_every_row(cfg, kernel, monkeypatch):
+    monkeypatch.setenv("RING_ATTN_TC_KERNEL", kernel)
+    run(cfg, rows=W.sample_rows(cfg, 0))
+
+
+@pytest.mark.parametrize("kernel", ["pair", "single"])
+@pytest.mark.parametrize("layout", ["zigzag", "striped"])
+def test_both_tensor_core_kernels_through_the_step_api(layout, kernel, monkeypatch):
+    monkeypatch.setenv("RING_ATTN_TC_KERNEL", kernel)
+    need_cuda()
+    cfg = W.Prefill("pair_steps", "bf16", True, layout, 1, 8, 2, 1536, 128, 3, 137)
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    out, lse = ring_by_steps(q, k, v, cfg.P, layout, True, cfg.scale)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    rows = W.sample_rows(cfg, 0)
+    ref_out, ref_lse = oracle_rows(q, k, v, rows, cfg.scale, True)
+    check_rows(out, lse, rows, ref_out, ref_lse, TOL_BF16_OUT, TOL_BF16_LSE, f"{kernel} {layout} steps")

@@ -39,7 +39,7 @@ def walker(tmp_path_factory):
     return lib
 
 
-FORWARD, BACKWARD_KV, BACKWARD_Q = 0, 1, 2
+FORWARD, BACKWARD_KV, BACKWARD_Q, FORWARD_PAIR = 0, 1, 2, 3
 
 
 def _ring(lib, B, Hq, Hkv, S, P, layout, cpr, causal, which=FORWARD, BM=128, BN=128):
@@ -61,12 +61,15 @@ for layout, cprs in (("contiguous", (1, 2, 3)), ("zigzag", (2, 3, 4, 8)), ("stri
                 CASES.append((layout, cpr, P, C))
 
 
-@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q])
+@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q, FORWARD_PAIR])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("layout,cpr,P,C", CASES)
 def test_ring_mode_covers_each_allowed_pair_once(walker, layout, cpr, P, C, causal, which):
     S = P * cpr * C
-    for Hq, Hkv in ((2, 1), (3, 3)):             # even group: head pairs; odd group: two row tiles per item
+    # even group: head pairs; odd group: two row tiles per item; the CTA-pair kernel also takes
+    # four heads (group 4), or two heads at two row tiles (group 2), or four row tiles
+    groups = ((2, 1), (3, 3), (4, 1), (8, 2)) if which == FORWARD_PAIR else ((2, 1), (3, 3))
+    for Hq, Hkv in groups:
         stats = _ring(walker, 1, Hq, Hkv, S, P, layout, cpr, causal, which)
         allowed = S * (S + 1) // 2 if causal else S * S
         assert stats[2] == Hq * allowed
@@ -74,9 +77,10 @@ def test_ring_mode_covers_each_allowed_pair_once(walker, layout, cpr, P, C, caus
 
 @pytest.mark.parametrize("BM,BN", [(128, 128), (128, 64), (64, 128)])
 def test_tile_shapes_batches_and_gqa(walker, BM, BN):
-    for (Hq, Hkv) in ((8, 2), (6, 3), (5, 1), (4, 4)):
-        _ring(walker, 2, Hq, Hkv, 4 * 2 * 200, 4, "zigzag", 2, True, FORWARD, BM, BN)
-        _ring(walker, 2, Hq, Hkv, 3 * 130, 3, "striped", 1, True, FORWARD, BM, BN)
+    for (Hq, Hkv) in ((8, 2), (6, 3), (5, 1), (4, 4), (16, 2), (12, 2)):
+        for which in (FORWARD, FORWARD_PAIR):
+            _ring(walker, 2, Hq, Hkv, 4 * 2 * 200, 4, "zigzag", 2, True, which, BM, BN)
+            _ring(walker, 2, Hq, Hkv, 3 * 130, 3, "striped", 1, True, which, BM, BN)
 
 
 def test_backward_batches_and_gqa(walker):
@@ -98,7 +102,7 @@ def _step(lib, C, qid, kid, stripes, causal, Hq=2, Hkv=1, which=FORWARD):
     return stats
 
 
-@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q])
+@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q, FORWARD_PAIR])
 @pytest.mark.parametrize("causal", [True, False])
 def test_step_mode_covers_each_allowed_pair_of_the_held_block_once(walker, causal, which):
     # every (query shard, held block) pair of a zig-zag ring with P = 4 (8 chunks), chunk length 200,
@@ -115,7 +119,7 @@ def test_step_mode_covers_each_allowed_pair_of_the_held_block_once(walker, causa
                 assert st[2] == 2 * expect
 
 
-@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q])
+@pytest.mark.parametrize("which", [FORWARD, BACKWARD_KV, BACKWARD_Q, FORWARD_PAIR])
 def test_step_mode_stripes(walker, which):
     P, C = 5, 150
     for r in range(P):
