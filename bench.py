@@ -422,6 +422,7 @@ def run_ours(args):
                       "ms_per_launch": round(m_ms, 4), "bytes_per_launch": merge_bytes(W.MERGE_ONLY),
                       "roofline": {"bound": "hbm", "achieved": round(m_gbs, 1), "peak": pk["hbm_gbs"],
                                    "unit": "GB/s", "frac": round(m_gbs / pk["hbm_gbs"], 4),
+                                   "traffic": load_traffic().get("merge"),
                                    "kernel": "merge_kernel<bf16>", "peak_kind": f"{pk_kind} HBM copy",
                                    "frac_of_published": round(m_gbs / PUBLISHED["hbm_gbs"], 4)}}
 
@@ -582,6 +583,10 @@ PROFILE_CASES = {
     # S=128k work, q 268 MB (> L2); a small case for full captures
     "tc_gqa": W.Prefill("ring_bf16_causal_zigzag_gqa_B1_Hq32_Hkv8_S32768_D128_P16", "bf16", True, "zigzag",
                         1, 32, 8, 32768, 128, 16, 4),
+    # one kv head (4 query heads) of the S=128k GQA workload: the same K/V per kv head (67 MB) and the
+    # same walk as the timed workload, whose 8 kv heads run one after another; 1/8 of its work
+    "tc_gqa_1head": W.Prefill("ring_bf16_causal_zigzag_gqa_B1_Hq4_Hkv1_S131072_D128_P16", "bf16", True, "zigzag",
+                              1, 4, 1, 131072, 128, 16, 4),
     # the same S=128k GQA workload under the other splits (same FLOPs, different tiles and order)
     "tc_full_contiguous": dataclasses.replace(W.CFG4, layout="contiguous",
                                               name="ring_bf16_causal_contiguous_gqa_B1_Hq32_Hkv8_S131072_D128_P16"),

@@ -85,11 +85,11 @@ def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monk
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(d))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     cur = bench.load_traffic()
-    assert cur["attn_tc"] == d["attn_tc"]["bytes"] and cur["decode"] == d["decode"]["bytes"]
+    assert cur["attn_tc_pair"] == d["attn_tc_pair"]["bytes"] and cur["decode"] == d["decode"]["bytes"]
     f = tmp_path / "context_exact_attention_ring_b200" / "csrc" / "decode.cu"
     f.write_text(f.read_text() + "\n")
     changed = bench.load_traffic()
-    assert changed["decode"] is None and changed["attn_tc"] == cur["attn_tc"]
+    assert changed["decode"] is None and changed["attn_tc_pair"] == cur["attn_tc_pair"]
 
 
 def test_profile_summaries_name_commands_the_bench_accepts():
