@@ -186,24 +186,32 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
             load_tile<D, BR>(p, smem_u32(sm.x[1]), x2, xb, it.g, it.ks, it.k_off, it.b, pol_x);
           }
           __syncwarp();
-          QStepIter si{0, 0, 0};
-          QStep st;
-          while (qstep_next(p, it, si, st)) {
-            // the step's lse (log2 units) and delta, loaded before waiting for a free stage so
-            // that their latency hides behind the wait; columns past the tile get +inf / 0 (P = 0)
-            const size_t base = ((size_t)it.b * p.Hq + st.h) * p.Sq;
-            float l2[BS / 32], dl[BS / 32];
+          // The step's lse (log2 units) and delta feed its elementwise pass.  They are loaded one
+          // step ahead: step i+1's loads are in flight while step i waits for a free stage and
+          // issues its copies.  Columns past the tile get +inf / 0 (P = 0).
+          auto load_ld = [&](const QStep& q, float (&l2)[BS / 32], float (&dl)[BS / 32]) {
+            const size_t base = ((size_t)it.b * p.Hq + q.h) * p.Sq;
 #pragma unroll
             for (int i = 0; i < BS / 32; ++i) {
               const int c = lane + 32 * i;
               l2[i] = CUDART_INF_F;
               dl[i] = 0.f;
-              if (c < st.nq) {
-                const size_t li = base + buf_row(p, st.qs, st.q_off + c);
+              if (c < q.nq) {
+                const size_t li = base + buf_row(p, q.qs, q.q_off + c);
                 l2[i] = __ldg(prm.a.lse + li);
                 dl[i] = __ldg(prm.a.delta + li);
               }
             }
+          };
+          QStepIter si{0, 0, 0};
+          QStep st, st_next;
+          float l2[BS / 32], dl[BS / 32];
+          bool have = qstep_next(p, it, si, st);
+          if (have) load_ld(st, l2, dl);
+          while (have) {
+            float l2n[BS / 32], dln[BS / 32];
+            const bool have_next = qstep_next(p, it, si, st_next);
+            if (have_next) load_ld(st_next, l2n, dln);
             if (!stage_wait(ycnt)) { ok = false; break; }
             const int s = ycnt % NST;
 #pragma unroll
@@ -220,6 +228,15 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
             }
             __syncwarp();
             ++ycnt;
+            have = have_next;
+            if (have) {
+              st = st_next;
+#pragma unroll
+              for (int i = 0; i < BS / 32; ++i) {
+                l2[i] = l2n[i];
+                dl[i] = dln[i];
+              }
+            }
           }
         } else {
           const QItem it = q_item(p, L);
