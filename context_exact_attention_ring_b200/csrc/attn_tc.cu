@@ -53,6 +53,7 @@ template <int D>
 struct TcSmem {
   alignas(1024) uint8_t q[2][tc::BM * D * 2];
   alignas(1024) uint8_t kv[tc::NST][tc::BN * D * 2];
+  alignas(16) float epi[8][tc::kEpiFloats];   // step-mode epilogue staging, one tile per softmax warp
   alignas(8) uint64_t q_full, q_empty, teardown;
   alignas(8) uint64_t kv_full[tc::NST];
   alignas(8) uint64_t kv_empty[tc::NST];
@@ -265,7 +266,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     setmaxnreg_inc<REG_HIGH>();
     // ================================================================ softmax groups
     tc_softmax_role<D, false>(prm, tmem, warp, lane, smem_u32(&sm.s_full[0]), smem_u32(&sm.p_full[0]),
-                              smem_u32(&sm.o_final[0]), abort_flag, blockIdx.x, gridDim.x, 0);
+                              smem_u32(&sm.o_final[0]), abort_flag, blockIdx.x, gridDim.x, 0, sm.epi[warp - 4]);
   }
 
   tc_fence_before();

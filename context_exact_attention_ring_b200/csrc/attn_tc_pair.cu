@@ -58,6 +58,7 @@ constexpr int REG_NEED = (128 * REG_LOW + 256 * tc::REG_HIGH + tc::THREADS - 1) 
 struct TcPairSmem {
   alignas(1024) uint8_t q[2][tcp::Q_BYTES];
   alignas(1024) uint8_t kv[tcp::NST][tcp::STAGE];
+  alignas(16) float epi[8][tc::kEpiFloats];   // step-mode epilogue staging, one tile per softmax warp
   alignas(8) uint64_t q_full, q_empty, teardown, exit_bar;
   alignas(8) uint64_t kv_full[tcp::NST];
   alignas(8) uint64_t kv_empty[tcp::NST];
@@ -314,7 +315,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     setmaxnreg_inc<REG_HIGH>();
     // ================================================================ softmax groups (both CTAs)
     tc_softmax_role<D, true>(prm, tmem, warp, lane, smem_u32(&sm.s_full[0]), mapa_shared(smem_u32(&sm.p_full[0]), 0),
-                             smem_u32(&sm.o_final[0]), abort_flag, PAIR_ITEM0, PAIR_STRIDE, (int)PAIR_CTA);
+                             smem_u32(&sm.o_final[0]), abort_flag, PAIR_ITEM0, PAIR_STRIDE, (int)PAIR_CTA,
+                             sm.epi[warp - 4]);
   }
 
   tc_fence_before();

@@ -35,6 +35,7 @@ constexpr float LAZY = 8.f;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int REG_LOW = 96, REG_HIGH = 184;
 constexpr int REG_NEED = (128 * REG_LOW + 256 * REG_HIGH + THREADS - 1) / THREADS;   // per thread at launch
+constexpr int kEpiFloats = 32 * 16;   // a softmax warp's staging tile: 32 rows x 16 columns
 }  // namespace tc
 
 struct TcParams {
@@ -53,11 +54,13 @@ __device__ __forceinline__ float mergew_exp(float x) { return expf(x); }
 // rescaled).  kPair: the p_full barriers live in the leader CTA and count one
 // arrival per warp of both CTAs (p_full_arrive is their shared::cluster
 // address); otherwise every thread arrives on the local barrier.  Items are
-// L = item0, item0 + stride, ...; `cta` picks the pair item's tiles.
+// L = item0, item0 + stride, ...; `cta` picks the pair item's tiles.  `epi` is
+// this warp's staging tile for the step-mode epilogue (kEpiFloats floats).
 template <int D, bool kPair>
 __device__ __forceinline__ void tc_softmax_role(const TcParams& prm, uint32_t tmem, int warp, int lane,
                                                 uint32_t s_full, uint32_t p_full_arrive, uint32_t o_final,
-                                                volatile int* abort_flag, int item0, int stride, int cta) {
+                                                volatile int* abort_flag, int item0, int stride, int cta,
+                                                float* epi) {
   using namespace tc;
   const Plan& p = prm.p;
   const ItemSpace& space = prm.space;
@@ -250,23 +253,55 @@ __device__ __forceinline__ void tc_softmax_role(const TcParams& prm, uint32_t tm
         w_old = a / l_new;
         w_blk = cb / l_new;
       }
-      float* Orow = prm.a.O + (((size_t)it.b * p.Sq + qr) * p.Hq + h) * D;
+      // The stored O rows are read and written through this warp's 32 x 16 staging tile in shared
+      // memory, 16 columns at a time: four lanes move a row's 64 bytes, so a warp instruction
+      // touches 8 rows instead of one row per lane (32 lines), and the loads of four chunks are
+      // in flight while a chunk is combined.  Tile layout: row r, float4 q at float4
+      // index r*4 + (q ^ ((r >> 1) & 3)), conflict-free for both access patterns.
+      const float wb = w_blk * inv_l;
+      const int rbase = wi * 32;                     // first tile row of this warp
+      const int crow = lane >> 2, cq = lane & 3;     // cooperative pattern: rows crow + 8k, float4 cq
+      float4* const tile = reinterpret_cast<float4*>(epi);
+      auto tidx = [](int r, int q) { return r * 4 + (q ^ ((r >> 1) & 3)); };
+      auto orow = [&](int r) {   // global O row of tile row rbase + r (step mode: rows not strided)
+        return prm.a.O + (((size_t)it.b * p.Sq + it.qrow0[i] + rbase + r) * p.Hq + h) * D;
+      };
+      // four chunks of loads in flight: chunk c + 4 is requested as soon as chunk c is staged
+      constexpr int NCH = D / 16, DEPTH = 4;
+      float4 ld[DEPTH][4];
+      auto load_chunk = [&](int c, float4 (&dst)[4]) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
+        for (int k = 0; k < 4; ++k) {
+          const int r = crow + 8 * k;
+          dst[k] = rbase + r < nrows ? reinterpret_cast<const float4*>(orow(r) + c * 16)[cq]
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      };
+#pragma unroll
+      for (int c = 0; c < DEPTH; ++c) load_chunk(c, ld[c]);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tile[tidx(crow + 8 * k, cq)] = ld[c % DEPTH][k];
+        if (c + DEPTH < NCH) load_chunk(c + DEPTH, ld[c % DEPTH]);
+        uint32_t r16[16];
+        tmem_ld16(tO + c * 16, r16);
         tmem_wait_ld();
-        if (active) {
-          float4* dst = reinterpret_cast<float4*>(Orow + c * 32);
+        __syncwarp();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float4 o = dst[e];
-            o.x = w_old * o.x + w_blk * (__uint_as_float(r[4 * e + 0]) * inv_l);
-            o.y = w_old * o.y + w_blk * (__uint_as_float(r[4 * e + 1]) * inv_l);
-            o.z = w_old * o.z + w_blk * (__uint_as_float(r[4 * e + 2]) * inv_l);
-            o.w = w_old * o.w + w_blk * (__uint_as_float(r[4 * e + 3]) * inv_l);
-            dst[e] = o;
-          }
+        for (int q = 0; q < 4; ++q) {   // this lane's own row
+          float4 o = tile[tidx(lane, q)];
+          o.x = w_old * o.x + wb * __uint_as_float(r16[4 * q + 0]);
+          o.y = w_old * o.y + wb * __uint_as_float(r16[4 * q + 1]);
+          o.z = w_old * o.z + wb * __uint_as_float(r16[4 * q + 2]);
+          o.w = w_old * o.w + wb * __uint_as_float(r16[4 * q + 3]);
+          tile[tidx(lane, q)] = o;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = crow + 8 * k;
+          if (rbase + r < nrows) reinterpret_cast<float4*>(orow(r) + c * 16)[cq] = tile[tidx(r, cq)];
         }
         __syncwarp();
       }
