@@ -435,7 +435,10 @@ ring_status ring_attn_sched_stats(int S, int P, int causal, int layout, int tile
  * in any kernel expired since the last call, RING_ECAPACITY if a KV append
  * dropped a token because its shard was full, RING_ECUDA if the device
  * reports an error, else RING_OK.  `where` (may be NULL) receives the code
- * of the site that recorded the error (0 if none).
+ * of the site that recorded the error (0 if none).  Code 12 (reported as
+ * RING_ETIMEOUT: the kernel unwound without results) means a CTA pair of the
+ * prefill kernel found its cluster ranks numbered otherwise than the blocks
+ * 2c, 2c+1 it assumes.
  * A library helper; the pages have no counterpart.
  */
 ring_status ring_attn_device_error(int* where);
