@@ -98,6 +98,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     tmem_alloc(smem_u32(&sm.tmem_base), TMEM_COLS);
     tmem_relinquish();
   }
+  // step mode: let the next call on the stream start on SMs as this call's CTAs exit; it
+  // waits for this call's completion before it touches the caller's state
+  if (prm.p.mode == kModeStep) grid_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -308,7 +311,19 @@ static cudaError_t launch_tc_d(const Plan& p, const TcArgs& a, cudaStream_t st) 
   if (e != cudaSuccess) return e;
   if (fa.numRegs < tc::REG_NEED) return cudaErrorNotSupported;
   const int grid = prm.space.count < num_sms() ? prm.space.count : num_sms();
-  kern<<<grid, tc::THREADS, smem, st>>>(tq, tk, tv, prm);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  // step mode: may overlap the previous kernel of the stream (see grid_dependency_wait)
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(tc::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.mode == kModeStep ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, prm);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

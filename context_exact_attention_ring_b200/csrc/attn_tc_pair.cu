@@ -117,6 +117,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     tmem_alloc_pair(smem_u32(&sm.tmem_base), TMEM_COLS);
     tmem_relinquish_pair();
   }
+  // step mode: let the next call on the stream start on SMs as this call's CTAs exit; it
+  // waits for this call's completion before it touches the caller's state
+  if (prm.p.mode == kModeStep) grid_launch_dependents();
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();   // both CTAs' barriers are initialised before any copy or arrival reaches them
@@ -370,11 +373,14 @@ cudaError_t launch_attn_tc_pair(const Plan& p, const TcArgs& a, cudaStream_t st)
   if (e != cudaSuccess) return e;
   if (fa.numRegs < tcp::REG_NEED) return cudaErrorNotSupported;   // setmaxnreg.inc could not be met
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // step mode: may overlap the previous kernel of the stream (see grid_dependency_wait)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(tc::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -387,6 +393,7 @@ cudaError_t launch_attn_tc_pair(const Plan& p, const TcArgs& a, cudaStream_t st)
   if (max_clusters < 1) return cudaErrorNotSupported;
   const int clusters = prm.space.count < max_clusters ? prm.space.count : max_clusters;
   cfg.gridDim = dim3(2 * clusters);
+  if (p.mode == kModeStep) cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, prm);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -486,6 +486,18 @@ __device__ __forceinline__ void mma_commit_pair_local(uint32_t bar) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of its stream is still
+// running, once every CTA of that kernel has executed launch_dependents (or
+// exited).  grid_dependency_wait blocks the calling thread until the previous
+// kernel has completed and its memory operations are visible.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // scalar helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float ex2(float x) {

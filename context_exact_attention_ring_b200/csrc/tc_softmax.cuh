@@ -233,7 +233,10 @@ __device__ __forceinline__ void tc_softmax_role(const TcParams& prm, uint32_t tm
         prm.a.lse[((size_t)it.b * p.Hq + h) * p.Sq + qr] =
             l > 0.f ? (m_run + log2f(l)) * 0.6931471805599453f : -CUDART_INF_F;
     } else {
-      // fold this block into the caller's state (natural-log units, exact max)
+      // fold this block into the caller's state (natural-log units, exact max).  The call
+      // before this one on the stream may still be writing the same state rows (step calls
+      // are launched to overlap their predecessor's tail): wait for it to complete first.
+      grid_dependency_wait();
       const size_t si = ((size_t)it.b * p.Hq + h) * p.Sq + (active ? qr : it.qrow0[i]);
       float m_old = -CUDART_INF_F, l_old = 0.f;
       if (active) {

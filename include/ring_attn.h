@@ -167,6 +167,9 @@ ring_status ring_attn_state_init(float* m, float* l, float* O, int B, int Hq, in
  * scores, natural units; l = sum exp(s - m)) and O [B, n_q*C, Hq, D] float,
  * normalised (O = sum exp(s - m) v / l), as in section 3.  Rows whose block
  * has no allowed key keep their state.  Fully masked tiles are skipped.
+ * A bf16 step may begin while the previous kernel on the stream is finishing
+ * (programmatic dependent launch); it reads the state only after that kernel
+ * has completed, so consecutive steps on one stream need no synchronisation.
  *
  * Returns RING_EINVAL for null/misaligned pointers, ids == NULL, n_q or n_kv
  * outside 1..RING_MAX_CHUNKS_PER_RANK, chunk_len < 1, negative chunk ids,
