@@ -600,6 +600,10 @@ PROFILE_CASES = {
     "bwd_full": W.CFG4,
     # backward of the causal zig-zag MHA workload with 1% of keys x8 (a small case for ncu)
     "bwd": W.CFG3,
+    # backward of one kv head (4 query heads) of the S=128k GQA workload: the same walk per kv
+    # head as the timed backward, 1/8 of its work (a small case for ncu)
+    "bwd_gqa_1head": W.Prefill("ring_bf16_causal_zigzag_gqa_B1_Hq4_Hkv1_S131072_D128_P16", "bf16", True, "zigzag",
+                               1, 4, 1, 131072, 128, 16, 4),
     # split-KV decode on 4 x 65536-token sequences (K+V 1.07 GB > L2, lengths U[32k, 64k])
     "decode": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),
     "decode_fused": W.Decode("decode_B4_Hq32_Hkv8_D128_ctx64k_P2", 4, 32, 8, 128, 1 << 16, 2, 5),

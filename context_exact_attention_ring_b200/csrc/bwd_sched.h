@@ -2,11 +2,12 @@
 // header of their own so that the host can walk them as the kernel does.
 //
 // K/V-major launch: an item is a 128-key tile of one kv head; its steps are
-// the 64-row query tiles (of every query head of the group) that the block
-// meets as it travels round the ring ("Lesson 8: Context Parallelism",
-// section 2: the block of rank s meets rank s+t at step t), in that order,
-// skipping under the causal rule ("Lesson 8", section 4) the tiles whose every
-// query precedes every key.  Q-major launch: an item is a 128-row query tile
+// the 64-row query tiles (of every query head of the group) the block meets
+// as it travels round the ring ("Lesson 8: Context Parallelism", section 2:
+// the block of rank s meets every rank once), skipping under the causal rule
+// ("Lesson 8", section 4) the tiles whose every query precedes every key.
+// Inside one GPU the tiles are walked in buffer order, not hop by hop (see
+// qstep_next).  Q-major launch: an item is a 128-row query tile
 // of one head, longest work first; its steps are the K/V tiles of the ring
 // scheduler (ring_sched.h).
 #pragma once
@@ -22,7 +23,7 @@ constexpr int BS = 64;                  // rows of a K/V-major step (query rows)
 // ---------------------------------------------------------------- work items
 // K/V-major item: one 128-key tile of chunk slot ks, kv head g, batch b.
 struct KvItem {
-  int b, g, ks, k_off, nk, srank;
+  int b, g, ks, k_off, nk;
 };
 RA_HD KvItem kv_item(const Plan& p, int L) {
   const int tpk = cdiv(p.C, tb::BR);
@@ -34,7 +35,6 @@ RA_HD KvItem kv_item(const Plan& p, int L) {
   it.ks = r / tpk;
   it.k_off = (r - it.ks * tpk) * tb::BR;
   it.nk = imin(tb::BR, p.C - it.k_off);
-  it.srank = p.mode == kModeRing ? chunk_owner(p, it.ks) : 0;
   return it;
 }
 
@@ -45,24 +45,27 @@ struct QStep {
 struct QStepIter {
   int h, n, qt;
 };
+// The steps of every item follow one path: the Q buffer's chunks in buffer
+// order (ring mode: the sequence in order), their 64-row tiles in order, and
+// the group's query heads innermost; the causal rule skips the tiles whose
+// every query precedes every key.  Items dealt out together hold neighbouring
+// key tiles, so at any time their CTAs are at nearby points of the same path
+// and read the same Q/dO tiles a short time apart.  (Walking each block in its
+// ring order, from its own rank, puts the CTAs of different ranks' blocks on
+// different parts of Q at once; the sums are the same either way.)
 RA_HD bool qstep_next(const Plan& p, const KvItem& it, QStepIter& s, QStep& out) {
   const int G = p.Hq / p.Hkv, tpq = cdiv(p.C, tb::BS);
-  while (s.h < G) {
-    if (s.n >= p.nqc) {
-      s.n = 0;
-      ++s.h;
-      continue;
-    }
+  while (s.n < p.nqc) {
     if (s.qt >= tpq) {
       s.qt = 0;
+      s.h = 0;
       ++s.n;
       continue;
     }
-    // the block of rank srank meets ranks srank, srank+1, ... (ring mode); buffer order (step mode)
-    const int qs = p.mode == kModeRing ? rank_chunk(p, (it.srank + s.n / p.cpr) % p.P, s.n % p.cpr) : s.n;
+    const int qs = s.n;
     const int qb = q_pos_base(p, qs);
     const int k0 = kv_pos_base(p, q_gid(p, qs), it.ks) + it.k_off;
-    if (s.qt == 0 && p.causal) {
+    if (s.qt == 0 && s.h == 0 && p.causal) {
       // tiles whose last query precedes the first key are never met: start at the first one that is
       if (qb + p.C - 1 < k0) {
         s.qt = tpq;
@@ -73,14 +76,21 @@ RA_HD bool qstep_next(const Plan& p, const KvItem& it, QStepIter& s, QStep& out)
     const int q_off = s.qt * tb::BS;
     const int nq = imin(tb::BS, p.C - q_off);
     const int q0 = qb + q_off;
-    ++s.qt;
-    if (p.causal && k0 > q0 + nq - 1) continue;   // every key after every query of the tile
+    if (p.causal && k0 > q0 + nq - 1) {   // every key after every query of the tile
+      ++s.qt;
+      s.h = 0;
+      continue;
+    }
     out.h = it.g * G + s.h;
     out.qs = qs;
     out.q_off = q_off;
     out.nq = nq;
     out.q0 = q0;
     out.k0 = k0;
+    if (++s.h == G) {
+      s.h = 0;
+      ++s.qt;
+    }
     return true;
   }
   return false;
@@ -89,8 +99,7 @@ RA_HD bool qstep_next(const Plan& p, const KvItem& it, QStepIter& s, QStep& out)
 RA_HD int qstep_count(const Plan& p, const KvItem& it) {
   const int G = p.Hq / p.Hkv, tpq = cdiv(p.C, tb::BS);
   int n = 0;
-  for (int c = 0; c < p.nqc; ++c) {
-    const int qs = p.mode == kModeRing ? rank_chunk(p, (it.srank + c / p.cpr) % p.P, c % p.cpr) : c;
+  for (int qs = 0; qs < p.nqc; ++qs) {
     const int qb = q_pos_base(p, qs);
     const int k0 = kv_pos_base(p, q_gid(p, qs), it.ks) + it.k_off;
     if (!p.causal) {
@@ -102,6 +111,22 @@ RA_HD int qstep_count(const Plan& p, const KvItem& it) {
     }
   }
   return n * G;
+}
+
+// The item of a persistent CTA's w-th turn (cta < grid CTAs), or -1 when it
+// has none left.  Turns run through the items in waves of `grid`.  K/V-major
+// items (snake): every other wave is dealt in reverse CTA order.  Neighbouring
+// K/V tiles have nearly equal walks whose lengths fall with the tile's
+// position, so a CTA's items of two consecutive waves add up to about the same
+// work as any other CTA's; the CTAs stay in step and their walks read each
+// Q/dO tile within a short time of one another, while it is still in L2.
+// Dealt in the same order every wave, the CTAs of the later tiles would gain
+// a step on the others with every wave.
+RA_HD int bwd_item_of_turn(int w, int cta, int grid, int items, bool snake) {
+  const long long base = (long long)w * grid;
+  if (base >= items) return -1;
+  const long long L = base + ((snake && (w & 1)) ? grid - 1 - cta : cta);
+  return L < items ? (int)L : -1;
 }
 
 // Q-major item: one 128-row query tile of head h (longest work first).

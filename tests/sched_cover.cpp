@@ -321,6 +321,35 @@ int sched_cover_ring(int B, int Hq, int Hkv, int S, int P, int layout, int cpr, 
   return run(pr, which, BM, BN, stats, msg);
 }
 
+// The backward's dealing of items to persistent CTAs (bwd_item_of_turn): every item of
+// [0, items) goes to exactly one turn of one CTA, each CTA's turns ascend through the waves,
+// and a CTA that has no item in some turn has none in any later turn (the kernels stop at the
+// first -1).  Returns 0, or a code naming the first failure.
+int sched_cover_turns(int items, int grid, int snake, char* msg) {
+  msg[0] = 0;
+  std::vector<int> seen((size_t)items, 0);
+  for (int cta = 0; cta < grid; ++cta) {
+    int last = -1;
+    bool ended = false;
+    for (int w = 0; w <= items / grid + 1; ++w) {
+      const int L = bwd_item_of_turn(w, cta, grid, items, snake != 0);
+      if (L < 0) {
+        ended = true;
+        continue;
+      }
+      if (ended) return snprintf(msg, 256, "cta %d gets item %d after a turn with none", cta, L), 1;
+      if (L >= items) return snprintf(msg, 256, "cta %d gets item %d of %d", cta, L, items), 2;
+      if (L <= last) return snprintf(msg, 256, "cta %d: item %d after %d", cta, L, last), 3;
+      if (L / grid != w) return snprintf(msg, 256, "cta %d: item %d outside wave %d", cta, L, w), 4;
+      last = L;
+      ++seen[(size_t)L];
+    }
+  }
+  for (int L = 0; L < items; ++L)
+    if (seen[(size_t)L] != 1) return snprintf(msg, 256, "item %d dealt %d times", L, seen[(size_t)L]), 5;
+  return 0;
+}
+
 // Step mode: a query shard of nq chunks (global ids qid) against a held block of nk chunks
 // (kid), C tokens each; with stripes = P > 0, one stripe qid[0] against one stripe kid[0].
 int sched_cover_step(int B, int Hq, int Hkv, int C, int nq, const int* qid, int nk, const int* kid, int stripes,

@@ -90,6 +90,18 @@ def test_backward_batches_and_gqa(walker):
             _ring(walker, 2, Hq, Hkv, 3 * 130, 3, "striped", 1, True, which)
 
 
+@pytest.mark.parametrize("snake", [True, False])
+def test_backward_deals_every_item_to_one_cta_turn(walker, snake):
+    walker.sched_cover_turns.argtypes = [ctypes.c_int] * 3 + [ctypes.c_char_p]
+    msg = ctypes.create_string_buffer(256)
+    for grid in (1, 2, 3, 148):
+        for items in (0, 1, grid - 1, grid, grid + 1, 2 * grid, 2 * grid + 5, 7 * grid + 3, 8192):
+            if items < 0:
+                continue
+            rc = walker.sched_cover_turns(items, grid, int(snake), msg)
+            assert rc == 0, (grid, items, rc, msg.value.decode())
+
+
 def _step(lib, C, qid, kid, stripes, causal, Hq=2, Hkv=1, which=FORWARD):
     stats = np.zeros(3, np.int64)
     msg = ctypes.create_string_buffer(256)
