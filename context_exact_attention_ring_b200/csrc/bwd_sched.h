@@ -22,6 +22,13 @@ constexpr int BS = 64;                  // rows of a K/V-major step (query rows)
 
 // ---------------------------------------------------------------- work items
 // K/V-major item: one 128-key tile of chunk slot ks, kv head g, batch b.
+// Items run (batch, kv head) by (batch, kv head); inside one, the key tiles
+// run in buffer order, and in the reverse order for every other one, counted
+// from the last (which thus runs forward).  In ring mode a tile's walk gets
+// shorter with its position, so the items dealt out at one time have nearly
+// equal walks also where one (batch, kv head) ends and the next begins: the
+// short walks at the end of one meet the short walks at the start of the
+// next, and the launch ends with short walks.
 struct KvItem {
   int b, g, ks, k_off, nk;
 };
@@ -29,7 +36,9 @@ RA_HD KvItem kv_item(const Plan& p, int L) {
   const int tpk = cdiv(p.C, tb::BR);
   const int per_bg = p.nkc * tpk;
   KvItem it;
-  const int bg = L / per_bg, r = L - bg * per_bg;
+  const int bg = L / per_bg;
+  int r = L - bg * per_bg;
+  if ((p.B * p.Hkv - 1 - bg) & 1) r = per_bg - 1 - r;
   it.b = bg / p.Hkv;
   it.g = bg - it.b * p.Hkv;
   it.ks = r / tpk;
