@@ -172,8 +172,8 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
         const bool w = mbar_wait(smem_u32(&sm.y_empty[c % NST]), ((c / NST) & 1u) ^ 1u, abort_flag, kWaitKvEmpty, err);
         return __all_sync(0xffffffffu, w);
       };
-      for (int w = 0, L = bwd_item_of_turn(0, blockIdx.x, gridDim.x, prm.items, kKvMajor); L >= 0 && ok;
-           L = bwd_item_of_turn(++w, blockIdx.x, gridDim.x, prm.items, kKvMajor), ++n_items) {
+      for (int w = 0, L = turn_item(0, blockIdx.x, gridDim.x, prm.items, kKvMajor); L >= 0 && ok;
+           L = turn_item(++w, blockIdx.x, gridDim.x, prm.items, kKvMajor), ++n_items) {
         if (n_items > 0) {
           const bool w = mbar_wait(smem_u32(&sm.x_empty), (n_items - 1) & 1u, abort_flag, kWaitQEmpty, err);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
@@ -329,8 +329,8 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
               mma_ts_lo(acc, tsrc + k * 8, bk, hi, idesc_ts);
           }
         };
-        for (int w = 0, L = bwd_item_of_turn(0, blockIdx.x, gridDim.x, prm.items, kKvMajor); L >= 0 && ok;
-             L = bwd_item_of_turn(++w, blockIdx.x, gridDim.x, prm.items, kKvMajor), ++n_items) {
+        for (int w = 0, L = turn_item(0, blockIdx.x, gridDim.x, prm.items, kKvMajor); L >= 0 && ok;
+             L = turn_item(++w, blockIdx.x, gridDim.x, prm.items, kKvMajor), ++n_items) {
           if (!mbar_wait(smem_u32(&sm.x_full), n_items & 1u, abort_flag, kWaitQFull, err)) { ok = false; break; }
           tc_fence_after();
           int n;
@@ -486,8 +486,8 @@ __global__ void __launch_bounds__(tb::THREADS, 1)
       return true;
     };
 
-    for (int w = 0, L = bwd_item_of_turn(0, blockIdx.x, gridDim.x, prm.items, kKvMajor); L >= 0 && ok;
-         L = bwd_item_of_turn(++w, blockIdx.x, gridDim.x, prm.items, kKvMajor), ++n_items) {
+    for (int w = 0, L = turn_item(0, blockIdx.x, gridDim.x, prm.items, kKvMajor); L >= 0 && ok;
+         L = turn_item(++w, blockIdx.x, gridDim.x, prm.items, kKvMajor), ++n_items) {
       int nsteps = 0;
       if constexpr (kKvMajor) {
         const KvItem it = kv_item(p, L);

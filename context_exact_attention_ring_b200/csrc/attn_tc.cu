@@ -123,7 +123,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const int tpc = cdiv(p.C, BN);
       uint32_t kv_cnt = 0, n_items = 0;
       bool ok = true;
-      for (int L = blockIdx.x; L < space.count && ok; L += gridDim.x, ++n_items) {
+      for (int w = 0, L = turn_item(0, blockIdx.x, gridDim.x, space.count, true); L >= 0 && ok;
+             L = turn_item(++w, blockIdx.x, gridDim.x, space.count, true), ++n_items) {
         const Item it = item_at(p, space, BM, L);
         if (n_items > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n_items - 1) & 1u, abort_flag, kWaitQEmpty, err)) {
           ok = false;
@@ -205,7 +206,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         return mbar_wait(smem_u32(&sm.kv_full[c % NST]), (c / NST) & 1u, abort_flag, kWaitKvFull, err);
       };
 
-      for (int L = blockIdx.x; L < space.count && ok; L += gridDim.x, ++n_items) {
+      for (int w = 0, L = turn_item(0, blockIdx.x, gridDim.x, space.count, true); L >= 0 && ok;
+             L = turn_item(++w, blockIdx.x, gridDim.x, space.count, true), ++n_items) {
         const Item it = item_at(p, space, BM, L);
         const int n = kv_count(p, it.qslot, it.qhi, BN, tpc);
         if (!mbar_wait(smem_u32(&sm.q_full), n_items & 1u, abort_flag, kWaitQFull, err)) { ok = false; break; }

@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const int tpc = cdiv(p.C, BN);
         uint32_t kv_cnt = 0, n_items = 0;
         bool ok = true;
-        for (int L = PAIR_ITEM0; L < space.count && ok; L += PAIR_STRIDE, ++n_items) {
+        for (int w = 0, L = turn_item(0, PAIR_ITEM0, PAIR_STRIDE, space.count, false); L >= 0 && ok;
+             L = turn_item(++w, PAIR_ITEM0, PAIR_STRIDE, space.count, false), ++n_items) {
           const Item it = item_pair_at(p, space, BM, L, (int)cta);
           if (n_items > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n_items - 1) & 1u, abort_flag, kWaitQEmpty, err)) {
             ok = false;
@@ -243,7 +244,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           return mbar_wait(smem_u32(&sm.p_full[i]), parity, abort_flag, kWaitPFull, err);
         };
         // the producer fills the stages in the order K_0, V_0, K_1, V_1, ... (one count kv_cnt)
-        for (int L = PAIR_ITEM0; L < space.count && ok; L += PAIR_STRIDE, ++n_items) {
+        for (int w = 0, L = turn_item(0, PAIR_ITEM0, PAIR_STRIDE, space.count, false); L >= 0 && ok;
+             L = turn_item(++w, PAIR_ITEM0, PAIR_STRIDE, space.count, false), ++n_items) {
           const Item it = item_pair_at(p, space, BM, L, 0);
           const int n = kv_count(p, it.qslot, it.qhi, BN, tpc);
           if (!mbar_wait(smem_u32(&sm.q_full), n_items & 1u, abort_flag, kWaitQFull, err)) {

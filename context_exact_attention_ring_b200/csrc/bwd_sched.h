@@ -122,22 +122,6 @@ RA_HD int qstep_count(const Plan& p, const KvItem& it) {
   return n * G;
 }
 
-// The item of a persistent CTA's w-th turn (cta < grid CTAs), or -1 when it
-// has none left.  Turns run through the items in waves of `grid`.  K/V-major
-// items (snake): every other wave is dealt in reverse CTA order.  Neighbouring
-// K/V tiles have nearly equal walks whose lengths fall with the tile's
-// position, so a CTA's items of two consecutive waves add up to about the same
-// work as any other CTA's; the CTAs stay in step and their walks read each
-// Q/dO tile within a short time of one another, while it is still in L2.
-// Dealt in the same order every wave, the CTAs of the later tiles would gain
-// a step on the others with every wave.
-RA_HD int bwd_item_of_turn(int w, int cta, int grid, int items, bool snake) {
-  const long long base = (long long)w * grid;
-  if (base >= items) return -1;
-  const long long L = base + ((snake && (w & 1)) ? grid - 1 - cta : cta);
-  return L < items ? (int)L : -1;
-}
-
 // Q-major item: one 128-row query tile of head h (longest work first).
 struct QItem {
   int b, h, g, qs, q_off, nq, q0;

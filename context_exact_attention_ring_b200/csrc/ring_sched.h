@@ -223,8 +223,10 @@ RA_HD ItemSpace item_space(const Plan& p, int BM) {
 // Items are ordered head group by head group, and inside one head group by
 // decreasing query position.  A wave of concurrently running CTAs therefore
 // streams the K/V of a single kv head (which stays resident in L2), and the
-// persistent CTAs, which take items with a stride of the grid size, each get
-// an even spread of long and short items; the shortest come last.
+// persistent CTAs, which take the items in waves of the grid size (turn_item;
+// the one-CTA kernel deals every other wave in reverse, the CTA-pair kernel
+// in the same order every wave, each measured the faster for it), each get an
+// even spread of long and short items; the shortest come last.
 RA_HD Item item_at(const Plan& p, const ItemSpace& s, int BM, int L) {
   Item it;
   const int per_bh = p.nqc * s.per_chunk;
@@ -364,6 +366,24 @@ RA_HD Item item_pair_at(const Plan& p, const ItemSpace& s, int BM, int L, int ct
     }
   }
   return it;
+}
+
+// The item of a persistent CTA's w-th turn (cta < grid CTAs or CTA pairs), or
+// -1 when it has none left.  Turns run through the items in waves of `grid`;
+// with `snake`, every other wave is dealt in reverse order.  The kernels'
+// items are ordered so that neighbouring items have nearly equal work, and
+// that work falls along the order (longest first); dealt in the same order
+// every wave, the CTAs given the later items of each wave would gain on the
+// others with every wave, and the CTAs would drift apart over the launch.  In
+// reverse every other wave, a CTA's items of two consecutive waves add up to
+// about the same work as any other CTA's, so the CTAs stay in step and read
+// the same K/V (or Q/dO) tiles within a short time of one another, while they
+// are still in L2.
+RA_HD int turn_item(int w, int cta, int grid, int items, bool snake) {
+  const long long base = (long long)w * grid;
+  if (base >= items) return -1;
+  const long long L = base + ((snake && (w & 1)) ? grid - 1 - cta : cta);
+  return L < items ? (int)L : -1;
 }
 
 // Causal class of a tile with valid query positions [q0,q1] and key positions

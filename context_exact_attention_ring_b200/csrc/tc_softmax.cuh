@@ -54,8 +54,9 @@ __device__ __forceinline__ float mergew_exp(float x) { return expf(x); }
 // rescaled).  kPair: the p_full barriers live in the leader CTA and count one
 // arrival per warp of both CTAs (p_full_arrive is their shared::cluster
 // address); otherwise every thread arrives on the local barrier.  Items are
-// L = item0, item0 + stride, ...; `cta` picks the pair item's tiles.  `epi` is
-// this warp's staging tile for the step-mode epilogue (kEpiFloats floats).
+// dealt to CTA (or pair) item0 of `stride` by turn_item, in alternating wave
+// order for one CTA per SM only; `cta` picks the pair item's tiles.  `epi` is this warp's staging tile for the step-mode epilogue
+// (kEpiFloats floats).
 template <int D, bool kPair>
 __device__ __forceinline__ void tc_softmax_role(const TcParams& prm, uint32_t tmem, int warp, int lane,
                                                 uint32_t s_full, uint32_t p_full_arrive, uint32_t o_final,
@@ -77,7 +78,10 @@ __device__ __forceinline__ void tc_softmax_role(const TcParams& prm, uint32_t tm
   unsigned long long cnt_full = 0, cnt_part = 0;
   bool ok = true;
 
-  for (int L = item0; L < space.count && ok; L += stride) {
+  // items dealt as in the role's kernel: in alternating wave order on one CTA per SM, in
+  // the same order every wave on CTA pairs (measured faster for each)
+  for (int w = 0, L = turn_item(0, item0, stride, space.count, !kPair); L >= 0 && ok;
+       L = turn_item(++w, item0, stride, space.count, !kPair)) {
     const Item it = kPair ? item_pair_at(p, space, BM, L, cta) : item_at(p, space, BM, L);
     const int nrows = it.nrows[i];
     const int q0 = it.qpos0[i], q1 = it.qpos0[i] + nrows - 1;

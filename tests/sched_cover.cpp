@@ -321,7 +321,7 @@ int sched_cover_ring(int B, int Hq, int Hkv, int S, int P, int layout, int cpr, 
   return run(pr, which, BM, BN, stats, msg);
 }
 
-// The backward's dealing of items to persistent CTAs (bwd_item_of_turn): every item of
+// The dealing of work items to persistent CTAs (turn_item, used by the forward and backward kernels): every item of
 // [0, items) goes to exactly one turn of one CTA, each CTA's turns ascend through the waves,
 // and a CTA that has no item in some turn has none in any later turn (the kernels stop at the
 // first -1).  Returns 0, or a code naming the first failure.
@@ -332,7 +332,7 @@ int sched_cover_turns(int items, int grid, int snake, char* msg) {
     int last = -1;
     bool ended = false;
     for (int w = 0; w <= items / grid + 1; ++w) {
-      const int L = bwd_item_of_turn(w, cta, grid, items, snake != 0);
+      const int L = turn_item(w, cta, grid, items, snake != 0);
       if (L < 0) {
         ended = true;
         continue;
