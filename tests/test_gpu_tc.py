@@ -1,8 +1,10 @@
 """GPU parity of the tensor-core (tcgen05) ring attention against the fp64
 oracle: small shapes on every row, the full-size workloads on the rows the
 oracle can afford (every row of the contiguous S=8192 workload; 256 sampled
-rows per head at S=32768 and S=131072), device work counters against the
-oracle's schedule enumeration, the step API, and the SIMT cross-check."""
+rows per head at S=32768 and S=131072), the S=131072 workload through the
+step API (sampled rows against the oracle, every row against the fused
+ring), device work counters against the oracle's schedule enumeration, and
+the SIMT cross-check."""
 import dataclasses
 
 import numpy as np
@@ -70,6 +72,24 @@ def test_cfg3_full_size_sampled():
 def test_cfg4_full_size_sampled():
     # causal zig-zag GQA, B1 Hq32 Hkv8 S131072 D128 P16: the timed workload
     run(W.CFG4)
+
+
+def test_cfg4_full_size_through_the_step_api():
+    # the timed workload as 16 ranks x 16 hops of ring_attn_step (state in HBM): sampled rows
+    # against the oracle, and every row against the fused ring of the same inputs
+    need_cuda()
+    cfg = W.CFG4
+    q, k, v = W.prefill_inputs(cfg, "cuda")
+    out, lse = ring_by_steps(q, k, v, cfg.P, cfg.layout, cfg.causal, cfg.scale)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_device_error()[0] == ra.RING_OK
+    rows = W.sample_rows(cfg, 2)
+    ref_out, ref_lse = oracle_rows(q, k, v, rows, cfg.scale, cfg.causal)
+    check_rows(out, lse, rows, ref_out, ref_lse, TOL_BF16_OUT, TOL_BF16_LSE, "steps")
+    fo, fl = ra.ring_attn_fwd(q, k, v, cfg.P, causal=True, layout=cfg.layout, scale=cfg.scale)
+    torch.cuda.synchronize()
+    margin("out", (out.float() - fo.float()).abs().max().item(), TOL_BF16_OUT, "steps vs fused, every row")
+    margin("lse", (lse - fl).abs().max().item(), TOL_BF16_LSE, "steps vs fused, every row")
 
 
 @pytest.mark.parametrize("cfg", [W.CFG2, W.CFG3, W.CFG4,
