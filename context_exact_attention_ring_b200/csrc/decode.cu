@@ -110,12 +110,13 @@ __device__ __forceinline__ bool count_chunk(const DecodeArgs& a, const DecodeExt
 // visible here).  The update of "Lesson 8: Context Parallelism", section 3,
 // applied to whole partial states:
 //   lse = m* + ln sum_p e^(lse_p - m*),  out = sum_p e^(lse_p - lse) O_p.
+// Heads h0 .. h0 + G - 1 of the group (query heads (b, g * Gq + h0 + i)); the
+// group is merged in passes of at most 8 heads, so that the per-head values of
+// a pass stay in registers (16 heads at once spilled).
 template <int G, int DH>
-__device__ __noinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
+__device__ __noinline__ void merge_heads(const DecodeArgs& a, const DecodeExtra& x, size_t bh0, int lane) {
   constexpr int D = DH;
-  __syncwarp();   // lane 0's acquire covers the warp from here on
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(x.out);
-  const size_t bh0 = (size_t)b * a.Hq + g * G;
   // lse of chunk (q0 + lane) of every head; the first 32 chunks stay in registers
   auto lse_at = [&](int h, int q) { return q < a.P ? __ldcg(a.part_lse + (bh0 + h) * a.P + q) : -CUDART_INF_F; };
   float lv[G], mx[G], L[G];
@@ -174,6 +175,13 @@ __device__ __noinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x,
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int k = 0; k < D / 32; ++k) out[(bh0 + h) * D + lane + 32 * k] = __float2bfloat16_rn(acc[h][k]);
+}
+
+template <int G, int DH>
+__device__ __forceinline__ void merge_bg(const DecodeArgs& a, const DecodeExtra& x, int b, int g, int lane) {
+  constexpr int GP = G > 8 ? 8 : G;   // heads per pass
+  __syncwarp();   // lane 0's acquire covers the warp from here on
+  for (int h0 = 0; h0 < G; h0 += GP) merge_heads<GP, DH>(a, x, (size_t)b * a.Hq + g * G + h0, lane);
 }
 
 // Called by the merge warp (all lanes) for a chunk whose final partial this CTA

@@ -109,7 +109,7 @@ def test_decode_ignores_rows_past_the_length(fused):
         margin("out", np.max(np.abs(host(out)[b, h] - ro)), TOL_BF16_OUT)
 
 
-@pytest.mark.parametrize("Hq,Hkv,P", [(8, 2, 3), (16, 2, 1)])
+@pytest.mark.parametrize("Hq,Hkv,P", [(8, 2, 3), (16, 2, 1), (16, 1, 2)])   # G = 4, 8, 16
 @pytest.mark.parametrize("fused", [False, True])
 def test_decode_head_dim_64(Hq, Hkv, P, fused):
     # D = 64: one 64-column block per K/V row; with P = 1 the 24576-row chunk spans 3 sub-splits
