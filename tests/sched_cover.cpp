@@ -350,6 +350,9 @@ int sched_cover_turns(int items, int grid, int snake, char* msg) {
   return 0;
 }
 
+// The item a CTA takes at its w-th turn (-1 when it has none), as the kernels deal them.
+int sched_turn_item(int w, int cta, int grid, int items, int snake) { return turn_item(w, cta, grid, items, snake != 0); }
+
 // Step mode: a query shard of nq chunks (global ids qid) against a held block of nk chunks
 // (kid), C tokens each; with stripes = P > 0, one stripe qid[0] against one stripe kid[0].
 int sched_cover_step(int B, int Hq, int Hkv, int C, int nq, const int* qid, int nk, const int* kid, int stripes,

@@ -102,6 +102,29 @@ def test_backward_deals_every_item_to_one_cta_turn(walker, snake):
             assert rc == 0, (grid, items, rc, msg.value.decode())
 
 
+def test_alternating_waves_keep_the_ctas_in_step(walker):
+    # Items ordered longest first with work falling linearly along the order (the kernels'
+    # orders): dealt in alternating wave order, the work a CTA has done after every second wave
+    # differs from any other CTA's by at most one wave's spread of item lengths; dealt in the
+    # same order every wave, the spread grows with every wave.
+    walker.sched_turn_item.argtypes = [ctypes.c_int] * 5
+    grid, items = 148, 148 * 40
+    work = lambda L: 10_000 - L   # falls by one unit per item
+    spread = {}
+    for snake in (True, False):
+        done = np.zeros(grid)
+        worst = 0.0
+        for w in range(items // grid):
+            for c in range(grid):
+                L = walker.sched_turn_item(w, c, grid, items, int(snake))
+                done[c] += work(L)
+            if w % 2 == 1:
+                worst = max(worst, done.max() - done.min())
+        spread[snake] = worst
+    assert spread[True] <= grid - 1                    # one wave's spread at most
+    assert spread[False] >= 20 * (grid - 1)            # 40 waves of the same spread, added up
+
+
 def _step(lib, C, qid, kid, stripes, causal, Hq=2, Hkv=1, which=FORWARD):
     stats = np.zeros(3, np.int64)
     msg = ctypes.create_string_buffer(256)
