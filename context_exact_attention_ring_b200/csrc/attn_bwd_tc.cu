@@ -8,7 +8,9 @@
 //   kKvMajor = true   a work item is a 128-key K/V tile of one kv head; its
 //                     steps are the 64-row query tiles (of every query head
 //                     of the group) that the block meets as it travels round
-//                     the ring ("Lesson 8: Context Parallelism", section 2):
+//                     the ring ("Lesson 8: Context Parallelism", section 2),
+//                     walked in buffer order with the heads innermost
+//                     (bwd_sched.h):
 //                       T1 = K Q^T, T2 = V dO^T      (SS: K, V, Q, dO in smem)
 //                       P^T, dS^T from T1, T2          (two elementwise groups)
 //                       dV += P^T dO, dK += dS^T Q    (TS: P^T, dS^T in tmem)

@@ -7,9 +7,9 @@
 // the block of rank s meets every rank once), skipping under the causal rule
 // ("Lesson 8", section 4) the tiles whose every query precedes every key.
 // Inside one GPU the tiles are walked in buffer order, not hop by hop (see
-// qstep_next).  Q-major launch: an item is a 128-row query tile
-// of one head, longest work first; its steps are the K/V tiles of the ring
-// scheduler (ring_sched.h).
+// qstep_next).  Q-major launch: an item is a 128-row query tile of one head,
+// longest work first; its steps are the K/V tiles of the ring scheduler
+// (ring_sched.h).
 #pragma once
 #include "ring_sched.h"
 
